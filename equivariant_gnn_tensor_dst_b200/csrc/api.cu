@@ -1,0 +1,712 @@
+// C ABI of the tensor-product convolution: plan builder, workspace layout and the
+// launch sequences of the forward, backward and double backward passes.
+//
+// Plan (Sobek, section 2, eqs. 3-5 and 9-10; section 4 on the generator's input):
+// irreps strings are parsed into blocks, valid paths are enumerated in the fixed order
+// (input block, harmonic order, output block), and every path is mapped to a
+// compile-time (l_in, l_sh, l_out) kernel specialisation whose coupling
+// coefficients are constants of the generated table.  Unlike the pages' generator,
+// nothing is compiled at run time: all 34 order triples with l <= 3 are built ahead
+// of time and selected per path.
+//
+// Pass structure (section 4): receiver ranges bounded by the scratch budget are
+// streamed through a receiver traversal that builds the bounded state S (eq. 33),
+// then channel contractions apply A (eqs. 34-36); the source-CSR traversal owns
+// x_bar with the mirrored state X, and the position gradient is assembled from
+// per-edge values in a fixed order.
+#include <algorithm>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+#include <cmath>
+
+#include "../../include/tpconv.h"
+#include "internal.h"
+#include "tables.inc"
+
+using namespace tpc;
+
+namespace {
+
+struct Block {
+  int mul, l, parity, offset;
+};
+
+struct PathH {
+  int l_in, l_sh, l_out, b_in, b_out, c_in, c_out, w_off, w_count, type, nnz;
+  int in_off, out_off, st_off, xst_off;
+};
+
+constexpr size_t kDefaultBudget = size_t(128) << 20;  // the pages' 128 MiB scratch cap
+constexpr int kSplitsMax = 32;
+constexpr int kUvuRanges = 64;
+
+int triple_index(int a, int b, int c) {
+  for (int t = 0; t < tpc_tab::NTRIPLES; ++t)
+    if (tpc_tab::TRIPLES[t][0] == a && tpc_tab::TRIPLES[t][1] == b && tpc_tab::TRIPLES[t][2] == c) return t;
+  return -1;
+}
+
+// host access to the generated coupling tables
+template <int A, int B, int C>
+void cg_host(std::vector<int>& idx, std::vector<double>& val) {
+  using T = tpc_tab::CG<A, B, C>;
+  for (int n = 0; n < T::nnz; ++n) {
+    idx.push_back(T::mi(n));
+    idx.push_back(T::my(n));
+    idx.push_back(T::mo(n));
+    val.push_back(T::val_d(n));
+  }
+}
+
+#define TPC_HCASE(n)                                                                        \
+  case n:                                                                                   \
+    cg_host<tpc_tab::TRIPLES[n][0], tpc_tab::TRIPLES[n][1], tpc_tab::TRIPLES[n][2]>(idx, val); \
+    break;
+
+void cg_of_type(int type, std::vector<int>& idx, std::vector<double>& val) {
+  switch (type) {
+    TPC_HCASE(0) TPC_HCASE(1) TPC_HCASE(2) TPC_HCASE(3) TPC_HCASE(4) TPC_HCASE(5) TPC_HCASE(6)
+    TPC_HCASE(7) TPC_HCASE(8) TPC_HCASE(9) TPC_HCASE(10) TPC_HCASE(11) TPC_HCASE(12)
+    TPC_HCASE(13) TPC_HCASE(14) TPC_HCASE(15) TPC_HCASE(16) TPC_HCASE(17) TPC_HCASE(18)
+    TPC_HCASE(19) TPC_HCASE(20) TPC_HCASE(21) TPC_HCASE(22) TPC_HCASE(23) TPC_HCASE(24)
+    TPC_HCASE(25) TPC_HCASE(26) TPC_HCASE(27) TPC_HCASE(28) TPC_HCASE(29) TPC_HCASE(30)
+    TPC_HCASE(31) TPC_HCASE(32) TPC_HCASE(33)
+    default: break;
+  }
+}
+
+tpconv_status parse_irreps(const char* s, std::vector<Block>& out) {
+  if (!s) return TPCONV_ERR_INVALID_ARG;
+  out.clear();
+  std::string str(s);
+  size_t pos = 0;
+  int off = 0;
+  if (str.find_first_not_of(" \t") == std::string::npos) return TPCONV_ERR_PARSE;
+  while (pos <= str.size()) {
+    size_t plus = str.find('+', pos);
+    std::string tok = str.substr(pos, plus == std::string::npos ? std::string::npos : plus - pos);
+    std::string t;
+    for (char ch : tok) if (ch != ' ' && ch != '\t') t.push_back(ch);
+    if (t.empty()) return TPCONV_ERR_PARSE;
+    long mul = 1;
+    size_t xp = t.find('x');
+    std::string lp = t;
+    if (xp != std::string::npos) {
+      std::string ms = t.substr(0, xp);
+      if (ms.empty() || ms.find_first_not_of("0123456789") != std::string::npos || ms.size() > 6) return TPCONV_ERR_PARSE;
+      mul = std::atol(ms.c_str());
+      lp = t.substr(xp + 1);
+    }
+    if (lp.size() < 2) return TPCONV_ERR_PARSE;
+    char par = lp.back();
+    std::string ls = lp.substr(0, lp.size() - 1);
+    if ((par != 'e' && par != 'o') || ls.empty() || ls.find_first_not_of("0123456789") != std::string::npos || ls.size() > 3)
+      return TPCONV_ERR_PARSE;
+    long l = std::atol(ls.c_str());
+    if (mul <= 0) return TPCONV_ERR_PARSE;
+    if (l > TPC_LMAX) return TPCONV_ERR_UNSUPPORTED;
+    Block b{(int)mul, (int)l, par == 'e' ? 1 : -1, off};
+    off += b.mul * (2 * b.l + 1);
+    out.push_back(b);
+    if (plus == std::string::npos) break;
+    pos = plus + 1;
+  }
+  if ((int)out.size() > MAX_BLOCKS) return TPCONV_ERR_UNSUPPORTED;
+  return TPCONV_OK;
+}
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+}  // namespace
+
+struct tpconv_plan {
+  std::vector<Block> in, out;
+  int lmax = 0, mode = 0;
+  tpconv_radial_spec radial{};
+  std::vector<PathH> paths;
+  std::vector<std::vector<int>> cg_idx;
+  std::vector<std::vector<double>> cg_val;
+  int dim_in = 0, dim_out = 0, n_w = 0, K = 0;
+  DevPlan dev{};
+  Tasks t_in{};   // (path, 32-chunk of C_in)
+  Tasks t_out{};  // (path, 32-chunk of C_out)
+  Tasks t_bo{};   // (output block, chunk)  uvu forward
+  Tasks t_bi{};   // (input block, chunk)   uvu source pass
+  BlockPaths bp_out{}, bp_in{};
+  size_t budget = kDefaultBudget;
+  long long max_mn_tn_bwd = 0;  // max over paths of C_in * K * C_out
+};
+
+namespace {
+
+struct Layout {
+  int recv_chunk = 0, src_chunk = 0;
+  size_t state_a = 0, state_b = 0;  // offsets of the (up to two) state arrays
+  size_t gbuf = 0, part = 0;
+  size_t total = 0;
+  bool has_gbuf = false, has_part = false;
+};
+
+int chunk_nodes(size_t budget, long long per_node_floats, int arrays, long long N) {
+  if (per_node_floats <= 0 || N <= 0) return (int)std::max<long long>(N, 0);
+  long long c = (long long)(budget / (size_t(4) * per_node_floats * arrays));
+  c = std::max<long long>(1, std::min<long long>(c, N));
+  return (int)c;
+}
+
+Layout make_layout(const tpconv_plan* P, long long N, long long E, uint32_t pass) {
+  Layout L;
+  size_t off = 0;
+  const long long st = P->dev.state_per_node, xs = P->dev.xstate_per_node;
+  if (P->mode == TPCONV_UVW) {
+    int arrays = (pass == TPCONV_PASS_DOUBLE_BACKWARD) ? 2 : 1;
+    L.recv_chunk = chunk_nodes(P->budget, st, arrays, N);
+    L.src_chunk = chunk_nodes(P->budget, xs, arrays, N);
+    size_t one = 0;
+    if (pass == TPCONV_PASS_FORWARD) {
+      one = align256(size_t(4) * L.recv_chunk * st);
+    } else {
+      one = std::max(align256(size_t(4) * L.recv_chunk * st), align256(size_t(4) * L.src_chunk * xs));
+    }
+    L.state_a = off;
+    off += one;
+    if (arrays == 2) { L.state_b = off; off += one; }
+    if (pass != TPCONV_PASS_FORWARD) {
+      L.has_part = true;
+      L.part = off;
+      off += align256(size_t(4) * kSplitsMax * P->max_mn_tn_bwd);
+    }
+  } else {
+    if (pass != TPCONV_PASS_FORWARD) {
+      L.has_part = true;
+      L.part = off;
+      off += align256(size_t(4) * kUvuRanges * P->K * (long long)P->n_w);
+    }
+  }
+  if (pass == TPCONV_PASS_BACKWARD) {
+    L.has_gbuf = true;
+    L.gbuf = off;
+    off += align256(size_t(16) * std::max<long long>(E, 1));
+  }
+  L.total = off;
+  return L;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int splits_for(long long kc) {
+  long long s = kc / 256;
+  return (int)std::max<long long>(1, std::min<long long>(kSplitsMax, s));
+}
+
+GemmArgs gemm_base() {
+  GemmArgs g{};
+  g.splits = 1;
+  return g;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+
+extern "C" {
+
+const char* tpconv_status_string(tpconv_status s) {
+  switch (s) {
+    case TPCONV_OK: return "ok";
+    case TPCONV_ERR_INVALID_ARG: return "invalid argument";
+    case TPCONV_ERR_PARSE: return "irreps parse error";
+    case TPCONV_ERR_UNSUPPORTED: return "unsupported configuration";
+    case TPCONV_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case TPCONV_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case TPCONV_ERR_CUDA: return "CUDA error";
+    case TPCONV_ERR_GRAPH_INVALID: return "invalid graph";
+  }
+  return "unknown status";
+}
+
+tpconv_status tpconv_plan_create(tpconv_plan_t* out, const char* irreps_in, int32_t sh_lmax,
+                                 const char* irreps_out, int32_t mode,
+                                 const tpconv_radial_spec* radial) {
+  if (!out || !irreps_in || !irreps_out || !radial) return TPCONV_ERR_INVALID_ARG;
+  if (mode != TPCONV_UVW && mode != TPCONV_UVU) return TPCONV_ERR_INVALID_ARG;
+  if (sh_lmax < 0) return TPCONV_ERR_INVALID_ARG;
+  if (sh_lmax > TPC_LMAX) return TPCONV_ERR_UNSUPPORTED;
+  const tpconv_radial_spec& R = *radial;
+  if (R.num_basis < 1) return TPCONV_ERR_INVALID_ARG;
+  if (R.num_basis > 16) return TPCONV_ERR_UNSUPPORTED;
+  if (!(R.r_cut > 0.f) || R.poly_p < 1 || R.poly_p > 32) return TPCONV_ERR_INVALID_ARG;
+  if (R.kind != TPCONV_RADIAL_BESSEL && R.kind != TPCONV_RADIAL_GAUSSIAN) return TPCONV_ERR_INVALID_ARG;
+  if (R.kind == TPCONV_RADIAL_GAUSSIAN && (R.num_basis < 2 || !(R.r_max > R.r_min)))
+    return TPCONV_ERR_INVALID_ARG;
+
+  tpconv_plan* P = new (std::nothrow) tpconv_plan();
+  if (!P) return TPCONV_ERR_INVALID_ARG;
+  tpconv_status st = parse_irreps(irreps_in, P->in);
+  if (st == TPCONV_OK) st = parse_irreps(irreps_out, P->out);
+  if (st != TPCONV_OK) { delete P; return st; }
+  P->lmax = sh_lmax;
+  P->mode = mode;
+  P->radial = R;
+  P->K = R.num_basis;
+  for (const Block& b : P->in) P->dim_in += b.mul * (2 * b.l + 1);
+  for (const Block& b : P->out) P->dim_out += b.mul * (2 * b.l + 1);
+
+  // eq. 5 path enumeration in the fixed order
+  int woff = 0, st_off = 0, xst_off = 0;
+  for (int bi = 0; bi < (int)P->in.size(); ++bi)
+    for (int ls = 0; ls <= sh_lmax; ++ls)
+      for (int bo = 0; bo < (int)P->out.size(); ++bo) {
+        const Block &a = P->in[bi], &c = P->out[bo];
+        const int psh = (ls % 2 == 0) ? 1 : -1;
+        if (!(std::abs(a.l - ls) <= c.l && c.l <= a.l + ls && c.parity == a.parity * psh)) continue;
+        PathH p{};
+        p.l_in = a.l; p.l_sh = ls; p.l_out = c.l; p.b_in = bi; p.b_out = bo;
+        p.c_in = a.mul; p.c_out = c.mul;
+        if (mode == TPCONV_UVU && a.mul != c.mul) { delete P; return TPCONV_ERR_INVALID_ARG; }
+        p.w_off = woff;
+        p.w_count = (mode == TPCONV_UVW) ? a.mul * c.mul : a.mul;
+        p.type = triple_index(a.l, ls, c.l);
+        p.in_off = a.offset; p.out_off = c.offset;
+        p.st_off = st_off; p.xst_off = xst_off;
+        woff += p.w_count;
+        st_off += (2 * c.l + 1) * P->K * a.mul;
+        xst_off += (2 * a.l + 1) * P->K * c.mul;
+        std::vector<int> idx;
+        std::vector<double> val;
+        cg_of_type(p.type, idx, val);
+        p.nnz = (int)val.size();
+        P->paths.push_back(p);
+        P->cg_idx.push_back(idx);
+        P->cg_val.push_back(val);
+      }
+  if (P->paths.empty()) { delete P; return TPCONV_ERR_INVALID_ARG; }
+  if ((int)P->paths.size() > MAX_PATHS) { delete P; return TPCONV_ERR_UNSUPPORTED; }
+  P->n_w = woff;
+
+  DevPlan& D = P->dev;
+  D.n_paths = (int)P->paths.size();
+  D.dim_in = P->dim_in; D.dim_out = P->dim_out; D.n_w = P->n_w; D.K = P->K; D.lmax = sh_lmax; D.mode = mode;
+  D.radial_kind = R.kind; D.poly_p = R.poly_p;
+  D.r_cut = R.r_cut; D.inv_r_cut = 1.0f / R.r_cut;
+  D.bessel_pref = (float)std::sqrt(2.0 / R.r_cut);
+  if (R.kind == TPCONV_RADIAL_GAUSSIAN) {
+    const double step = (double(R.r_max) - R.r_min) / (R.num_basis - 1);
+    D.g_mu0 = R.r_min; D.g_step = (float)step; D.g_inv_sigma2 = (float)(1.0 / (step * step));
+  }
+  const double pp = R.poly_p;
+  D.env_a = (float)((pp + 1) * (pp + 2) / 2.0);
+  D.env_b = (float)(pp * (pp + 2));
+  D.env_c = (float)(pp * (pp + 1) / 2.0);
+  D.state_per_node = st_off;
+  D.xstate_per_node = xst_off;
+  for (int k = 0; k < D.n_paths; ++k) {
+    const PathH& h = P->paths[k];
+    DevPath& d = D.p[k];
+    d.type = h.type; d.l_in = h.l_in; d.l_sh = h.l_sh; d.l_out = h.l_out;
+    d.c_in = h.c_in; d.c_out = h.c_out; d.in_off = h.in_off; d.out_off = h.out_off;
+    d.w_off = h.w_off; d.st_off = h.st_off; d.xst_off = h.xst_off; d.b_in = h.b_in; d.b_out = h.b_out;
+    P->max_mn_tn_bwd = std::max<long long>(P->max_mn_tn_bwd, (long long)h.c_in * P->K * h.c_out);
+  }
+  // warp task lists
+  auto push = [](Tasks& T, int a, int b) {
+    if (T.n >= MAX_TASKS) return false;
+    T.a[T.n] = (short)a; T.b[T.n] = (short)b; ++T.n;
+    return true;
+  };
+  bool ok = true;
+  for (int k = 0; k < D.n_paths; ++k) {
+    for (int c = 0; c < (P->paths[k].c_in + 31) / 32; ++c) ok = ok && push(P->t_in, k, c);
+    for (int c = 0; c < (P->paths[k].c_out + 31) / 32; ++c) ok = ok && push(P->t_out, k, c);
+  }
+  auto fill_bp = [&](BlockPaths& BP, Tasks& T, const std::vector<Block>& blocks, bool by_out) {
+    BP.n_blocks = (int)blocks.size();
+    for (int b = 0; b < BP.n_blocks; ++b) {
+      BP.l[b] = blocks[b].l; BP.c[b] = blocks[b].mul; BP.off[b] = blocks[b].offset; BP.count[b] = 0;
+      for (int k = 0; k < D.n_paths; ++k)
+        if ((by_out ? P->paths[k].b_out : P->paths[k].b_in) == b) BP.list[b][BP.count[b]++] = (short)k;
+      for (int c = 0; c < (blocks[b].mul + 31) / 32; ++c) ok = ok && push(T, b, c);
+    }
+  };
+  fill_bp(P->bp_out, P->t_bo, P->out, true);
+  fill_bp(P->bp_in, P->t_bi, P->in, false);
+  if (!ok) { delete P; return TPCONV_ERR_UNSUPPORTED; }
+  *out = P;
+  return TPCONV_OK;
+}
+
+tpconv_status tpconv_plan_destroy(tpconv_plan_t plan) {
+  delete plan;
+  return TPCONV_OK;
+}
+
+tpconv_status tpconv_plan_info(tpconv_plan_t P, int64_t* num_paths, int64_t* dim_in,
+                               int64_t* dim_out, int64_t* num_basis, int64_t* weight_cols) {
+  if (!P) return TPCONV_ERR_INVALID_ARG;
+  if (num_paths) *num_paths = (int64_t)P->paths.size();
+  if (dim_in) *dim_in = P->dim_in;
+  if (dim_out) *dim_out = P->dim_out;
+  if (num_basis) *num_basis = P->K;
+  if (weight_cols) *weight_cols = P->n_w;
+  return TPCONV_OK;
+}
+
+tpconv_status tpconv_plan_path(tpconv_plan_t P, int64_t index, int32_t out[10]) {
+  if (!P || !out || index < 0 || index >= (int64_t)P->paths.size()) return TPCONV_ERR_INVALID_ARG;
+  const PathH& p = P->paths[index];
+  const int32_t v[10] = {p.l_in, p.l_sh, p.l_out, p.b_in, p.b_out, p.c_in, p.c_out, p.w_off, p.w_count, p.nnz};
+  std::memcpy(out, v, sizeof v);
+  return TPCONV_OK;
+}
+
+tpconv_status tpconv_plan_path_coupling(tpconv_plan_t P, int64_t index, int32_t* idx, double* val,
+                                        int64_t cap) {
+  if (!P || !idx || !val || index < 0 || index >= (int64_t)P->paths.size()) return TPCONV_ERR_INVALID_ARG;
+  const auto& vi = P->cg_idx[index];
+  const auto& vv = P->cg_val[index];
+  if ((int64_t)vv.size() > cap) return TPCONV_ERR_INVALID_ARG;
+  for (size_t k = 0; k < vv.size(); ++k) {
+    idx[3 * k] = vi[3 * k]; idx[3 * k + 1] = vi[3 * k + 1]; idx[3 * k + 2] = vi[3 * k + 2];
+    val[k] = vv[k];
+  }
+  return TPCONV_OK;
+}
+
+tpconv_status tpconv_set_workspace_budget(tpconv_plan_t P, size_t bytes) {
+  if (!P || bytes < 4096) return TPCONV_ERR_INVALID_ARG;
+  P->budget = bytes;
+  return TPCONV_OK;
+}
+
+tpconv_status tpconv_workspace_bytes(tpconv_plan_t P, int64_t N, int64_t E, uint32_t pass_mask,
+                                     size_t* bytes) {
+  if (!P || !bytes || N < 0 || E < 0) return TPCONV_ERR_INVALID_ARG;
+  size_t best = 0;
+  for (uint32_t b : {TPCONV_PASS_FORWARD, TPCONV_PASS_BACKWARD, TPCONV_PASS_DOUBLE_BACKWARD})
+    if (pass_mask & b) best = std::max(best, make_layout(P, N, E, b).total);
+  *bytes = best;
+  return TPCONV_OK;
+}
+
+tpconv_status tpconv_csr_transpose_workspace_bytes(int64_t N, int64_t E, size_t* bytes) {
+  if (!bytes || N < 0 || E < 0) return TPCONV_ERR_INVALID_ARG;
+  *bytes = align256(size_t(4) * std::max<int64_t>(N, 1));
+  return TPCONV_OK;
+}
+
+tpconv_status tpconv_csr_transpose(int64_t N, int64_t E, const int32_t* row_ptr, const int32_t* src,
+                                   int32_t* t_ptr, int32_t* t_eid, int32_t* t_dst, void* ws,
+                                   size_t ws_bytes, struct CUstream_st* stream) {
+  if (N < 0 || E < 0 || N > 0x7ffffffe || E > 0x7ffffffe) return TPCONV_ERR_INVALID_ARG;
+  if (!row_ptr || !t_ptr || (E > 0 && (!src || !t_eid || !t_dst)) || !ws) return TPCONV_ERR_INVALID_ARG;
+  size_t need = 0;
+  tpconv_csr_transpose_workspace_bytes(N, E, &need);
+  if (ws_bytes < need) return TPCONV_ERR_WORKSPACE_TOO_SMALL;
+  if (!aligned16(row_ptr) || !aligned16(t_ptr) || (E > 0 && (!aligned16(src) || !aligned16(t_eid) || !aligned16(t_dst))) || !aligned16(ws))
+    return TPCONV_ERR_MISALIGNED;
+  cudaError_t e = launch_csr_transpose((int)N, (int)E, row_ptr, src, t_ptr, t_eid, t_dst,
+                                       static_cast<int*>(ws), (cudaStream_t)stream);
+  return e == cudaSuccess ? TPCONV_OK : TPCONV_ERR_CUDA;
+}
+
+tpconv_status tpconv_validate_graph(int64_t N, int64_t E, const int32_t* row_ptr, const int32_t* src,
+                                    int32_t* d_err, struct CUstream_st* stream) {
+  if (N < 0 || E < 0 || N > 0x7ffffffe || E > 0x7ffffffe || !row_ptr || !d_err || (E > 0 && !src))
+    return TPCONV_ERR_INVALID_ARG;
+  cudaError_t e = launch_validate_graph((int)N, (int)E, row_ptr, src, d_err, (cudaStream_t)stream);
+  return e == cudaSuccess ? TPCONV_OK : TPCONV_ERR_CUDA;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// pass implementations
+// ---------------------------------------------------------------------------
+
+namespace {
+
+#define TPC_TRY(expr)                                   \
+  do {                                                  \
+    cudaError_t e_ = (expr);                            \
+    if (e_ != cudaSuccess) return TPCONV_ERR_CUDA;      \
+  } while (0)
+
+tpconv_status common_checks(const tpconv_plan* P, int64_t N, int64_t E) {
+  if (!P || N < 0 || E < 0 || N > 0x7ffffffe || E > 0x7ffffffe) return TPCONV_ERR_INVALID_ARG;
+  return TPCONV_OK;
+}
+
+tpconv_status check_ptrs(std::initializer_list<const void*> required, std::initializer_list<const void*> optional) {
+  for (const void* p : required) {
+    if (!p) return TPCONV_ERR_INVALID_ARG;
+    if (!aligned16(p)) return TPCONV_ERR_MISALIGNED;
+  }
+  for (const void* p : optional)
+    if (p && !aligned16(p)) return TPCONV_ERR_MISALIGNED;
+  return TPCONV_OK;
+}
+
+tpconv_status check_ws(const Layout& L, void* ws, size_t ws_bytes) {
+  if (L.total == 0) return TPCONV_OK;
+  if (ws_bytes < L.total) return TPCONV_ERR_WORKSPACE_TOO_SMALL;
+  if (!ws) return TPCONV_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return TPCONV_ERR_MISALIGNED;
+  return TPCONV_OK;
+}
+
+// m[(i,mo), w] += sum_{q,u} S[(i,mo),(q,u)] A[(q,u), w]          (eqs. 34-35)
+GemmArgs g_state_times_A(const tpconv_plan* P, const PathH& p, const float* S, const float* W,
+                         float* out, int n0, int cn) {
+  const int RO = 2 * p.l_out + 1;
+  GemmArgs g = gemm_base();
+  g.M = cn * RO; g.N = p.c_out; g.K = P->K * p.c_in;
+  g.A = S + p.st_off; g.Am = idx2(RO, P->dev.state_per_node, (long long)P->K * p.c_in); g.Ak = idx1(1);
+  g.B = W + p.w_off; g.Bk = idx2(p.c_in, P->n_w, p.c_out); g.Bn = idx1(1);
+  g.C = out + (long long)n0 * P->dim_out + p.out_off; g.Cm = idx2(RO, P->dim_out, p.c_out); g.Cn = idx1(1);
+  g.accumulate = 1;
+  return g;
+}
+
+// S_bar[(i,mo),(q,u)] = sum_w m_bar[(i,mo), w] A[(q,u), w]        (eq. 36)
+GemmArgs g_sbar(const tpconv_plan* P, const PathH& p, const float* gout, const float* W,
+                float* Sbar, int n0, int cn) {
+  const int RO = 2 * p.l_out + 1;
+  GemmArgs g = gemm_base();
+  g.M = cn * RO; g.N = P->K * p.c_in; g.K = p.c_out;
+  g.A = gout + (long long)n0 * P->dim_out + p.out_off; g.Am = idx2(RO, P->dim_out, p.c_out); g.Ak = idx1(1);
+  g.B = W + p.w_off; g.Bk = idx1(1); g.Bn = idx2(p.c_in, P->n_w, p.c_out);
+  g.C = Sbar + p.st_off; g.Cm = idx2(RO, P->dev.state_per_node, (long long)P->K * p.c_in); g.Cn = idx1(1);
+  g.accumulate = 0;
+  return g;
+}
+
+// x_bar[(j,mi), u] += sum_{q,w} X[(j,mi),(q,w)] A[(q,u), w]      (mirrored eq. 21)
+GemmArgs g_xbar(const tpconv_plan* P, const PathH& p, const float* X, const float* W,
+                float* gx, int n0, int cn) {
+  const int RI = 2 * p.l_in + 1;
+  GemmArgs g = gemm_base();
+  g.M = cn * RI; g.N = p.c_in; g.K = P->K * p.c_out;
+  g.A = X + p.xst_off; g.Am = idx2(RI, P->dev.xstate_per_node, (long long)P->K * p.c_out); g.Ak = idx1(1);
+  g.B = W + p.w_off; g.Bk = idx2(p.c_out, P->n_w, 1); g.Bn = idx1(p.c_out);
+  g.C = gx + (long long)n0 * P->dim_in + p.in_off; g.Cm = idx2(RI, P->dim_in, p.c_in); g.Cn = idx1(1);
+  g.accumulate = 1;
+  return g;
+}
+
+// A_bar[(q,u), w] += sum_{(j,mi)} x[(j,mi), u] X[(j,mi),(q,w)]    (mirrored eq. 19)
+GemmArgs g_abar_src(const tpconv_plan* P, const PathH& p, const float* x, const float* X,
+                    float* gW, int n0, int cn, float* part) {
+  const int RI = 2 * p.l_in + 1;
+  GemmArgs g = gemm_base();
+  g.M = p.c_in; g.N = P->K * p.c_out; g.K = cn * RI;
+  g.A = x + (long long)n0 * P->dim_in + p.in_off; g.Am = idx1(1); g.Ak = idx2(RI, P->dim_in, p.c_in);
+  g.B = X + p.xst_off; g.Bk = idx2(RI, P->dev.xstate_per_node, (long long)P->K * p.c_out); g.Bn = idx1(1);
+  g.C = gW + p.w_off; g.Cm = idx1(p.c_out); g.Cn = idx2(p.c_out, P->n_w, 1);
+  g.accumulate = 1;
+  g.splits = splits_for(g.K);
+  g.partial = part;
+  return g;
+}
+
+// A_bar[(q,u), w] += sum_{(i,mo)} dS[(i,mo),(q,u)] m_bar[(i,mo), w]   (eq. 39)
+GemmArgs g_abar_recv(const tpconv_plan* P, const PathH& p, const float* S, const float* gout,
+                     float* gW, int n0, int cn, float* part) {
+  const int RO = 2 * p.l_out + 1;
+  GemmArgs g = gemm_base();
+  g.M = P->K * p.c_in; g.N = p.c_out; g.K = cn * RO;
+  g.A = S + p.st_off; g.Am = idx1(1); g.Ak = idx2(RO, P->dev.state_per_node, (long long)P->K * p.c_in);
+  g.B = gout + (long long)n0 * P->dim_out + p.out_off; g.Bk = idx2(RO, P->dim_out, p.c_out); g.Bn = idx1(1);
+  g.C = gW + p.w_off; g.Cm = idx2(p.c_in, P->n_w, p.c_out); g.Cn = idx1(1);
+  g.accumulate = 1;
+  g.splits = splits_for(g.K);
+  g.partial = part;
+  return g;
+}
+
+float* fptr(void* ws, size_t off) { return reinterpret_cast<float*>(static_cast<char*>(ws) + off); }
+
+}  // namespace
+
+extern "C" {
+
+tpconv_status tpconv_forward(tpconv_plan_t P, int64_t N, int64_t E, const float* x,
+                             const float* pos, const int32_t* row_ptr, const int32_t* src,
+                             const float* W, float* out, void* ws, size_t ws_bytes,
+                             struct CUstream_st* stream) {
+  tpconv_status st = common_checks(P, N, E);
+  if (st != TPCONV_OK) return st;
+  if (N == 0) return TPCONV_OK;
+  st = check_ptrs({x, pos, row_ptr, W, out}, {src});
+  if (st != TPCONV_OK) return st;
+  if (E > 0 && !src) return TPCONV_ERR_INVALID_ARG;
+  const Layout L = make_layout(P, N, E, TPCONV_PASS_FORWARD);
+  st = check_ws(L, ws, ws_bytes);
+  if (st != TPCONV_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int n = (int)N;
+  if (P->mode == TPCONV_UVU) {
+    TPC_TRY(launch_uvu_fwd(P->dev, P->bp_out, P->t_bo, 0, x, nullptr, pos, nullptr, row_ptr, src, W,
+                           nullptr, n, out, s));
+    return TPCONV_OK;
+  }
+  TPC_TRY(cudaMemsetAsync(out, 0, sizeof(float) * (size_t)N * P->dim_out, s));
+  float* S = fptr(ws, L.state_a);
+  for (int n0 = 0; n0 < n; n0 += L.recv_chunk) {
+    const int cn = std::min(L.recv_chunk, n - n0);
+    TPC_TRY(launch_uvw_state(P->dev, P->t_in, 0, x, nullptr, pos, nullptr, row_ptr, src, n0, cn, S,
+                             nullptr, s));
+    for (const PathH& p : P->paths) TPC_TRY(launch_gemm(g_state_times_A(P, p, S, W, out, n0, cn), s));
+  }
+  return TPCONV_OK;
+}
+
+tpconv_status tpconv_backward(tpconv_plan_t P, int64_t N, int64_t E, const float* x,
+                              const float* pos, const int32_t* row_ptr, const int32_t* src,
+                              const int32_t* t_ptr, const int32_t* t_eid, const int32_t* t_dst,
+                              const float* W, const float* grad_out, float* grad_x,
+                              float* grad_pos, float* grad_W, void* ws, size_t ws_bytes,
+                              struct CUstream_st* stream) {
+  tpconv_status st = common_checks(P, N, E);
+  if (st != TPCONV_OK) return st;
+  st = check_ptrs({}, {x, pos, row_ptr, src, t_ptr, t_eid, t_dst, W, grad_out, grad_x, grad_pos, grad_W});
+  if (st != TPCONV_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (N == 0) {
+    if (grad_W) TPC_TRY(cudaMemsetAsync(grad_W, 0, sizeof(float) * (size_t)P->K * P->n_w, s));
+    return TPCONV_OK;
+  }
+  if (!x || !pos || !row_ptr || !W || !grad_out || (E > 0 && !src)) return TPCONV_ERR_INVALID_ARG;
+  if ((grad_x || grad_pos || grad_W) && (!t_ptr || (E > 0 && (!t_eid || !t_dst)))) return TPCONV_ERR_INVALID_ARG;
+  const Layout L = make_layout(P, N, E, TPCONV_PASS_BACKWARD);
+  st = check_ws(L, ws, ws_bytes);
+  if (st != TPCONV_OK) return st;
+  const int n = (int)N;
+  float4* gbuf = reinterpret_cast<float4*>(static_cast<char*>(ws) + L.gbuf);
+  float* part = fptr(ws, L.part);
+
+  if (P->mode == TPCONV_UVU) {
+    if (grad_pos) {
+      TPC_TRY(launch_uvu_recv_bwd(P->dev, P->t_in, x, pos, row_ptr, src, W, grad_out, n, gbuf, s));
+      TPC_TRY(launch_pos_finish(n, row_ptr, t_ptr, t_eid, gbuf, grad_pos, s));
+    }
+    if (grad_W) {
+      const int nr = std::min(kUvuRanges, n);
+      TPC_TRY(launch_uvu_gradw(P->dev, P->t_in, 0, x, nullptr, pos, nullptr, row_ptr, src, grad_out, n,
+                               nr, part, s));
+      TPC_TRY(launch_reduce_partials(part, nr, (long long)P->K * P->n_w, grad_W, 0, s));
+    }
+    if (grad_x)
+      TPC_TRY(launch_uvu_src(P->dev, P->bp_in, P->t_bi, 0, pos, nullptr, t_ptr, t_eid, t_dst, W,
+                             nullptr, grad_out, n, grad_x, s));
+    return TPCONV_OK;
+  }
+
+  float* state = fptr(ws, L.state_a);
+  if (grad_pos) {
+    for (int n0 = 0; n0 < n; n0 += L.recv_chunk) {
+      const int cn = std::min(L.recv_chunk, n - n0);
+      for (const PathH& p : P->paths) TPC_TRY(launch_gemm(g_sbar(P, p, grad_out, W, state, n0, cn), s));
+      TPC_TRY(launch_uvw_recv_bwd(P->dev, P->t_in, x, pos, row_ptr, src, state, n0, cn, gbuf, s));
+    }
+    TPC_TRY(launch_pos_finish(n, row_ptr, t_ptr, t_eid, gbuf, grad_pos, s));
+  }
+  if (grad_x) TPC_TRY(cudaMemsetAsync(grad_x, 0, sizeof(float) * (size_t)N * P->dim_in, s));
+  if (grad_W) TPC_TRY(cudaMemsetAsync(grad_W, 0, sizeof(float) * (size_t)P->K * P->n_w, s));
+  if (grad_x || grad_W) {
+    for (int n0 = 0; n0 < n; n0 += L.src_chunk) {
+      const int cn = std::min(L.src_chunk, n - n0);
+      TPC_TRY(launch_uvw_src_state(P->dev, P->t_out, 0, pos, nullptr, t_ptr, t_eid, t_dst, grad_out, n0,
+                                   cn, state, nullptr, s));
+      for (const PathH& p : P->paths) {
+        if (grad_x) TPC_TRY(launch_gemm(g_xbar(P, p, state, W, grad_x, n0, cn), s));
+        if (grad_W) TPC_TRY(launch_gemm(g_abar_src(P, p, x, state, grad_W, n0, cn, part), s));
+      }
+    }
+  }
+  return TPCONV_OK;
+}
+
+tpconv_status tpconv_double_backward(tpconv_plan_t P, int64_t N, int64_t E, const float* x,
+                                     const float* pos, const int32_t* row_ptr, const int32_t* src,
+                                     const int32_t* t_ptr, const int32_t* t_eid,
+                                     const int32_t* t_dst, const float* W, const float* grad_out,
+                                     const float* gg_x, const float* gg_pos, const float* gg_W,
+                                     float* grad_x, float* grad_W, float* grad_grad_out,
+                                     float* grad_pos, void* ws, size_t ws_bytes,
+                                     struct CUstream_st* stream) {
+  tpconv_status st = common_checks(P, N, E);
+  if (st != TPCONV_OK) return st;
+  if (grad_pos) return TPCONV_ERR_UNSUPPORTED;
+  st = check_ptrs({}, {x, pos, row_ptr, src, t_ptr, t_eid, t_dst, W, grad_out, gg_x, gg_pos, gg_W, grad_x,
+                       grad_W, grad_grad_out});
+  if (st != TPCONV_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (N == 0) {
+    if (grad_W) TPC_TRY(cudaMemsetAsync(grad_W, 0, sizeof(float) * (size_t)P->K * P->n_w, s));
+    return TPCONV_OK;
+  }
+  if (!x || !pos || !row_ptr || !W || !grad_out || (E > 0 && !src)) return TPCONV_ERR_INVALID_ARG;
+  if (grad_x && (!t_ptr || (E > 0 && !t_dst))) return TPCONV_ERR_INVALID_ARG;
+  const Layout L = make_layout(P, N, E, TPCONV_PASS_DOUBLE_BACKWARD);
+  st = check_ws(L, ws, ws_bytes);
+  if (st != TPCONV_OK) return st;
+  const int n = (int)N;
+  float* part = fptr(ws, L.part);
+  const bool tan_xp = gg_x || gg_pos;
+
+  if (P->mode == TPCONV_UVU) {
+    if (grad_grad_out)
+      TPC_TRY(launch_uvu_fwd(P->dev, P->bp_out, P->t_bo, 1, x, gg_x, pos, gg_pos, row_ptr, src, W, gg_W,
+                             n, grad_grad_out, s));
+    if (grad_W) {
+      const int nr = std::min(kUvuRanges, n);
+      TPC_TRY(launch_uvu_gradw(P->dev, P->t_in, 1, x, gg_x, pos, gg_pos, row_ptr, src, grad_out, n, nr,
+                               part, s));
+      TPC_TRY(launch_reduce_partials(part, nr, (long long)P->K * P->n_w, grad_W, 0, s));
+    }
+    if (grad_x)
+      TPC_TRY(launch_uvu_src(P->dev, P->bp_in, P->t_bi, 1, pos, gg_pos, t_ptr, t_eid, t_dst, W, gg_W,
+                             grad_out, n, grad_x, s));
+    return TPCONV_OK;
+  }
+
+  float* sa = fptr(ws, L.state_a);
+  float* sb = fptr(ws, L.state_b);
+  if (grad_grad_out) TPC_TRY(cudaMemsetAsync(grad_grad_out, 0, sizeof(float) * (size_t)N * P->dim_out, s));
+  if (grad_W) TPC_TRY(cudaMemsetAsync(grad_W, 0, sizeof(float) * (size_t)P->K * P->n_w, s));
+  const bool need_S = grad_grad_out && gg_W;
+  if ((grad_grad_out || grad_W) && (tan_xp || need_S)) {
+    for (int n0 = 0; n0 < n; n0 += L.recv_chunk) {
+      const int cn = std::min(L.recv_chunk, n - n0);
+      // sa = dS (tangent of eq. 33), sb = S (needed for S dA in eq. 37)
+      TPC_TRY(launch_uvw_state(P->dev, P->t_in, 1, x, gg_x, pos, gg_pos, row_ptr, src, n0, cn,
+                               need_S ? sb : nullptr, sa, s));
+      for (const PathH& p : P->paths) {
+        if (grad_grad_out && tan_xp) TPC_TRY(launch_gemm(g_state_times_A(P, p, sa, W, grad_grad_out, n0, cn), s));
+        if (need_S) TPC_TRY(launch_gemm(g_state_times_A(P, p, sb, gg_W, grad_grad_out, n0, cn), s));
+        if (grad_W && tan_xp) TPC_TRY(launch_gemm(g_abar_recv(P, p, sa, grad_out, grad_W, n0, cn, part), s));
+      }
+    }
+  }
+  if (grad_x) {
+    TPC_TRY(cudaMemsetAsync(grad_x, 0, sizeof(float) * (size_t)N * P->dim_in, s));
+    if (gg_pos || gg_W) {
+      for (int n0 = 0; n0 < n; n0 += L.src_chunk) {
+        const int cn = std::min(L.src_chunk, n - n0);
+        // sa = X' (tangent of the source state), sb = X
+        TPC_TRY(launch_uvw_src_state(P->dev, P->t_out, 1, pos, gg_pos, t_ptr, t_eid, t_dst, grad_out, n0,
+                                     cn, gg_W ? sb : nullptr, sa, s));
+        for (const PathH& p : P->paths) {
+          if (gg_pos) TPC_TRY(launch_gemm(g_xbar(P, p, sa, W, grad_x, n0, cn), s));
+          if (gg_W) TPC_TRY(launch_gemm(g_xbar(P, p, sb, gg_W, grad_x, n0, cn), s));
+        }
+      }
+    }
+  }
+  return TPCONV_OK;
+}
+
+}  // extern "C"

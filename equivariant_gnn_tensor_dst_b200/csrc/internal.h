@@ -1,0 +1,152 @@
+// Internal types shared by the host plan/launch code and the kernels.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace tpc {
+
+constexpr int MAX_PATHS = 64;
+constexpr int MAX_TASKS = 256;
+constexpr int MAX_BLOCKS = 16;
+constexpr int WARPS_PER_CTA = 4;
+
+// One path of the plan as the kernels see it.
+struct DevPath {
+  int type;            // index into tpc_tab::TRIPLES (the (l_in, l_sh, l_out) triple)
+  int l_in, l_sh, l_out;
+  int c_in, c_out;
+  int in_off, out_off; // float offsets of the input / output block inside a node row
+  int w_off;           // first weight column
+  int st_off;          // offset of the path inside a receiver-state row  (R_out*K*C_in floats)
+  int xst_off;         // offset of the path inside a source-state row    (R_in*K*C_out floats)
+  int b_in, b_out;
+};
+
+struct DevPlan {
+  int n_paths, dim_in, dim_out, n_w, K, lmax, mode;
+  int radial_kind, poly_p;
+  float r_cut, inv_r_cut, bessel_pref, g_mu0, g_step, g_inv_sigma2;
+  float env_a, env_b, env_c;
+  int state_per_node;   // sum_pi R_out * K * C_in
+  int xstate_per_node;  // sum_pi R_in * K * C_out
+  DevPath p[MAX_PATHS];
+};
+
+// A list of warp tasks: (a, b) pairs whose meaning depends on the kernel
+// (path & 32-channel chunk, or block & chunk).
+struct Tasks {
+  int n;
+  short a[MAX_TASKS];
+  short b[MAX_TASKS];
+};
+
+// Paths grouped by an irrep block (output block for uvu forward, input block for the
+// uvu source pass).
+struct BlockPaths {
+  int n_blocks;
+  int l[MAX_BLOCKS];
+  int c[MAX_BLOCKS];
+  int off[MAX_BLOCKS];
+  int count[MAX_BLOCKS];
+  short list[MAX_BLOCKS][MAX_PATHS];
+};
+
+// Two-level affine index map f(i) = (i / d) * s1 + (i % d) * s2.
+struct Idx2 {
+  int d;
+  long long s1, s2;
+};
+inline Idx2 idx1(long long s) { return Idx2{0x7fffffff, 0, s}; }
+inline Idx2 idx2(int d, long long s1, long long s2) { return Idx2{d, s1, s2}; }
+
+struct GemmArgs {
+  const float* A; Idx2 Am, Ak;   // A(m, k)
+  const float* B; Idx2 Bk, Bn;   // B(k, n)
+  float* C; Idx2 Cm, Cn;         // C(m, n)
+  int M, N, K;
+  int accumulate;                // C += AB (1) or C = AB (0)
+  float* partial;                // split-K scratch [splits][M][N] (splits > 1)
+  int splits;
+};
+
+// Per-(KP, MODE) kernel runners.  Each is explicitly instantiated in its own
+// translation unit (the build compiles k_uvw.cu / k_uvu.cu once per unit) so that the
+// heavily unrolled kernels compile in parallel.
+template <int KP, int MODE>
+cudaError_t run_uvw_state(const DevPlan& P, const Tasks& T, const float* x, const float* xdot,
+                          const float* pos, const float* posdot, const int* row_ptr,
+                          const int* src, int node0, int n_nodes, float* S, float* Sdot,
+                          cudaStream_t s);
+template <int KP>
+cudaError_t run_uvw_recv_bwd(const DevPlan& P, const Tasks& T, const float* x, const float* pos,
+                             const int* row_ptr, const int* src, const float* Sbar, int node0,
+                             int n_nodes, float4* gbuf, cudaStream_t s);
+template <int KP, int MODE>
+cudaError_t run_uvw_src_state(const DevPlan& P, const Tasks& T, const float* pos,
+                              const float* posdot, const int* t_ptr, const int* t_dst,
+                              const float* grad_out, int node0, int n_nodes, float* X,
+                              float* Xdot, cudaStream_t s);
+template <int KP, int MODE>
+cudaError_t run_uvu_fwd(const DevPlan& P, const BlockPaths& BP, const Tasks& T, const float* x,
+                        const float* xdot, const float* pos, const float* posdot,
+                        const int* row_ptr, const int* src, const float* W, const float* Wdot,
+                        int N, float* out, cudaStream_t s);
+template <int KP>
+cudaError_t run_uvu_recv_bwd(const DevPlan& P, const Tasks& T, const float* x, const float* pos,
+                             const int* row_ptr, const int* src, const float* W,
+                             const float* grad_out, int N, float4* gbuf, cudaStream_t s);
+template <int KP, int MODE>
+cudaError_t run_uvu_gradw(const DevPlan& P, const Tasks& T, const float* x, const float* xdot,
+                          const float* pos, const float* posdot, const int* row_ptr,
+                          const int* src, const float* grad_out, int N, int n_ranges,
+                          float* partial, cudaStream_t s);
+template <int KP, int MODE>
+cudaError_t run_uvu_src(const DevPlan& P, const BlockPaths& BP, const Tasks& T, const float* pos,
+                        const float* posdot, const int* t_ptr, const int* t_dst, const float* W,
+                        const float* Wdot, const float* grad_out, int N, float* grad_x,
+                        cudaStream_t s);
+
+// kernel launchers (dispatch on K and mode; defined in launch.cu and k_misc.cu)
+cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
+
+cudaError_t launch_uvw_state(const DevPlan& P, const Tasks& T, int mode, const float* x,
+                             const float* xdot, const float* pos, const float* posdot,
+                             const int* row_ptr, const int* src, int node0, int n_nodes,
+                             float* S, float* Sdot, cudaStream_t s);
+cudaError_t launch_uvw_recv_bwd(const DevPlan& P, const Tasks& T, const float* x,
+                                const float* pos, const int* row_ptr, const int* src,
+                                const float* Sbar, int node0, int n_nodes, float4* gbuf,
+                                cudaStream_t s);
+cudaError_t launch_uvw_src_state(const DevPlan& P, const Tasks& T, int mode,
+                                 const float* pos, const float* posdot, const int* t_ptr,
+                                 const int* t_eid, const int* t_dst, const float* grad_out,
+                                 int node0, int n_nodes, float* X, float* Xdot,
+                                 cudaStream_t s);
+cudaError_t launch_uvu_fwd(const DevPlan& P, const BlockPaths& BP, const Tasks& T, int mode,
+                           const float* x, const float* xdot, const float* pos,
+                           const float* posdot, const int* row_ptr, const int* src,
+                           const float* W, const float* Wdot, int N, float* out,
+                           cudaStream_t s);
+cudaError_t launch_uvu_recv_bwd(const DevPlan& P, const Tasks& T, const float* x,
+                                const float* pos, const int* row_ptr, const int* src,
+                                const float* W, const float* grad_out, int N, float4* gbuf,
+                                cudaStream_t s);
+cudaError_t launch_uvu_gradw(const DevPlan& P, const Tasks& T, int mode, const float* x,
+                             const float* xdot, const float* pos, const float* posdot,
+                             const int* row_ptr, const int* src, const float* grad_out,
+                             int N, int n_ranges, float* partial, cudaStream_t s);
+cudaError_t launch_uvu_src(const DevPlan& P, const BlockPaths& BP, const Tasks& T, int mode,
+                           const float* pos, const float* posdot, const int* t_ptr,
+                           const int* t_eid, const int* t_dst, const float* W,
+                           const float* Wdot, const float* grad_out, int N, float* grad_x,
+                           cudaStream_t s);
+cudaError_t launch_reduce_partials(const float* partial, int n_parts, long long n, float* out,
+                                   int accumulate, cudaStream_t s);
+cudaError_t launch_pos_finish(int N, const int* row_ptr, const int* t_ptr, const int* t_eid,
+                              const float4* gbuf, float* grad_pos, cudaStream_t s);
+cudaError_t launch_csr_transpose(int N, int E, const int* row_ptr, const int* src, int* t_ptr,
+                                 int* t_eid, int* t_dst, int* cursor, cudaStream_t s);
+cudaError_t launch_validate_graph(int N, int E, const int* row_ptr, const int* src, int* err,
+                                  cudaStream_t s);
+
+}  // namespace tpc

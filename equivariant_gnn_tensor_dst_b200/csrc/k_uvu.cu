@@ -1,0 +1,572 @@
+// Channelwise (uvu) streaming kernels.
+//
+// Sobek: Streaming Equivariant Tensor Product Convolutions, eq. 7 (uvu ties the output
+// channel to the input channel) and section 4 ("compiles channelwise uvu directly
+// rather than pruning off-diagonal mixing from dense uvw ... without edge workspace").
+// With one weight per (path, channel), the edge weight w_{e,pi,u} = sum_q phi_q A_{q,pi,u}
+// (eq. 17) is formed in registers and consumed at once; there is no receiver state and
+// no channel GEMM.
+//
+//  * k_uvu_fwd      -- m_i (eq. 11), or its tangent m_dot (eq. 25) for the double backward
+//  * k_uvu_recv_bwd -- per edge phi_bar (eq. 20) and Y_bar (eq. 22) -> d L / d r_e
+//  * k_uvu_gradw    -- A_bar (eq. 19), or its directional derivative (eq. 27), as
+//                      deterministic per-receiver-range partials
+//  * k_uvu_src      -- x_bar (eq. 21), or eq. 30, owned by the source CSR
+#include "common.cuh"
+
+namespace tpc {
+
+template <int KP>
+struct USmem {
+  int j[WARPS_PER_CTA][32];
+  float Y[WARPS_PER_CTA][32][8];
+  float phi[WARPS_PER_CTA][32][KP];
+  float Yd[WARPS_PER_CTA][32][8];
+  float phid[WARPS_PER_CTA][32][KP];
+};
+
+template <int LS, int KP, bool TAN>
+__device__ __forceinline__ void uprep(const DevPlan& P, const float* __restrict__ pos,
+                                      const float* __restrict__ posdot, int i, int j, int store,
+                                      USmem<KP>& sm, int w, int lane) {
+  constexpr int RS = 2 * LS + 1;
+  const EdgeGeo g = edge_geo(pos, i, j);
+  const Pow3 pw(g.ux, g.uy, g.uz);
+  float Y[RS], phi[KP], dphi[KP];
+  sh_block<LS>(pw, Y);
+  radial<KP, TAN>(P, g.d, phi, dphi);
+  sm.j[w][lane] = store;
+#pragma unroll
+  for (int k = 0; k < RS; ++k) sm.Y[w][lane][k] = Y[k];
+#pragma unroll
+  for (int q = 0; q < KP; ++q) sm.phi[w][lane][q] = phi[q];
+  if (TAN) {
+    float vx = 0.f, vy = 0.f, vz = 0.f;
+    if (posdot) {
+      vx = __ldg(posdot + 3 * j) - __ldg(posdot + 3 * i);
+      vy = __ldg(posdot + 3 * j + 1) - __ldg(posdot + 3 * i + 1);
+      vz = __ldg(posdot + 3 * j + 2) - __ldg(posdot + 3 * i + 2);
+    }
+    const float s = g.ux * vx + g.uy * vy + g.uz * vz;
+    const float tx = (vx - s * g.ux) * g.inv_d, ty = (vy - s * g.uy) * g.inv_d,
+                tz = (vz - s * g.uz) * g.inv_d;
+    float Yd[RS];
+    sh_block_dir<LS>(pw, tx, ty, tz, Yd);
+#pragma unroll
+    for (int k = 0; k < RS; ++k) sm.Yd[w][lane][k] = Yd[k];
+#pragma unroll
+    for (int q = 0; q < KP; ++q) sm.phid[w][lane][q] = dphi[q] * s;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// forward (MODE 0) and forward tangent (MODE 1)
+// ---------------------------------------------------------------------------
+
+template <int LI, int LS, int LO, int KP, int MODE>
+__device__ __forceinline__ void uvu_fwd_body(const DevPlan& P, const DevPath& p, int u, bool act,
+                                             int i, const float* __restrict__ x,
+                                             const float* __restrict__ xdot,
+                                             const float* __restrict__ pos,
+                                             const float* __restrict__ posdot,
+                                             const int* __restrict__ row_ptr,
+                                             const int* __restrict__ src,
+                                             const float* __restrict__ W,
+                                             const float* __restrict__ Wdot, float* m,
+                                             USmem<KP>& sm) {
+  constexpr int RI = 2 * LI + 1, RS = 2 * LS + 1, RO = 2 * LO + 1;
+  constexpr bool TAN = MODE == 1;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float a[KP], ad[KP];
+#pragma unroll
+  for (int q = 0; q < KP; ++q) {
+    a[q] = (act && q < P.K) ? __ldg(W + (long long)q * P.n_w + p.w_off + u) : 0.f;
+    ad[q] = (TAN && Wdot && act && q < P.K) ? __ldg(Wdot + (long long)q * P.n_w + p.w_off + u) : 0.f;
+  }
+  const float* xb = x + p.in_off + (act ? u : 0);
+  const float* xdb = xdot ? xdot + p.in_off + (act ? u : 0) : nullptr;
+  const int eb = __ldg(row_ptr + i), ee = __ldg(row_ptr + i + 1);
+  for (int e0 = eb; e0 < ee; e0 += 32) {
+    const int ne = min(32, ee - e0);
+    if (lane < ne) {
+      const int j = __ldg(src + e0 + lane);
+      uprep<LS, KP, TAN>(P, pos, posdot, i, j, j, sm, w, lane);
+    }
+    __syncwarp();
+    for (int t = 0; t < ne; ++t) {
+      const long long row = (long long)sm.j[w][t] * P.dim_in;
+      float xv[RI], Y[RS], C[RO];
+#pragma unroll
+      for (int k = 0; k < RI; ++k) xv[k] = act ? __ldg(xb + row + k * p.c_in) : 0.f;
+#pragma unroll
+      for (int k = 0; k < RS; ++k) Y[k] = sm.Y[w][t][k];
+      float we = 0.f;
+#pragma unroll
+      for (int q = 0; q < KP; ++q) we = fmaf(sm.phi[w][t][q], a[q], we);
+      cg_couple<LI, LS, LO>(xv, Y, C);
+      if (!TAN) {
+#pragma unroll
+        for (int o = 0; o < RO; ++o) m[o] = fmaf(we, C[o], m[o]);
+      } else {
+        float Yd[RS], Cd[RO], C2[RO];
+        float wd = 0.f;
+#pragma unroll
+        for (int q = 0; q < KP; ++q) wd = fmaf(sm.phid[w][t][q], a[q], fmaf(sm.phi[w][t][q], ad[q], wd));
+#pragma unroll
+        for (int k = 0; k < RS; ++k) Yd[k] = sm.Yd[w][t][k];
+        cg_couple<LI, LS, LO>(xv, Yd, Cd);
+        if (xdb) {
+          float xdv[RI];
+#pragma unroll
+          for (int k = 0; k < RI; ++k) xdv[k] = act ? __ldg(xdb + row + k * p.c_in) : 0.f;
+          cg_couple<LI, LS, LO>(xdv, Y, C2);
+#pragma unroll
+          for (int o = 0; o < RO; ++o) Cd[o] += C2[o];
+        }
+#pragma unroll
+        for (int o = 0; o < RO; ++o) m[o] = fmaf(wd, C[o], fmaf(we, Cd[o], m[o]));
+      }
+    }
+    __syncwarp();
+  }
+}
+
+template <int KP, int MODE>
+__global__ void __launch_bounds__(WARPS_PER_CTA * 32)
+    k_uvu_fwd(DevPlan P, BlockPaths BP, Tasks T, const float* __restrict__ x,
+              const float* __restrict__ xdot, const float* __restrict__ pos,
+              const float* __restrict__ posdot, const int* __restrict__ row_ptr,
+              const int* __restrict__ src, const float* __restrict__ W,
+              const float* __restrict__ Wdot, int N, float* out) {
+  __shared__ USmem<KP> sm;
+  const long long gw = (long long)blockIdx.x * WARPS_PER_CTA + (threadIdx.x >> 5);
+  const int i = (int)(gw / T.n);
+  const int task = (int)(gw % T.n);
+  if (i >= N) return;
+  const int bo = T.a[task];
+  const int lane = threadIdx.x & 31;
+  const int u = T.b[task] * 32 + lane;
+  const int c = BP.c[bo];
+  const bool act = u < c;
+  float m[7];
+#pragma unroll
+  for (int o = 0; o < 7; ++o) m[o] = 0.f;
+  for (int k = 0; k < BP.count[bo]; ++k) {
+    const DevPath& p = P.p[BP.list[bo][k]];
+    dispatch_type(p.type, [&](auto tr) {
+      using TR = decltype(tr);
+      uvu_fwd_body<TR::li, TR::ls, TR::lo, KP, MODE>(P, p, u, act, i, x, xdot, pos, posdot, row_ptr,
+                                                     src, W, Wdot, m, sm);
+    });
+  }
+  if (!act) return;
+  const int ro = 2 * BP.l[bo] + 1;
+  float* dst = out + (long long)i * P.dim_out + BP.off[bo] + u;
+#pragma unroll
+  for (int o = 0; o < 7; ++o)
+    if (o < ro) dst[o * c] = m[o];
+}
+
+// ---------------------------------------------------------------------------
+// receiver backward: phi_bar, Y_bar -> d L / d r_e
+// ---------------------------------------------------------------------------
+
+template <int KP>
+struct URecvSmem {
+  int j[WARPS_PER_CTA][32];
+  float Y[WARPS_PER_CTA][32][16];
+  float phi[WARPS_PER_CTA][32][KP];
+  float accY[WARPS_PER_CTA][32][16];
+  float accphi[WARPS_PER_CTA][32][KP];
+};
+
+template <int LI, int LS, int LO, int KP>
+__device__ __forceinline__ void uvu_recv_body(const DevPlan& P, const DevPath& p, int chunk, int i,
+                                              int ne, const float* __restrict__ x,
+                                              const float* __restrict__ W,
+                                              const float* __restrict__ gout,
+                                              URecvSmem<KP>& sm) {
+  constexpr int RI = 2 * LI + 1, RS = 2 * LS + 1, RO = 2 * LO + 1;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int u = chunk * 32 + lane;
+  const bool act = u < p.c_in;
+  float a[KP], mb[RO];
+#pragma unroll
+  for (int q = 0; q < KP; ++q) a[q] = (act && q < P.K) ? __ldg(W + (long long)q * P.n_w + p.w_off + u) : 0.f;
+#pragma unroll
+  for (int o = 0; o < RO; ++o)
+    mb[o] = act ? __ldg(gout + (long long)i * P.dim_out + p.out_off + o * p.c_out + u) : 0.f;
+  const float* xb = x + p.in_off + (act ? u : 0);
+  const int yw = reduce_multi_index<8>(lane), pw_ = reduce_multi_index<KP>(lane);
+  const bool ywr = reduce_multi_writer<8>(lane), pwr = reduce_multi_writer<KP>(lane);
+  for (int t = 0; t < ne; ++t) {
+    const long long row = (long long)sm.j[w][t] * P.dim_in;
+    float xv[RI], Y[RS], C[RO];
+#pragma unroll
+    for (int k = 0; k < RI; ++k) xv[k] = act ? __ldg(xb + row + k * p.c_in) : 0.f;
+#pragma unroll
+    for (int k = 0; k < RS; ++k) Y[k] = sm.Y[w][t][LS * LS + k];
+    cg_couple<LI, LS, LO>(xv, Y, C);
+    float h = 0.f;
+#pragma unroll
+    for (int o = 0; o < RO; ++o) h = fmaf(mb[o], C[o], h);   // eq. 18
+    float we = 0.f;
+    float pp[KP];
+#pragma unroll
+    for (int q = 0; q < KP; ++q) {
+      we = fmaf(sm.phi[w][t][q], a[q], we);
+      pp[q] = a[q] * h;                                        // eq. 20 (per channel)
+    }
+    float G[RO], py[8];
+#pragma unroll
+    for (int o = 0; o < RO; ++o) G[o] = mb[o] * we;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) py[k] = 0.f;
+    cg_adj_y<LI, LS, LO>(xv, G, py);                            // eq. 22 (per channel)
+    const float rphi = warp_reduce_multi<KP>(pp);
+    const float ry = warp_reduce_multi<8>(py);
+    if (pwr) sm.accphi[w][t][pw_] += rphi;
+    if (ywr && yw < RS) sm.accY[w][t][LS * LS + yw] += ry;
+    __syncwarp();
+  }
+}
+
+template <int KP>
+__global__ void __launch_bounds__(WARPS_PER_CTA * 32)
+    k_uvu_recv_bwd(DevPlan P, Tasks T, const float* __restrict__ x, const float* __restrict__ pos,
+                   const int* __restrict__ row_ptr, const int* __restrict__ src,
+                   const float* __restrict__ W, const float* __restrict__ gout, int N,
+                   float4* gbuf) {
+  __shared__ URecvSmem<KP> sm;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * WARPS_PER_CTA + w;
+  if (i >= N) return;
+  const int eb = __ldg(row_ptr + i), ee = __ldg(row_ptr + i + 1);
+  for (int e0 = eb; e0 < ee; e0 += 32) {
+    const int ne = min(32, ee - e0);
+    if (lane < ne) {
+      const int j = __ldg(src + e0 + lane);
+      const EdgeGeo g = edge_geo(pos, i, j);
+      const Pow3 pw(g.ux, g.uy, g.uz);
+      float Y[16], phi[KP], dphi[KP];
+      sh_all(pw, Y);
+      radial<KP, false>(P, g.d, phi, dphi);
+      sm.j[w][lane] = j;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) { sm.Y[w][lane][k] = Y[k]; sm.accY[w][lane][k] = 0.f; }
+#pragma unroll
+      for (int q = 0; q < KP; ++q) { sm.phi[w][lane][q] = phi[q]; sm.accphi[w][lane][q] = 0.f; }
+    }
+    __syncwarp();
+    for (int task = 0; task < T.n; ++task) {
+      const DevPath& p = P.p[T.a[task]];
+      const int chunk = T.b[task];
+      dispatch_type(p.type, [&](auto tr) {
+        using TR = decltype(tr);
+        uvu_recv_body<TR::li, TR::ls, TR::lo, KP>(P, p, chunk, i, ne, x, W, gout, sm);
+      });
+    }
+    __syncwarp();
+    if (lane < ne) {
+      const int j = sm.j[w][lane];
+      const EdgeGeo g = edge_geo(pos, i, j);
+      const Pow3 pw(g.ux, g.uy, g.uz);
+      float phi[KP], dphi[KP], Yb[16];
+      radial<KP, true>(P, g.d, phi, dphi);
+#pragma unroll
+      for (int k = 0; k < 16; ++k) Yb[k] = sm.accY[w][lane][k];
+      float vx = 0.f, vy = 0.f, vz = 0.f;
+      sh_vjp_all(pw, Yb, vx, vy, vz);
+      const float vr = vx * g.ux + vy * g.uy + vz * g.uz;
+      float s = 0.f;
+#pragma unroll
+      for (int q = 0; q < KP; ++q) s = fmaf(sm.accphi[w][lane][q], dphi[q], s);
+      float4 o;
+      o.x = (vx - vr * g.ux) * g.inv_d + s * g.ux;
+      o.y = (vy - vr * g.uy) * g.inv_d + s * g.uy;
+      o.z = (vz - vr * g.uz) * g.inv_d + s * g.uz;
+      o.w = 0.f;
+      gbuf[e0 + lane] = o;
+    }
+    __syncwarp();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// radial-parameter gradient (eq. 19; MODE 1: eq. 27) as per-range partials
+// ---------------------------------------------------------------------------
+
+template <int LI, int LS, int LO, int KP, int MODE>
+__device__ __forceinline__ void uvu_gradw_body(const DevPlan& P, const DevPath& p, int chunk, int r0,
+                                               int r1, const float* __restrict__ x,
+                                               const float* __restrict__ xdot,
+                                               const float* __restrict__ pos,
+                                               const float* __restrict__ posdot,
+                                               const int* __restrict__ row_ptr,
+                                               const int* __restrict__ src,
+                                               const float* __restrict__ gout, float* part,
+                                               USmem<KP>& sm) {
+  constexpr int RI = 2 * LI + 1, RS = 2 * LS + 1, RO = 2 * LO + 1;
+  constexpr bool TAN = MODE == 1;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int u = chunk * 32 + lane;
+  const bool act = u < p.c_in;
+  const float* xb = x + p.in_off + (act ? u : 0);
+  const float* xdb = xdot ? xdot + p.in_off + (act ? u : 0) : nullptr;
+  float acc[KP];
+#pragma unroll
+  for (int q = 0; q < KP; ++q) acc[q] = 0.f;
+  for (int i = r0; i < r1; ++i) {
+    float mb[RO];
+#pragma unroll
+    for (int o = 0; o < RO; ++o)
+      mb[o] = act ? __ldg(gout + (long long)i * P.dim_out + p.out_off + o * p.c_out + u) : 0.f;
+    const int eb = __ldg(row_ptr + i), ee = __ldg(row_ptr + i + 1);
+    for (int e0 = eb; e0 < ee; e0 += 32) {
+      const int ne = min(32, ee - e0);
+      if (lane < ne) {
+        const int j = __ldg(src + e0 + lane);
+        uprep<LS, KP, TAN>(P, pos, posdot, i, j, j, sm, w, lane);
+      }
+      __syncwarp();
+      for (int t = 0; t < ne; ++t) {
+        const long long row = (long long)sm.j[w][t] * P.dim_in;
+        float xv[RI], Y[RS], C[RO];
+#pragma unroll
+        for (int k = 0; k < RI; ++k) xv[k] = act ? __ldg(xb + row + k * p.c_in) : 0.f;
+#pragma unroll
+        for (int k = 0; k < RS; ++k) Y[k] = sm.Y[w][t][k];
+        cg_couple<LI, LS, LO>(xv, Y, C);
+        float h = 0.f;
+#pragma unroll
+        for (int o = 0; o < RO; ++o) h = fmaf(mb[o], C[o], h);
+        if (!TAN) {
+#pragma unroll
+          for (int q = 0; q < KP; ++q) acc[q] = fmaf(sm.phi[w][t][q], h, acc[q]);
+        } else {
+          float Yd[RS], Cd[RO], C2[RO];
+#pragma unroll
+          for (int k = 0; k < RS; ++k) Yd[k] = sm.Yd[w][t][k];
+          cg_couple<LI, LS, LO>(xv, Yd, Cd);
+          if (xdb) {
+            float xdv[RI];
+#pragma unroll
+            for (int k = 0; k < RI; ++k) xdv[k] = act ? __ldg(xdb + row + k * p.c_in) : 0.f;
+            cg_couple<LI, LS, LO>(xdv, Y, C2);
+#pragma unroll
+            for (int o = 0; o < RO; ++o) Cd[o] += C2[o];
+          }
+          float hd = 0.f;
+#pragma unroll
+          for (int o = 0; o < RO; ++o) hd = fmaf(mb[o], Cd[o], hd);
+#pragma unroll
+          for (int q = 0; q < KP; ++q) acc[q] = fmaf(sm.phid[w][t][q], h, fmaf(sm.phi[w][t][q], hd, acc[q]));
+        }
+      }
+      __syncwarp();
+    }
+  }
+  if (!act) return;
+#pragma unroll
+  for (int q = 0; q < KP; ++q)
+    if (q < P.K) part[(long long)q * P.n_w + p.w_off + u] = acc[q];
+}
+
+template <int KP, int MODE>
+__global__ void __launch_bounds__(WARPS_PER_CTA * 32)
+    k_uvu_gradw(DevPlan P, Tasks T, const float* __restrict__ x, const float* __restrict__ xdot,
+                const float* __restrict__ pos, const float* __restrict__ posdot,
+                const int* __restrict__ row_ptr, const int* __restrict__ src,
+                const float* __restrict__ gout, int N, int n_ranges, float* partial) {
+  __shared__ USmem<KP> sm;
+  const long long gw = (long long)blockIdx.x * WARPS_PER_CTA + (threadIdx.x >> 5);
+  const int range = (int)(gw / T.n);
+  const int task = (int)(gw % T.n);
+  if (range >= n_ranges) return;
+  const int r0 = (int)((long long)N * range / n_ranges);
+  const int r1 = (int)((long long)N * (range + 1) / n_ranges);
+  const DevPath& p = P.p[T.a[task]];
+  const int chunk = T.b[task];
+  float* part = partial + (long long)range * P.K * P.n_w;
+  dispatch_type(p.type, [&](auto tr) {
+    using TR = decltype(tr);
+    uvu_gradw_body<TR::li, TR::ls, TR::lo, KP, MODE>(P, p, chunk, r0, r1, x, xdot, pos, posdot,
+                                                     row_ptr, src, gout, part, sm);
+  });
+}
+
+// ---------------------------------------------------------------------------
+// source pass: x_bar (eq. 21; MODE 1: eq. 30)
+// ---------------------------------------------------------------------------
+
+template <int LI, int LS, int LO, int KP, int MODE>
+__device__ __forceinline__ void uvu_src_body(const DevPlan& P, const DevPath& p, int u, bool act,
+                                             int j, const float* __restrict__ pos,
+                                             const float* __restrict__ posdot,
+                                             const int* __restrict__ t_ptr,
+                                             const int* __restrict__ t_dst,
+                                             const float* __restrict__ W,
+                                             const float* __restrict__ Wdot,
+                                             const float* __restrict__ gout, float* xb_acc,
+                                             USmem<KP>& sm) {
+  constexpr int RI = 2 * LI + 1, RS = 2 * LS + 1, RO = 2 * LO + 1;
+  constexpr bool TAN = MODE == 1;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float a[KP], ad[KP];
+#pragma unroll
+  for (int q = 0; q < KP; ++q) {
+    a[q] = (act && q < P.K) ? __ldg(W + (long long)q * P.n_w + p.w_off + u) : 0.f;
+    ad[q] = (TAN && Wdot && act && q < P.K) ? __ldg(Wdot + (long long)q * P.n_w + p.w_off + u) : 0.f;
+  }
+  const float* gb = gout + p.out_off + (act ? u : 0);
+  const int kb = __ldg(t_ptr + j), ke = __ldg(t_ptr + j + 1);
+  for (int k0 = kb; k0 < ke; k0 += 32) {
+    const int ne = min(32, ke - k0);
+    if (lane < ne) {
+      const int i = __ldg(t_dst + k0 + lane);
+      uprep<LS, KP, TAN>(P, pos, posdot, i, j, i, sm, w, lane);
+    }
+    __syncwarp();
+    for (int t = 0; t < ne; ++t) {
+      const long long row = (long long)sm.j[w][t] * P.dim_out;
+      float mb[RO], Y[RS], U[RI];
+#pragma unroll
+      for (int o = 0; o < RO; ++o) mb[o] = act ? __ldg(gb + row + o * p.c_out) : 0.f;
+#pragma unroll
+      for (int k = 0; k < RS; ++k) Y[k] = sm.Y[w][t][k];
+      float we = 0.f;
+#pragma unroll
+      for (int q = 0; q < KP; ++q) we = fmaf(sm.phi[w][t][q], a[q], we);
+      cg_adj_x<LI, LS, LO>(Y, mb, U);
+      if (!TAN) {
+#pragma unroll
+        for (int k = 0; k < RI; ++k) xb_acc[k] = fmaf(we, U[k], xb_acc[k]);
+      } else {
+        float Yd[RS], Ud[RI];
+        float wd = 0.f;
+#pragma unroll
+        for (int q = 0; q < KP; ++q) wd = fmaf(sm.phid[w][t][q], a[q], fmaf(sm.phi[w][t][q], ad[q], wd));
+#pragma unroll
+        for (int k = 0; k < RS; ++k) Yd[k] = sm.Yd[w][t][k];
+        cg_adj_x<LI, LS, LO>(Yd, mb, Ud);
+#pragma unroll
+        for (int k = 0; k < RI; ++k) xb_acc[k] = fmaf(wd, U[k], fmaf(we, Ud[k], xb_acc[k]));
+      }
+    }
+    __syncwarp();
+  }
+}
+
+template <int KP, int MODE>
+__global__ void __launch_bounds__(WARPS_PER_CTA * 32)
+    k_uvu_src(DevPlan P, BlockPaths BP, Tasks T, const float* __restrict__ pos,
+              const float* __restrict__ posdot, const int* __restrict__ t_ptr,
+              const int* __restrict__ t_dst, const float* __restrict__ W,
+              const float* __restrict__ Wdot, const float* __restrict__ gout, int N,
+              float* grad_x) {
+  __shared__ USmem<KP> sm;
+  const long long gw = (long long)blockIdx.x * WARPS_PER_CTA + (threadIdx.x >> 5);
+  const int j = (int)(gw / T.n);
+  const int task = (int)(gw % T.n);
+  if (j >= N) return;
+  const int bi = T.a[task];
+  const int lane = threadIdx.x & 31;
+  const int u = T.b[task] * 32 + lane;
+  const int c = BP.c[bi];
+  const bool act = u < c;
+  float acc[7];
+#pragma unroll
+  for (int k = 0; k < 7; ++k) acc[k] = 0.f;
+  for (int k = 0; k < BP.count[bi]; ++k) {
+    const DevPath& p = P.p[BP.list[bi][k]];
+    dispatch_type(p.type, [&](auto tr) {
+      using TR = decltype(tr);
+      uvu_src_body<TR::li, TR::ls, TR::lo, KP, MODE>(P, p, u, act, j, pos, posdot, t_ptr, t_dst, W,
+                                                     Wdot, gout, acc, sm);
+    });
+  }
+  if (!act) return;
+  const int ri = 2 * BP.l[bi] + 1;
+  float* dst = grad_x + (long long)j * P.dim_in + BP.off[bi] + u;
+#pragma unroll
+  for (int k = 0; k < 7; ++k)
+    if (k < ri) dst[k * c] = acc[k];
+}
+
+// ---------------------------------------------------------------------------
+// runners, explicitly instantiated per translation unit
+// ---------------------------------------------------------------------------
+
+static inline unsigned ugrid(long long warps) {
+  return (unsigned)((warps + WARPS_PER_CTA - 1) / WARPS_PER_CTA);
+}
+
+template <int KP, int MODE>
+cudaError_t run_uvu_fwd(const DevPlan& P, const BlockPaths& BP, const Tasks& T, const float* x,
+                        const float* xdot, const float* pos, const float* posdot,
+                        const int* row_ptr, const int* src, const float* W, const float* Wdot,
+                        int N, float* out, cudaStream_t s) {
+  k_uvu_fwd<KP, MODE><<<ugrid((long long)N * T.n), WARPS_PER_CTA * 32, 0, s>>>(
+      P, BP, T, x, xdot, pos, posdot, row_ptr, src, W, Wdot, N, out);
+  return cudaGetLastError();
+}
+
+template <int KP>
+cudaError_t run_uvu_recv_bwd(const DevPlan& P, const Tasks& T, const float* x, const float* pos,
+                             const int* row_ptr, const int* src, const float* W,
+                             const float* grad_out, int N, float4* gbuf, cudaStream_t s) {
+  k_uvu_recv_bwd<KP><<<ugrid(N), WARPS_PER_CTA * 32, 0, s>>>(P, T, x, pos, row_ptr, src, W,
+                                                            grad_out, N, gbuf);
+  return cudaGetLastError();
+}
+
+template <int KP, int MODE>
+cudaError_t run_uvu_gradw(const DevPlan& P, const Tasks& T, const float* x, const float* xdot,
+                          const float* pos, const float* posdot, const int* row_ptr,
+                          const int* src, const float* grad_out, int N, int n_ranges,
+                          float* partial, cudaStream_t s) {
+  k_uvu_gradw<KP, MODE><<<ugrid((long long)n_ranges * T.n), WARPS_PER_CTA * 32, 0, s>>>(
+      P, T, x, xdot, pos, posdot, row_ptr, src, grad_out, N, n_ranges, partial);
+  return cudaGetLastError();
+}
+
+template <int KP, int MODE>
+cudaError_t run_uvu_src(const DevPlan& P, const BlockPaths& BP, const Tasks& T, const float* pos,
+                        const float* posdot, const int* t_ptr, const int* t_dst, const float* W,
+                        const float* Wdot, const float* grad_out, int N, float* grad_x,
+                        cudaStream_t s) {
+  k_uvu_src<KP, MODE><<<ugrid((long long)N * T.n), WARPS_PER_CTA * 32, 0, s>>>(
+      P, BP, T, pos, posdot, t_ptr, t_dst, W, Wdot, grad_out, N, grad_x);
+  return cudaGetLastError();
+}
+
+#if defined(TPC_UNIT_KP) && defined(TPC_UNIT_MODE) && defined(TPC_UNIT_PART)
+#define TPC_PART_STATE 1
+#define TPC_PART_SRC 2
+#define TPC_PART_RECV 3
+#define TPC_PART_FWD 4
+#define TPC_PART_GRADW 5
+#if TPC_UNIT_PART == TPC_PART_FWD
+template cudaError_t run_uvu_fwd<TPC_UNIT_KP, TPC_UNIT_MODE>(
+    const DevPlan&, const BlockPaths&, const Tasks&, const float*, const float*, const float*,
+    const float*, const int*, const int*, const float*, const float*, int, float*, cudaStream_t);
+#endif
+#if TPC_UNIT_PART == TPC_PART_GRADW
+template cudaError_t run_uvu_gradw<TPC_UNIT_KP, TPC_UNIT_MODE>(
+    const DevPlan&, const Tasks&, const float*, const float*, const float*, const float*,
+    const int*, const int*, const float*, int, int, float*, cudaStream_t);
+#endif
+#if TPC_UNIT_PART == TPC_PART_SRC
+template cudaError_t run_uvu_src<TPC_UNIT_KP, TPC_UNIT_MODE>(
+    const DevPlan&, const BlockPaths&, const Tasks&, const float*, const float*, const int*,
+    const int*, const float*, const float*, const float*, int, float*, cudaStream_t);
+#endif
+#if TPC_UNIT_PART == TPC_PART_RECV
+template cudaError_t run_uvu_recv_bwd<TPC_UNIT_KP>(const DevPlan&, const Tasks&, const float*,
+                                                   const float*, const int*, const int*,
+                                                   const float*, const float*, int, float4*,
+                                                   cudaStream_t);
+#endif
+#endif
+
+}  // namespace tpc

@@ -1,0 +1,489 @@
+// Fully connected (uvw) streaming kernels.
+//
+// Sobek: Streaming Equivariant Tensor Product Convolutions, section 4.
+//  * k_uvw_state      -- receiver traversal building the state of eq. 33,
+//                        S_{i,pi,q,u,mo} = sum_j phi_{ij,q} C_{pi,u,mo}(x_j, Y_ij),
+//                        or (double backward) its directional derivative dS along
+//                        (x_dot, pos_dot) as used in eq. 37/39.
+//  * k_uvw_recv_bwd   -- receiver traversal differentiating eq. 33 given S_bar = m_bar A^T
+//                        (eq. 36): per edge phi_bar (eq. 20) and Y_bar (eq. 22), carried
+//                        to the edge vector r_e and staged per edge for the positions.
+//  * k_uvw_src_state  -- source traversal (source-contiguous CSR owns x_bar):
+//                        X_{j,pi,q,w,mi} = sum_{e out of j} phi_{e,q} U_{e,pi,w,mi},
+//                        U = adjoint of the coupling in x applied to m_bar of the
+//                        receiver; then x_bar = X A^T (eq. 21) and A_bar = x^T X (eq. 19).
+//
+// One warp owns one (node, path, 32-channel chunk) task; lane = channel.  Edge
+// geometry, harmonics and radial values are computed lane-per-edge for 32 edges at a
+// time and broadcast through shared memory.  Per-lane state lives in registers and is
+// written once to the caller's workspace; nothing is accumulated with atomics.
+#include "common.cuh"
+
+namespace tpc {
+
+template <int KP>
+struct GeoSmem {
+  int j[WARPS_PER_CTA][32];
+  float Y[WARPS_PER_CTA][32][8];
+  float phi[WARPS_PER_CTA][32][KP];
+  float Yd[WARPS_PER_CTA][32][8];
+  float phid[WARPS_PER_CTA][32][KP];
+};
+
+// lane-per-edge preparation for one path's harmonic block (and optional tangents)
+template <int LS, int KP, bool TAN>
+__device__ __forceinline__ void prep_edge(const DevPlan& P, const float* __restrict__ pos,
+                                          const float* __restrict__ posdot, int i, int j,
+                                          int store, GeoSmem<KP>& sm, int w, int lane) {
+  constexpr int RS = 2 * LS + 1;
+  const EdgeGeo g = edge_geo(pos, i, j);
+  const Pow3 pw(g.ux, g.uy, g.uz);
+  float Y[RS];
+  sh_block<LS>(pw, Y);
+  float phi[KP], dphi[KP];
+  radial<KP, TAN>(P, g.d, phi, dphi);
+  sm.j[w][lane] = store;
+#pragma unroll
+  for (int k = 0; k < RS; ++k) sm.Y[w][lane][k] = Y[k];
+#pragma unroll
+  for (int q = 0; q < KP; ++q) sm.phi[w][lane][q] = phi[q];
+  if (TAN) {
+    float vx = 0.f, vy = 0.f, vz = 0.f;
+    if (posdot) {
+      vx = __ldg(posdot + 3 * j) - __ldg(posdot + 3 * i);
+      vy = __ldg(posdot + 3 * j + 1) - __ldg(posdot + 3 * i + 1);
+      vz = __ldg(posdot + 3 * j + 2) - __ldg(posdot + 3 * i + 2);
+    }
+    const float s = g.ux * vx + g.uy * vy + g.uz * vz;     // d|r| along r_dot
+    const float tx = (vx - s * g.ux) * g.inv_d;            // d r_hat along r_dot
+    const float ty = (vy - s * g.uy) * g.inv_d;
+    const float tz = (vz - s * g.uz) * g.inv_d;
+    float Yd[RS];
+    sh_block_dir<LS>(pw, tx, ty, tz, Yd);
+#pragma unroll
+    for (int k = 0; k < RS; ++k) sm.Yd[w][lane][k] = Yd[k];
+#pragma unroll
+    for (int q = 0; q < KP; ++q) sm.phid[w][lane][q] = dphi[q] * s;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// receiver state (eq. 33) and its tangent
+// ---------------------------------------------------------------------------
+
+template <int LI, int LS, int LO, int KP, int MODE>
+__device__ __forceinline__ void uvw_state_body(const DevPlan& P, const DevPath& p, int chunk, int i,
+                                               int node_local, const float* __restrict__ x,
+                                               const float* __restrict__ xdot,
+                                               const float* __restrict__ pos,
+                                               const float* __restrict__ posdot,
+                                               const int* __restrict__ row_ptr,
+                                               const int* __restrict__ src, float* S, float* Sd,
+                                               GeoSmem<KP>& sm) {
+  constexpr int RI = 2 * LI + 1, RS = 2 * LS + 1, RO = 2 * LO + 1;
+  constexpr bool TAN = MODE == 1;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int u = chunk * 32 + lane;
+  const bool act = u < p.c_in;
+  const float* xb = x + p.in_off + (act ? u : 0);
+  const float* xdb = xdot ? xdot + p.in_off + (act ? u : 0) : nullptr;
+  float acc[KP][RO], acc0[KP][RO];
+#pragma unroll
+  for (int q = 0; q < KP; ++q)
+#pragma unroll
+    for (int o = 0; o < RO; ++o) { acc[q][o] = 0.f; acc0[q][o] = 0.f; }
+
+  const int eb = __ldg(row_ptr + i), ee = __ldg(row_ptr + i + 1);
+  for (int e0 = eb; e0 < ee; e0 += 32) {
+    const int ne = min(32, ee - e0);
+    if (lane < ne) {
+      const int j = __ldg(src + e0 + lane);
+      prep_edge<LS, KP, TAN>(P, pos, posdot, i, j, j, sm, w, lane);
+    }
+    __syncwarp();
+    for (int t = 0; t < ne; ++t) {
+      const long long row = (long long)sm.j[w][t] * P.dim_in;
+      float xv[RI];
+#pragma unroll
+      for (int m = 0; m < RI; ++m) xv[m] = act ? __ldg(xb + row + m * p.c_in) : 0.f;
+      float Y[RS], phi[KP];
+#pragma unroll
+      for (int k = 0; k < RS; ++k) Y[k] = sm.Y[w][t][k];
+#pragma unroll
+      for (int q = 0; q < KP; ++q) phi[q] = sm.phi[w][t][q];
+      float C[RO];
+      cg_couple<LI, LS, LO>(xv, Y, C);
+      if (!TAN) {
+#pragma unroll
+        for (int q = 0; q < KP; ++q)
+#pragma unroll
+          for (int o = 0; o < RO; ++o) acc[q][o] = fmaf(phi[q], C[o], acc[q][o]);
+      } else {
+        float Yd[RS], phid[KP], Cd[RO], C2[RO];
+#pragma unroll
+        for (int k = 0; k < RS; ++k) Yd[k] = sm.Yd[w][t][k];
+#pragma unroll
+        for (int q = 0; q < KP; ++q) phid[q] = sm.phid[w][t][q];
+        cg_couple<LI, LS, LO>(xv, Yd, Cd);
+        if (xdb) {
+          float xdv[RI];
+#pragma unroll
+          for (int m = 0; m < RI; ++m) xdv[m] = act ? __ldg(xdb + row + m * p.c_in) : 0.f;
+          cg_couple<LI, LS, LO>(xdv, Y, C2);
+#pragma unroll
+          for (int o = 0; o < RO; ++o) Cd[o] += C2[o];
+        }
+#pragma unroll
+        for (int q = 0; q < KP; ++q)
+#pragma unroll
+          for (int o = 0; o < RO; ++o) {
+            acc[q][o] = fmaf(phid[q], C[o], fmaf(phi[q], Cd[o], acc[q][o]));
+            acc0[q][o] = fmaf(phi[q], C[o], acc0[q][o]);
+          }
+      }
+    }
+    __syncwarp();
+  }
+  if (!act) return;
+  const long long base = (long long)node_local * P.state_per_node + p.st_off + u;
+  const int rs = P.K * p.c_in;
+  float* out = TAN ? Sd : S;
+#pragma unroll
+  for (int o = 0; o < RO; ++o)
+#pragma unroll
+    for (int q = 0; q < KP; ++q)
+      if (q < P.K) out[base + (long long)o * rs + q * p.c_in] = acc[q][o];
+  if (TAN && S) {
+#pragma unroll
+    for (int o = 0; o < RO; ++o)
+#pragma unroll
+      for (int q = 0; q < KP; ++q)
+        if (q < P.K) S[base + (long long)o * rs + q * p.c_in] = acc0[q][o];
+  }
+}
+
+template <int KP, int MODE>
+__global__ void __launch_bounds__(WARPS_PER_CTA * 32)
+    k_uvw_state(DevPlan P, Tasks T, const float* __restrict__ x, const float* __restrict__ xdot,
+                const float* __restrict__ pos, const float* __restrict__ posdot,
+                const int* __restrict__ row_ptr, const int* __restrict__ src, int node0,
+                int n_nodes, float* S, float* Sd) {
+  __shared__ GeoSmem<KP> sm;
+  const long long gw = (long long)blockIdx.x * WARPS_PER_CTA + (threadIdx.x >> 5);
+  const int node_local = (int)(gw / T.n);
+  const int task = (int)(gw % T.n);
+  if (node_local >= n_nodes) return;
+  const DevPath& p = P.p[T.a[task]];
+  const int chunk = T.b[task];
+  const int i = node0 + node_local;
+  dispatch_type(p.type, [&](auto tr) {
+    using TR = decltype(tr);
+    uvw_state_body<TR::li, TR::ls, TR::lo, KP, MODE>(P, p, chunk, i, node_local, x, xdot, pos,
+                                                     posdot, row_ptr, src, S, Sd, sm);
+  });
+}
+
+// ---------------------------------------------------------------------------
+// receiver backward: phi_bar and Y_bar per edge -> d L / d r_e
+// ---------------------------------------------------------------------------
+
+template <int KP>
+struct RecvSmem {
+  int j[WARPS_PER_CTA][32];
+  float Y[WARPS_PER_CTA][32][16];
+  float phi[WARPS_PER_CTA][32][KP];
+  float accY[WARPS_PER_CTA][32][16];
+  float accphi[WARPS_PER_CTA][32][KP];
+};
+
+template <int LI, int LS, int LO, int KP>
+__device__ __forceinline__ void uvw_recv_body(const DevPlan& P, const DevPath& p, int chunk,
+                                              int node_local, int ne,
+                                              const float* __restrict__ x,
+                                              const float* __restrict__ Sbar, RecvSmem<KP>& sm) {
+  constexpr int RI = 2 * LI + 1, RS = 2 * LS + 1, RO = 2 * LO + 1;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int u = chunk * 32 + lane;
+  const bool act = u < p.c_in;
+  const float* xb = x + p.in_off + (act ? u : 0);
+  float sb[KP][RO];
+  {
+    const long long base = (long long)node_local * P.state_per_node + p.st_off + u;
+    const int rs = P.K * p.c_in;
+#pragma unroll
+    for (int o = 0; o < RO; ++o)
+#pragma unroll
+      for (int q = 0; q < KP; ++q)
+        sb[q][o] = (act && q < P.K) ? Sbar[base + (long long)o * rs + q * p.c_in] : 0.f;
+  }
+  const int yw = reduce_multi_index<8>(lane), pw_ = reduce_multi_index<KP>(lane);
+  const bool ywr = reduce_multi_writer<8>(lane), pwr = reduce_multi_writer<KP>(lane);
+  for (int t = 0; t < ne; ++t) {
+    const long long row = (long long)sm.j[w][t] * P.dim_in;
+    float xv[RI];
+#pragma unroll
+    for (int m = 0; m < RI; ++m) xv[m] = act ? __ldg(xb + row + m * p.c_in) : 0.f;
+    float Y[RS], phi[KP];
+#pragma unroll
+    for (int k = 0; k < RS; ++k) Y[k] = sm.Y[w][t][LS * LS + k];
+#pragma unroll
+    for (int q = 0; q < KP; ++q) phi[q] = sm.phi[w][t][q];
+    float C[RO];
+    cg_couple<LI, LS, LO>(xv, Y, C);
+    float pp[KP];
+#pragma unroll
+    for (int q = 0; q < KP; ++q) {
+      float s = 0.f;
+#pragma unroll
+      for (int o = 0; o < RO; ++o) s = fmaf(sb[q][o], C[o], s);
+      pp[q] = s;
+    }
+    float Tb[RO];
+#pragma unroll
+    for (int o = 0; o < RO; ++o) {
+      float s = 0.f;
+#pragma unroll
+      for (int q = 0; q < KP; ++q) s = fmaf(phi[q], sb[q][o], s);
+      Tb[o] = s;
+    }
+    float py[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) py[k] = 0.f;
+    cg_adj_y<LI, LS, LO>(xv, Tb, py);
+    const float rphi = warp_reduce_multi<KP>(pp);
+    const float ry = warp_reduce_multi<8>(py);
+    if (pwr) sm.accphi[w][t][pw_] += rphi;
+    if (ywr && yw < RS) sm.accY[w][t][LS * LS + yw] += ry;
+    __syncwarp();
+  }
+}
+
+template <int KP>
+__global__ void __launch_bounds__(WARPS_PER_CTA * 32)
+    k_uvw_recv_bwd(DevPlan P, Tasks T, const float* __restrict__ x, const float* __restrict__ pos,
+                   const int* __restrict__ row_ptr, const int* __restrict__ src,
+                   const float* __restrict__ Sbar, int node0, int n_nodes, float4* gbuf) {
+  __shared__ RecvSmem<KP> sm;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int node_local = blockIdx.x * WARPS_PER_CTA + w;
+  if (node_local >= n_nodes) return;
+  const int i = node0 + node_local;
+  const int eb = __ldg(row_ptr + i), ee = __ldg(row_ptr + i + 1);
+  for (int e0 = eb; e0 < ee; e0 += 32) {
+    const int ne = min(32, ee - e0);
+    if (lane < ne) {
+      const int j = __ldg(src + e0 + lane);
+      const EdgeGeo g = edge_geo(pos, i, j);
+      const Pow3 pw(g.ux, g.uy, g.uz);
+      float Y[16], phi[KP], dphi[KP];
+      sh_all(pw, Y);
+      radial<KP, false>(P, g.d, phi, dphi);
+      sm.j[w][lane] = j;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) { sm.Y[w][lane][k] = Y[k]; sm.accY[w][lane][k] = 0.f; }
+#pragma unroll
+      for (int q = 0; q < KP; ++q) { sm.phi[w][lane][q] = phi[q]; sm.accphi[w][lane][q] = 0.f; }
+    }
+    __syncwarp();
+    for (int task = 0; task < T.n; ++task) {
+      const DevPath& p = P.p[T.a[task]];
+      const int chunk = T.b[task];
+      dispatch_type(p.type, [&](auto tr) {
+        using TR = decltype(tr);
+        uvw_recv_body<TR::li, TR::ls, TR::lo, KP>(P, p, chunk, node_local, ne, x, Sbar, sm);
+      });
+    }
+    __syncwarp();
+    if (lane < ne) {
+      const int j = sm.j[w][lane];
+      const EdgeGeo g = edge_geo(pos, i, j);
+      const Pow3 pw(g.ux, g.uy, g.uz);
+      float phi[KP], dphi[KP], Yb[16];
+      radial<KP, true>(P, g.d, phi, dphi);
+#pragma unroll
+      for (int k = 0; k < 16; ++k) Yb[k] = sm.accY[w][lane][k];
+      float vx = 0.f, vy = 0.f, vz = 0.f;
+      sh_vjp_all(pw, Yb, vx, vy, vz);
+      const float vr = vx * g.ux + vy * g.uy + vz * g.uz;
+      float s = 0.f;
+#pragma unroll
+      for (int q = 0; q < KP; ++q) s = fmaf(sm.accphi[w][lane][q], dphi[q], s);
+      float4 out;
+      out.x = (vx - vr * g.ux) * g.inv_d + s * g.ux;
+      out.y = (vy - vr * g.uy) * g.inv_d + s * g.uy;
+      out.z = (vz - vr * g.uz) * g.inv_d + s * g.uz;
+      out.w = 0.f;
+      gbuf[e0 + lane] = out;
+    }
+    __syncwarp();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// source state X (and its tangent for the double backward)
+// ---------------------------------------------------------------------------
+
+template <int LI, int LS, int LO, int KP, int MODE>
+__device__ __forceinline__ void uvw_src_body(const DevPlan& P, const DevPath& p, int chunk, int j,
+                                             int node_local, const float* __restrict__ pos,
+                                             const float* __restrict__ posdot,
+                                             const int* __restrict__ t_ptr,
+                                             const int* __restrict__ t_dst,
+                                             const float* __restrict__ gout, float* X, float* Xd,
+                                             GeoSmem<KP>& sm) {
+  constexpr int RI = 2 * LI + 1, RS = 2 * LS + 1, RO = 2 * LO + 1;
+  constexpr bool TAN = MODE == 1;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = chunk * 32 + lane;
+  const bool act = c < p.c_out;
+  const float* gb = gout + p.out_off + (act ? c : 0);
+  float acc[KP][RI], acc0[KP][RI];
+#pragma unroll
+  for (int q = 0; q < KP; ++q)
+#pragma unroll
+    for (int m = 0; m < RI; ++m) { acc[q][m] = 0.f; acc0[q][m] = 0.f; }
+  const int kb = __ldg(t_ptr + j), ke = __ldg(t_ptr + j + 1);
+  for (int k0 = kb; k0 < ke; k0 += 32) {
+    const int ne = min(32, ke - k0);
+    // edge j -> i seen from its source: r = pos[j] - pos[i]; keep the receiver index
+    if (lane < ne) {
+      const int i = __ldg(t_dst + k0 + lane);
+      prep_edge<LS, KP, TAN>(P, pos, posdot, i, j, i, sm, w, lane);
+    }
+    __syncwarp();
+    for (int t = 0; t < ne; ++t) {
+      const long long row = (long long)sm.j[w][t] * P.dim_out;
+      float mb[RO];
+#pragma unroll
+      for (int o = 0; o < RO; ++o) mb[o] = act ? __ldg(gb + row + o * p.c_out) : 0.f;
+      float Y[RS], phi[KP];
+#pragma unroll
+      for (int k = 0; k < RS; ++k) Y[k] = sm.Y[w][t][k];
+#pragma unroll
+      for (int q = 0; q < KP; ++q) phi[q] = sm.phi[w][t][q];
+      float U[RI];
+      cg_adj_x<LI, LS, LO>(Y, mb, U);
+      if (!TAN) {
+#pragma unroll
+        for (int q = 0; q < KP; ++q)
+#pragma unroll
+          for (int m = 0; m < RI; ++m) acc[q][m] = fmaf(phi[q], U[m], acc[q][m]);
+      } else {
+        float Yd[RS], phid[KP], Ud[RI];
+#pragma unroll
+        for (int k = 0; k < RS; ++k) Yd[k] = sm.Yd[w][t][k];
+#pragma unroll
+        for (int q = 0; q < KP; ++q) phid[q] = sm.phid[w][t][q];
+        cg_adj_x<LI, LS, LO>(Yd, mb, Ud);
+#pragma unroll
+        for (int q = 0; q < KP; ++q)
+#pragma unroll
+          for (int m = 0; m < RI; ++m) {
+            acc[q][m] = fmaf(phid[q], U[m], fmaf(phi[q], Ud[m], acc[q][m]));
+            acc0[q][m] = fmaf(phi[q], U[m], acc0[q][m]);
+          }
+      }
+    }
+    __syncwarp();
+  }
+  if (!act) return;
+  const long long base = (long long)node_local * P.xstate_per_node + p.xst_off + c;
+  const int rs = P.K * p.c_out;
+  float* out = TAN ? Xd : X;
+#pragma unroll
+  for (int m = 0; m < RI; ++m)
+#pragma unroll
+    for (int q = 0; q < KP; ++q)
+      if (q < P.K) out[base + (long long)m * rs + q * p.c_out] = acc[q][m];
+  if (TAN && X) {
+#pragma unroll
+    for (int m = 0; m < RI; ++m)
+#pragma unroll
+      for (int q = 0; q < KP; ++q)
+        if (q < P.K) X[base + (long long)m * rs + q * p.c_out] = acc0[q][m];
+  }
+}
+
+template <int KP, int MODE>
+__global__ void __launch_bounds__(WARPS_PER_CTA * 32)
+    k_uvw_src_state(DevPlan P, Tasks T, const float* __restrict__ pos,
+                    const float* __restrict__ posdot, const int* __restrict__ t_ptr,
+                    const int* __restrict__ t_dst, const float* __restrict__ gout, int node0,
+                    int n_nodes, float* X, float* Xd) {
+  __shared__ GeoSmem<KP> sm;
+  const long long gw = (long long)blockIdx.x * WARPS_PER_CTA + (threadIdx.x >> 5);
+  const int node_local = (int)(gw / T.n);
+  const int task = (int)(gw % T.n);
+  if (node_local >= n_nodes) return;
+  const DevPath& p = P.p[T.a[task]];
+  const int chunk = T.b[task];
+  const int j = node0 + node_local;
+  dispatch_type(p.type, [&](auto tr) {
+    using TR = decltype(tr);
+    uvw_src_body<TR::li, TR::ls, TR::lo, KP, MODE>(P, p, chunk, j, node_local, pos, posdot, t_ptr,
+                                                   t_dst, gout, X, Xd, sm);
+  });
+}
+
+// ---------------------------------------------------------------------------
+// runners, explicitly instantiated per translation unit
+// ---------------------------------------------------------------------------
+
+static inline unsigned grid_for(long long warps) {
+  return (unsigned)((warps + WARPS_PER_CTA - 1) / WARPS_PER_CTA);
+}
+
+template <int KP, int MODE>
+cudaError_t run_uvw_state(const DevPlan& P, const Tasks& T, const float* x, const float* xdot,
+                          const float* pos, const float* posdot, const int* row_ptr,
+                          const int* src, int node0, int n_nodes, float* S, float* Sdot,
+                          cudaStream_t s) {
+  k_uvw_state<KP, MODE><<<grid_for((long long)n_nodes * T.n), WARPS_PER_CTA * 32, 0, s>>>(
+      P, T, x, xdot, pos, posdot, row_ptr, src, node0, n_nodes, S, Sdot);
+  return cudaGetLastError();
+}
+
+template <int KP>
+cudaError_t run_uvw_recv_bwd(const DevPlan& P, const Tasks& T, const float* x, const float* pos,
+                             const int* row_ptr, const int* src, const float* Sbar, int node0,
+                             int n_nodes, float4* gbuf, cudaStream_t s) {
+  k_uvw_recv_bwd<KP><<<grid_for(n_nodes), WARPS_PER_CTA * 32, 0, s>>>(P, T, x, pos, row_ptr, src,
+                                                                     Sbar, node0, n_nodes, gbuf);
+  return cudaGetLastError();
+}
+
+template <int KP, int MODE>
+cudaError_t run_uvw_src_state(const DevPlan& P, const Tasks& T, const float* pos,
+                              const float* posdot, const int* t_ptr, const int* t_dst,
+                              const float* grad_out, int node0, int n_nodes, float* X,
+                              float* Xdot, cudaStream_t s) {
+  k_uvw_src_state<KP, MODE><<<grid_for((long long)n_nodes * T.n), WARPS_PER_CTA * 32, 0, s>>>(
+      P, T, pos, posdot, t_ptr, t_dst, grad_out, node0, n_nodes, X, Xdot);
+  return cudaGetLastError();
+}
+
+#if defined(TPC_UNIT_KP) && defined(TPC_UNIT_MODE) && defined(TPC_UNIT_PART)
+#define TPC_PART_STATE 1
+#define TPC_PART_SRC 2
+#define TPC_PART_RECV 3
+#define TPC_PART_FWD 4
+#define TPC_PART_GRADW 5
+#if TPC_UNIT_PART == TPC_PART_STATE
+template cudaError_t run_uvw_state<TPC_UNIT_KP, TPC_UNIT_MODE>(
+    const DevPlan&, const Tasks&, const float*, const float*, const float*, const float*,
+    const int*, const int*, int, int, float*, float*, cudaStream_t);
+#endif
+#if TPC_UNIT_PART == TPC_PART_SRC
+template cudaError_t run_uvw_src_state<TPC_UNIT_KP, TPC_UNIT_MODE>(
+    const DevPlan&, const Tasks&, const float*, const float*, const int*, const int*,
+    const float*, int, int, float*, float*, cudaStream_t);
+#endif
+#if TPC_UNIT_PART == TPC_PART_RECV
+template cudaError_t run_uvw_recv_bwd<TPC_UNIT_KP>(const DevPlan&, const Tasks&, const float*,
+                                                   const float*, const int*, const int*,
+                                                   const float*, int, int, float4*,
+                                                   cudaStream_t);
+#endif
+#endif
+
+}  // namespace tpc

@@ -1,0 +1,74 @@
+// Dispatch of the streaming kernels on the padded radial size KP (8 or 16) and on the
+// pass mode (0: primal, 1: tangent for the double backward).
+#include "internal.h"
+
+namespace tpc {
+
+#define TPC_BY_KP_MODE(RUN, ...)                                      \
+  if (P.K <= 8) return mode == 0 ? RUN<8, 0>(__VA_ARGS__) : RUN<8, 1>(__VA_ARGS__); \
+  return mode == 0 ? RUN<16, 0>(__VA_ARGS__) : RUN<16, 1>(__VA_ARGS__);
+
+cudaError_t launch_uvw_state(const DevPlan& P, const Tasks& T, int mode, const float* x,
+                             const float* xdot, const float* pos, const float* posdot,
+                             const int* row_ptr, const int* src, int node0, int n_nodes,
+                             float* S, float* Sdot, cudaStream_t s) {
+  if (n_nodes <= 0 || T.n == 0) return cudaSuccess;
+  TPC_BY_KP_MODE(run_uvw_state, P, T, x, xdot, pos, posdot, row_ptr, src, node0, n_nodes, S, Sdot, s)
+}
+
+cudaError_t launch_uvw_recv_bwd(const DevPlan& P, const Tasks& T, const float* x,
+                                const float* pos, const int* row_ptr, const int* src,
+                                const float* Sbar, int node0, int n_nodes, float4* gbuf,
+                                cudaStream_t s) {
+  if (n_nodes <= 0) return cudaSuccess;
+  if (P.K <= 8) return run_uvw_recv_bwd<8>(P, T, x, pos, row_ptr, src, Sbar, node0, n_nodes, gbuf, s);
+  return run_uvw_recv_bwd<16>(P, T, x, pos, row_ptr, src, Sbar, node0, n_nodes, gbuf, s);
+}
+
+cudaError_t launch_uvw_src_state(const DevPlan& P, const Tasks& T, int mode,
+                                 const float* pos, const float* posdot, const int* t_ptr,
+                                 const int* t_eid, const int* t_dst, const float* grad_out,
+                                 int node0, int n_nodes, float* X, float* Xdot,
+                                 cudaStream_t s) {
+  (void)t_eid;
+  if (n_nodes <= 0 || T.n == 0) return cudaSuccess;
+  TPC_BY_KP_MODE(run_uvw_src_state, P, T, pos, posdot, t_ptr, t_dst, grad_out, node0, n_nodes, X, Xdot, s)
+}
+
+cudaError_t launch_uvu_fwd(const DevPlan& P, const BlockPaths& BP, const Tasks& T, int mode,
+                           const float* x, const float* xdot, const float* pos,
+                           const float* posdot, const int* row_ptr, const int* src,
+                           const float* W, const float* Wdot, int N, float* out,
+                           cudaStream_t s) {
+  if (N <= 0 || T.n == 0) return cudaSuccess;
+  TPC_BY_KP_MODE(run_uvu_fwd, P, BP, T, x, xdot, pos, posdot, row_ptr, src, W, Wdot, N, out, s)
+}
+
+cudaError_t launch_uvu_recv_bwd(const DevPlan& P, const Tasks& T, const float* x,
+                                const float* pos, const int* row_ptr, const int* src,
+                                const float* W, const float* grad_out, int N, float4* gbuf,
+                                cudaStream_t s) {
+  if (N <= 0) return cudaSuccess;
+  if (P.K <= 8) return run_uvu_recv_bwd<8>(P, T, x, pos, row_ptr, src, W, grad_out, N, gbuf, s);
+  return run_uvu_recv_bwd<16>(P, T, x, pos, row_ptr, src, W, grad_out, N, gbuf, s);
+}
+
+cudaError_t launch_uvu_gradw(const DevPlan& P, const Tasks& T, int mode, const float* x,
+                             const float* xdot, const float* pos, const float* posdot,
+                             const int* row_ptr, const int* src, const float* grad_out,
+                             int N, int n_ranges, float* partial, cudaStream_t s) {
+  if (N <= 0 || T.n == 0) return cudaSuccess;
+  TPC_BY_KP_MODE(run_uvu_gradw, P, T, x, xdot, pos, posdot, row_ptr, src, grad_out, N, n_ranges, partial, s)
+}
+
+cudaError_t launch_uvu_src(const DevPlan& P, const BlockPaths& BP, const Tasks& T, int mode,
+                           const float* pos, const float* posdot, const int* t_ptr,
+                           const int* t_eid, const int* t_dst, const float* W,
+                           const float* Wdot, const float* grad_out, int N, float* grad_x,
+                           cudaStream_t s) {
+  (void)t_eid;
+  if (N <= 0 || T.n == 0) return cudaSuccess;
+  TPC_BY_KP_MODE(run_uvu_src, P, BP, T, pos, posdot, t_ptr, t_dst, W, Wdot, grad_out, N, grad_x, s)
+}
+
+}  // namespace tpc

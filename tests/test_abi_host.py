@@ -1,0 +1,151 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+* the shared library loads and exports every function declared in include/tpconv.h;
+* the plan builder enumerates the same paths, widths and weight offsets as the oracle
+  and its coupling tables (computed by a different algorithm at build time) equal the
+  oracle's to 1e-12;
+* argument errors are reported before anything is launched.
+"""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from equivariant_gnn_tensor_dst_b200 import binding
+from equivariant_gnn_tensor_dst_b200.workloads import CONFIGS
+from oracle import conv, radial
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    txt = open(os.path.join(ROOT, "include", "tpconv.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(tpconv_\w+)\s*\(", txt)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = binding.lib()
+    names = _declared()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(binding.SIGNATURES)
+
+
+def _oracle_plan(cfg):
+    c = CONFIGS[cfg]
+    rs = radial.RadialSpec(c.radial, c.num_basis, c.r_cut, c.r_min, c.r_max)
+    return conv.make_plan(c.irreps_in, c.sh_lmax, c.irreps_out, c.mode, rs)
+
+
+def _lib_plan(cfg):
+    c = CONFIGS[cfg]
+    return binding.Plan(c.irreps_in, c.sh_lmax, c.irreps_out, c.mode, c.radial, c.num_basis, c.r_cut,
+                        c.r_min, c.r_max)
+
+
+@pytest.mark.parametrize("cfg", sorted(CONFIGS))
+def test_plan_matches_oracle(cfg):
+    op, lp = _oracle_plan(cfg), _lib_plan(cfg)
+    assert (lp.dim_in, lp.dim_out, lp.weight_cols, lp.num_basis) == (op.dim_in, op.dim_out, op.n_w,
+                                                                     op.radial.num_basis)
+    assert lp.num_paths == len(op.paths)
+    for i, p in enumerate(op.paths):
+        q = lp.path(i)
+        assert (q["l_in"], q["l_sh"], q["l_out"], q["block_in"], q["block_out"], q["c_in"], q["c_out"],
+                q["w_offset"], q["w_count"]) == (p.l_in, p.l_sh, p.l_out, p.block_in, p.block_out, p.c_in,
+                                                 p.c_out, p.w_offset, p.w_count)
+        idx, val = lp.coupling(i)
+        dense = np.zeros_like(op.coupling[i])
+        for (a, b, c), v in zip(idx, val):
+            dense[a, b, c] = v
+        assert np.abs(dense - op.coupling[i]).max() < 1e-12
+    assert np.array_equal(lp.fan_in_per_column(), op.fan_in_per_column())
+
+
+def test_plan_general_parities_match_oracle():
+    rs = radial.RadialSpec(radial.BESSEL, 6, 2.5)
+    ii, io = "2x0e+2x1o+1x1e+1x3o", "2x0e+1x1e+2x1o+1x2e+1x2o+1x3e"
+    op = conv.make_plan(ii, 3, io, "uvw", rs)
+    lp = binding.Plan(ii, 3, io, "uvw", "bessel", 6, 2.5)
+    assert lp.num_paths == len(op.paths)
+    for i, p in enumerate(op.paths):
+        idx, val = lp.coupling(i)
+        dense = np.zeros_like(op.coupling[i])
+        for (a, b, c), v in zip(idx, val):
+            dense[a, b, c] = v
+        assert np.abs(dense - op.coupling[i]).max() < 1e-12
+
+
+@pytest.mark.parametrize("args,code", [
+    (("4x0q", 2, "4x0e", "uvw"), 2),
+    (("4x0e", 2, "", "uvw"), 2),
+    (("4x5e", 2, "4x0e", "uvw"), 3),
+    (("4x0e", 4, "4x0e", "uvw"), 3),
+    (("4x0e+4x1o", 1, "2x1o", "uvu"), 1),
+    (("4x0e", 0, "4x1o", "uvw"), 1),   # no valid path
+])
+def test_plan_errors(args, code):
+    with pytest.raises(binding.TPConvError) as e:
+        binding.Plan(*args)
+    assert e.value.status == code
+
+
+def test_radial_spec_errors():
+    with pytest.raises(binding.TPConvError):
+        binding.Plan("4x0e", 1, "4x0e", "uvw", "bessel", 17, 5.0)
+    with pytest.raises(binding.TPConvError):
+        binding.Plan("4x0e", 1, "4x0e", "uvw", "bessel", 8, -1.0)
+    with pytest.raises(binding.TPConvError):
+        binding.Plan("4x0e", 1, "4x0e", "uvw", "gaussian", 8, 5.0, 3.0, 1.0)
+
+
+def test_workspace_is_bounded_and_independent_of_edges():
+    lp = _lib_plan(2)
+    fwd = [lp.workspace_bytes(4096, 4096 * k, binding.PASS_FORWARD) for k in (8, 32, 128)]
+    assert fwd[0] == fwd[1] == fwd[2]
+    assert fwd[0] <= (128 << 20) + 4096
+    lp.set_workspace_budget(1 << 20)
+    assert lp.workspace_bytes(4096, 131072, binding.PASS_FORWARD) < fwd[0]
+    bwd = [lp.workspace_bytes(4096, 4096 * k, binding.PASS_BACKWARD) for k in (8, 32)]
+    # backward: bounded node state plus 16 bytes of position staging per edge
+    assert bwd[1] - bwd[0] == pytest.approx(16 * 4096 * 24, abs=512)
+
+
+def test_forward_rejects_bad_arguments_before_launch():
+    L = binding.lib()
+    lp = _lib_plan(2)
+    fake = ctypes.c_void_p(1 << 20)      # aligned, never dereferenced: the checks fail first
+    mis = ctypes.c_void_p((1 << 20) + 4)
+    ws_need = lp.workspace_bytes(100, 1000, binding.PASS_FORWARD)
+    args = [lp.handle, 100, 1000, fake, fake, fake, fake, fake, fake, fake]
+    assert L.tpconv_forward(*args, ws_need - 1, None) == 4             # workspace too small
+    assert L.tpconv_forward(lp.handle, 100, 1000, mis, fake, fake, fake, fake, fake, fake, ws_need,
+                            None) == 5                                 # misaligned
+    assert L.tpconv_forward(lp.handle, 100, 1000, None, fake, fake, fake, fake, fake, fake, ws_need,
+                            None) == 1                                 # null x
+    assert L.tpconv_forward(lp.handle, -1, 1000, fake, fake, fake, fake, fake, fake, fake, ws_need,
+                            None) == 1
+    assert L.tpconv_forward(None, 100, 1000, fake, fake, fake, fake, fake, fake, fake, ws_need,
+                            None) == 1
+    # N == 0 is a no-op
+    assert L.tpconv_forward(lp.handle, 0, 0, None, None, None, None, None, None, None, 0, None) == 0
+
+
+def test_double_backward_position_output_unsupported():
+    L = binding.lib()
+    lp = _lib_plan(5)
+    fake = ctypes.c_void_p(1 << 20)
+    st = L.tpconv_double_backward(lp.handle, 10, 20, *([fake] * 17), 1 << 30, None)
+    assert st == 3
+
+
+def test_status_strings():
+    L = binding.lib()
+    for s in range(8):
+        assert L.tpconv_status_string(s)
+    assert L.tpconv_status_string(99) == b"unknown status"
