@@ -42,7 +42,7 @@ SIGNATURES = {
     "tpconv_csr_transpose": (ctypes.c_int, [_c_i64, _c_i64] + [_c_p] * 6 + [ctypes.c_size_t, _c_p]),
     "tpconv_validate_graph": (ctypes.c_int, [_c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p]),
     "tpconv_forward": (ctypes.c_int, [_c_p, _c_i64, _c_i64] + [_c_p] * 7 + [ctypes.c_size_t, _c_p]),
-    "tpconv_backward": (ctypes.c_int, [_c_p, _c_i64, _c_i64] + [_c_p] * 14 + [ctypes.c_size_t, _c_p]),
+    "tpconv_backward": (ctypes.c_int, [_c_p, _c_i64, _c_i64] + [_c_p] * 13 + [ctypes.c_size_t, _c_p]),
     "tpconv_double_backward": (ctypes.c_int, [_c_p, _c_i64, _c_i64] + [_c_p] * 17 + [ctypes.c_size_t, _c_p]),
 }
 

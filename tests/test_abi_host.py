@@ -149,3 +149,11 @@ def test_status_strings():
     for s in range(8):
         assert L.tpconv_status_string(s)
     assert L.tpconv_status_string(99) == b"unknown status"
+
+
+def test_binding_arity_matches_header():
+    txt = open(os.path.join(ROOT, "include", "tpconv.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    for name, params in re.findall(r"\b(tpconv_\w+)\s*\(([^;{]*?)\)\s*;", txt, flags=re.S):
+        n = 0 if params.strip() in ("", "void") else params.count(",") + 1
+        assert len(binding.SIGNATURES[name][1]) == n, name
