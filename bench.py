@@ -1,0 +1,387 @@
+"""Benchmark of the streaming tensor-product convolution on B200.
+
+One step = one pass of the whole hot path over one batch: forward plus backward
+(gradients with respect to x, positions and W) of the uvw workload
+"64x0e+64x1o+64x2e, SH lmax 3, N=4096, kNN k=32, E=131072, K=8 Bessel, cutoff 5"
+(synthetic, seeded).  Metric: edges per second of the step (higher is better).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+N > 1 runs under torchrun: every rank processes its own independent graph (weak
+scaling, no data-path collective); the time is the max over ranks.  Rank 0 prints one
+JSON line.  `--impl reference` times the float64 CPU oracle on a bounded sample of the
+same workload instead (rank 0 only).
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from equivariant_gnn_tensor_dst_b200 import workloads  # noqa: E402
+
+METRIC = "TP-conv edges/sec fwd/bwd/double-bwd; % of roofline; peak workspace bytes"
+UNIT = "edges/s"
+CFG = 2
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # SM count x FP32 lanes x FMA x max clock
+L2_FLUSH_BYTES = 256 << 20                          # > 126 MB L2
+
+
+def _workload_config(c, E):
+    return {"workload": "uvw forward+backward, N=4096 kNN k=32 (E=131072), 64x0e+64x1o+64x2e, "
+                        "SH lmax 3, K=8 Bessel r_c=5",
+            "nodes": c.n_nodes, "edges": int(E), "irreps": c.irreps_in, "sh_lmax": c.sh_lmax,
+            "mode": c.mode, "radial": f"{c.radial} K={c.num_basis} r_c={c.r_cut}",
+            "pass": "forward + backward (x, pos, W)", "l2": "flushed between timed steps"}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ---------------------------------------------------------------------------
+# algorithmic operation counts (per edge and per node), from the plan's paths
+# ---------------------------------------------------------------------------
+
+def flop_model(plan):
+    K = plan.num_basis
+    f = dict(state=0, recv=0, src=0, gemm_node=0)
+    for p in plan.paths():
+        ri, ro = 2 * p["l_in"] + 1, 2 * p["l_out"] + 1
+        nnz, ci, co = p["nnz"], p["c_in"], p["c_out"]
+        f["state"] += 2 * ci * (nnz + K * ro)              # eq. 32 coupling + eq. 33 outer product
+        f["recv"] += 2 * ci * (2 * nnz + 2 * K * ro)       # coupling, phi_bar, T_bar, Y_bar
+        f["src"] += 2 * co * (nnz + K * ri)                # adjoint coupling + source state
+        f["gemm_node"] += 2 * K * ci * co * (2 * ro + 2 * ri)  # S A, m_bar A^T, X A^T, x^T X
+    return f
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# native arm
+# ---------------------------------------------------------------------------
+
+def run_native(args):
+    import torch
+
+    from equivariant_gnn_tensor_dst_b200 import binding
+
+    world, rank, local = _dist()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    c = workloads.CONFIGS[CFG]
+    plan = binding.Plan(c.irreps_in, c.sh_lmax, c.irreps_out, c.mode, c.radial, c.num_basis, c.r_cut,
+                        c.r_min, c.r_max)
+    g, rng = workloads.make_graph(c, seed=1000 + CFG + 7919 * rank)
+    N, E = g.n_nodes, g.n_edges
+    x_h = workloads.normal(rng, (N, plan.dim_in))
+    W_h = workloads.weights(rng, c.num_basis, plan.fan_in_per_column())
+    go_h = workloads.normal(rng, (N, plan.dim_out))
+
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)  # noqa: E731
+    x, pos, row_ptr, src, W, gout = t(x_h), t(g.pos), t(g.row_ptr), t(g.src), t(W_h), t(go_h)
+    t_ptr, t_eid, t_dst = binding.tpconv_csr_transpose(row_ptr, src, N)
+    out = torch.empty(N, plan.dim_out, device=dev)
+    gx = torch.empty(N, plan.dim_in, device=dev)
+    gp = torch.empty(N, 3, device=dev)
+    gw = torch.empty(plan.num_basis, plan.weight_cols, device=dev)
+    ws_bytes = plan.workspace_bytes(N, E, binding.PASS_FORWARD | binding.PASS_BACKWARD)
+    torch.cuda.synchronize()
+    mem0 = torch.cuda.memory_allocated(dev)
+    torch.cuda.reset_peak_memory_stats(dev)
+    ws = binding.workspace(ws_bytes, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        binding.tpconv_forward(plan, x, pos, row_ptr, src, W, out=out, ws=ws, stream=stream)
+        binding.tpconv_backward(plan, x, pos, row_ptr, src, t_ptr, t_eid, t_dst, W, gout, ws=ws,
+                                outputs=(gx, gp, gw), stream=stream)
+
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    peak_delta = torch.cuda.max_memory_allocated(dev) - mem0
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.25)
+    binding.tpconv_profile_begin(max(8192, 64 * args.steps))
+    for k in range(args.steps):
+        flush.zero_()
+        starts[k].record(stream)
+        step()
+        ends[k].record(stream)
+    torch.cuda.synchronize()
+    prof = binding.tpconv_profile_end()
+    barrier()
+    clocks = sampler.stop()
+    total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    if world > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+        ee = torch.tensor([float(E)], device=dev, dtype=torch.float64)
+        dist.all_reduce(ee, op=dist.ReduceOp.SUM)
+        edges_all = float(ee.item())
+    else:
+        edges_all = float(E)
+    ms_step = total_ms / args.steps
+    value = edges_all * args.steps / (total_ms / 1e3)
+
+    # live roofline of the dominant kernel category (CUDA events over the timed region)
+    fm = flop_model(plan)
+    algo = {"uvw_receiver_state": fm["state"] * E, "uvw_receiver_backward": fm["recv"] * E,
+            "uvw_source_state": fm["src"] * E, "channel_gemm": fm["gemm_node"] * N}
+    kern = {k: v for k, v in prof.items() if v[1] > 0}
+    gpu_launches = int(sum(v[1] for v in kern.values()))
+    timed_ms = sum(v[0] for v in kern.values())
+    dom = max((k for k in kern if k in algo), key=lambda k: kern[k][0])
+    dom_ms_step = kern[dom][0] / args.steps
+    achieved = algo[dom] / (dom_ms_step / 1e3) / 1e12
+    roofline = {"bound": "alu", "kernel": dom, "achieved": round(achieved, 3),
+                "peak": round(FP32_PEAK_TFLOPS, 1), "unit": "TFLOP/s",
+                "frac": round(achieved / FP32_PEAK_TFLOPS, 4), "traffic": None,
+                "peak_note": "derived: 148 SMs x 128 FP32 lanes x 2 flop x 1965 MHz"}
+    breakdown = {k: {"ms_per_step": round(v[0] / args.steps, 4), "launches_per_step": v[1] / args.steps,
+                     "share": round(v[0] / timed_ms, 4) if timed_ms else None} for k, v in kern.items()}
+    total_algo = sum(algo.values())
+
+    # end-to-end through the public API: pinned host inputs in, results out, every step
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()  # noqa: E731
+        hx, hp, hr, hs, hw, hg = pin(x_h), pin(g.pos), pin(g.row_ptr), pin(g.src), pin(W_h), pin(go_h)
+        ho, hgx, hgp, hgw = (torch.empty(tuple(a.shape), dtype=a.dtype).pin_memory() for a in (out, gx, gp, gw))
+        d_in = [torch.empty_like(a, device=dev) for a in (hx, hp, hr, hs, hw, hg)]
+        bi = sum(a.numel() * a.element_size() for a in (hx, hp, hr, hs, hw, hg))
+        bo = sum(a.numel() * a.element_size() for a in (ho, hgx, hgp, hgw))
+        ne2e = max(3, min(args.steps, 30))
+
+        def e2e_step():
+            for d, h in zip(d_in, (hx, hp, hr, hs, hw, hg)):
+                d.copy_(h, non_blocking=True)
+            xx, pp, rr, ss, WW, GG = d_in
+            tp, te, td = binding.tpconv_csr_transpose(rr, ss, N, stream=stream)
+            o = binding.tpconv_forward(plan, xx, pp, rr, ss, WW, ws=ws, stream=stream)
+            a, b, cc = binding.tpconv_backward(plan, xx, pp, rr, ss, tp, te, td, WW, GG, ws=ws, stream=stream)
+            for h, d in zip((ho, hgx, hgp, hgw), (o, a, b, cc)):
+                h.copy_(d, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(ne2e):
+            e2e_step()
+        s1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = s0.elapsed_time(s1)
+        if world > 1:
+            import torch.distributed as dist
+            tt = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        e2e = {"value": round(edges_all * ne2e / (e_ms / 1e3), 1), "unit": UNIT, "h2d_bytes_per_step": int(bi),
+               "d2h_bytes_per_step": int(bo), "steps": ne2e,
+               "includes": "H2D of x, pos, CSR, W, grad_out; source-view build; forward; backward; "
+                           "D2H of out, grad_x, grad_pos, grad_W"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.cpu_seconds)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": _workload_config(c, E), "impl": "native",
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": gpu_launches,
+                "gpu_launches_per_step": gpu_launches / args.steps, "clocks": clocks,
+                "workspace_bytes": {"declared": int(ws_bytes), "peak_alloc_delta": int(peak_delta)},
+                "step_algorithmic_tflop": round(total_algo / 1e12, 4),
+                "step_tflops_achieved": round(total_algo / (ms_step / 1e3) / 1e12, 3),
+                "breakdown": breakdown}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline and reference arm)
+# ---------------------------------------------------------------------------
+
+def _oracle_sample(seconds_target):
+    from oracle import conv, radial
+    c = workloads.CONFIGS[CFG]
+    rs = radial.RadialSpec(c.radial, c.num_basis, c.r_cut, c.r_min, c.r_max)
+    op = conv.make_plan(c.irreps_in, c.sh_lmax, c.irreps_out, c.mode, rs)
+    g, rng = workloads.make_graph(c)
+    x = workloads.normal(rng, (g.n_nodes, op.dim_in))
+    W = workloads.weights(rng, c.num_basis, op.fan_in_per_column())
+    go = workloads.normal(rng, (g.n_nodes, op.dim_out))
+    rp = g.row_ptr.astype(np.int64)
+
+    def run(n_recv):
+        edges = np.arange(rp[0], rp[n_recv])
+        t0 = time.perf_counter()
+        conv.forward(op, x, g.pos, g.row_ptr, g.src, W, edges=edges)
+        conv.backward(op, x, g.pos, g.row_ptr, g.src, W, go, edges=edges)
+        return time.perf_counter() - t0, edges.size
+
+    # warm up, calibrate on a small sample, then size the sample for the target duration
+    run(2)
+    t_small, _ = run(16)
+    n_recv = int(np.clip(16 * seconds_target / max(t_small, 1e-3), 8, g.n_nodes))
+    return run, n_recv, g
+
+
+def _threads_used():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    except Exception:
+        return 1
+
+
+def cpu_baseline(seconds):
+    run, n_recv, g = _oracle_sample(seconds)
+    dt, ne = run(n_recv)
+    return {"value": round(ne / dt, 2), "unit": UNIT, "cores": _threads_used(), "kind": "oracle",
+            "sample": f"forward+backward over the first {n_recv} receivers ({ne} edges) of the workload",
+            "seconds": round(dt, 2)}
+
+
+def run_reference(args):
+    world, rank, _ = _dist()
+    if rank != 0:
+        return
+    run, n_recv, g = _oracle_sample(args.cpu_seconds / max(1, args.steps))
+    for _ in range(args.warmup):
+        run(min(n_recv, 8))
+    times, ne = [], 0
+    for _ in range(args.steps):
+        dt, ne = run(n_recv)
+        times.append(dt)
+    total = sum(times)
+    value = ne * args.steps / total
+    c = workloads.CONFIGS[CFG]
+    cpu = {"value": round(value, 2), "unit": UNIT, "cores": _threads_used(), "kind": "oracle",
+           "sample": f"each step: forward+backward over the first {n_recv} receivers ({ne} edges)"}
+    line = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": _workload_config(c, g.n_edges), "impl": "reference", "cpu_baseline": cpu,
+            "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("native", "reference"), default="native")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "native":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_native(args)
+
+
+if __name__ == "__main__":
+    main()

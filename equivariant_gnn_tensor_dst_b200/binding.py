@@ -44,7 +44,11 @@ SIGNATURES = {
     "tpconv_forward": (ctypes.c_int, [_c_p, _c_i64, _c_i64] + [_c_p] * 7 + [ctypes.c_size_t, _c_p]),
     "tpconv_backward": (ctypes.c_int, [_c_p, _c_i64, _c_i64] + [_c_p] * 13 + [ctypes.c_size_t, _c_p]),
     "tpconv_double_backward": (ctypes.c_int, [_c_p, _c_i64, _c_i64] + [_c_p] * 17 + [ctypes.c_size_t, _c_p]),
+    "tpconv_profile_begin": (ctypes.c_int, [ctypes.c_int32]),
+    "tpconv_profile_end": (ctypes.c_int, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_c_i64), ctypes.c_int32]),
+    "tpconv_profile_category_name": (ctypes.c_char_p, [ctypes.c_int32]),
 }
+PROF_CATEGORIES = 12
 
 _lib = None
 
@@ -261,3 +265,16 @@ def tpconv_double_backward(plan, x, pos, row_ptr, src, t_ptr, t_eid, t_dst, W, g
                                        None, _ptr(ws), ws.numel(), _stream(stream)),
           "tpconv_double_backward")
     return gx, gw, gg
+
+
+def tpconv_profile_begin(max_records=8192):
+    check(lib().tpconv_profile_begin(int(max_records)), "tpconv_profile_begin")
+
+
+def tpconv_profile_end():
+    """Returns {category: (milliseconds, launches)} for the launches since begin()."""
+    n = PROF_CATEGORIES
+    ms = (ctypes.c_double * n)()
+    cnt = (_c_i64 * n)()
+    check(lib().tpconv_profile_end(ms, cnt, n), "tpconv_profile_end")
+    return {lib().tpconv_profile_category_name(c).decode(): (ms[c], cnt[c]) for c in range(n)}

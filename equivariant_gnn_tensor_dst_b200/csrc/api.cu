@@ -21,6 +21,7 @@
 #include <string>
 #include <vector>
 #include <cmath>
+#include <mutex>
 
 #include "../../include/tpconv.h"
 #include "internal.h"
@@ -40,7 +41,7 @@ struct PathH {
 };
 
 constexpr size_t kDefaultBudget = size_t(128) << 20;  // the pages' 128 MiB scratch cap
-constexpr int kSplitsMax = 32;
+constexpr int kSplits = 8;  // split-K factor of the weight-gradient contractions
 constexpr int kUvuRanges = 64;
 
 int triple_index(int a, int b, int c) {
@@ -120,6 +121,53 @@ tpconv_status parse_irreps(const char* s, std::vector<Block>& out) {
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
+// ---------------------------------------------------------------------------
+// profiling: optional CUDA-event bracketing of every kernel launch, by category
+// ---------------------------------------------------------------------------
+
+enum ProfCat {
+  PC_UVW_STATE = 0, PC_UVW_STATE_TAN, PC_UVW_RECV_BWD, PC_UVW_SRC, PC_UVW_SRC_TAN, PC_GEMM,
+  PC_UVU_FWD, PC_UVU_RECV_BWD, PC_UVU_GRADW, PC_UVU_SRC, PC_POS, PC_GRAPH, PC_COUNT
+};
+static_assert(PC_COUNT == TPCONV_PROF_CATEGORIES, "category count");
+const char* const kProfNames[PC_COUNT] = {
+    "uvw_receiver_state", "uvw_receiver_state_tangent", "uvw_receiver_backward", "uvw_source_state",
+    "uvw_source_state_tangent", "channel_gemm", "uvu_forward", "uvu_receiver_backward",
+    "uvu_weight_gradient", "uvu_source_backward", "position_gradient", "graph"};
+
+struct Prof {
+  std::mutex mu;
+  bool on = false;
+  std::vector<cudaEvent_t> pool;
+  std::vector<int> cat;
+  size_t used = 0;
+  long long launches[PC_COUNT] = {};
+};
+Prof& prof() {
+  static Prof p;
+  return p;
+}
+
+// Brackets one library call that launches `nk` kernels on stream s.
+struct ProfScope {
+  int slot = -1;
+  cudaStream_t s;
+  ProfScope(int c, int nk, cudaStream_t st) : s(st) {
+    Prof& P = prof();
+    std::lock_guard<std::mutex> g(P.mu);
+    if (!P.on) return;
+    P.launches[c] += nk;
+    if (2 * (P.used + 1) > P.pool.size()) return;
+    slot = (int)P.used++;
+    P.cat[slot] = c;
+    cudaEventRecord(P.pool[2 * slot], s);
+  }
+  ~ProfScope() {
+    if (slot < 0) return;
+    cudaEventRecord(prof().pool[2 * slot + 1], s);
+  }
+};
+
 }  // namespace
 
 struct tpconv_plan {
@@ -137,7 +185,6 @@ struct tpconv_plan {
   Tasks t_bi{};   // (input block, chunk)   uvu source pass
   BlockPaths bp_out{}, bp_in{};
   size_t budget = kDefaultBudget;
-  long long max_mn_tn_bwd = 0;  // max over paths of C_in * K * C_out
 };
 
 namespace {
@@ -177,7 +224,7 @@ Layout make_layout(const tpconv_plan* P, long long N, long long E, uint32_t pass
     if (pass != TPCONV_PASS_FORWARD) {
       L.has_part = true;
       L.part = off;
-      off += align256(size_t(4) * kSplitsMax * P->max_mn_tn_bwd);
+      off += align256(size_t(4) * kSplits * P->K * (long long)P->n_w);
     }
   } else {
     if (pass != TPCONV_PASS_FORWARD) {
@@ -196,17 +243,6 @@ Layout make_layout(const tpconv_plan* P, long long N, long long E, uint32_t pass
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-int splits_for(long long kc) {
-  long long s = kc / 256;
-  return (int)std::max<long long>(1, std::min<long long>(kSplitsMax, s));
-}
-
-GemmArgs gemm_base() {
-  GemmArgs g{};
-  g.splits = 1;
-  return g;
-}
 
 }  // namespace
 
@@ -309,7 +345,6 @@ tpconv_status tpconv_plan_create(tpconv_plan_t* out, const char* irreps_in, int3
     d.type = h.type; d.l_in = h.l_in; d.l_sh = h.l_sh; d.l_out = h.l_out;
     d.c_in = h.c_in; d.c_out = h.c_out; d.in_off = h.in_off; d.out_off = h.out_off;
     d.w_off = h.w_off; d.st_off = h.st_off; d.xst_off = h.xst_off; d.b_in = h.b_in; d.b_out = h.b_out;
-    P->max_mn_tn_bwd = std::max<long long>(P->max_mn_tn_bwd, (long long)h.c_in * P->K * h.c_out);
   }
   // warp task lists
   auto push = [](Tasks& T, int a, int b) {
@@ -407,8 +442,10 @@ tpconv_status tpconv_csr_transpose(int64_t N, int64_t E, const int32_t* row_ptr,
   if (ws_bytes < need) return TPCONV_ERR_WORKSPACE_TOO_SMALL;
   if (!aligned16(row_ptr) || !aligned16(t_ptr) || (E > 0 && (!aligned16(src) || !aligned16(t_eid) || !aligned16(t_dst))) || !aligned16(ws))
     return TPCONV_ERR_MISALIGNED;
+  cudaStream_t s = (cudaStream_t)stream;
+  ProfScope ps(PC_GRAPH, 4, s);
   cudaError_t e = launch_csr_transpose((int)N, (int)E, row_ptr, src, t_ptr, t_eid, t_dst,
-                                       static_cast<int*>(ws), (cudaStream_t)stream);
+                                       static_cast<int*>(ws), s);
   return e == cudaSuccess ? TPCONV_OK : TPCONV_ERR_CUDA;
 }
 
@@ -430,6 +467,14 @@ namespace {
 
 #define TPC_TRY(expr)                                   \
   do {                                                  \
+    cudaError_t e_ = (expr);                            \
+    if (e_ != cudaSuccess) return TPCONV_ERR_CUDA;      \
+  } while (0)
+
+// launch under a profiling scope: category, number of kernels, call
+#define TPC_RUN(cat, nk, expr)                          \
+  do {                                                  \
+    ProfScope ps_(cat, nk, s);                          \
     cudaError_t e_ = (expr);                            \
     if (e_ != cudaSuccess) return TPCONV_ERR_CUDA;      \
   } while (0)
@@ -457,73 +502,121 @@ tpconv_status check_ws(const Layout& L, void* ws, size_t ws_bytes) {
   return TPCONV_OK;
 }
 
-// m[(i,mo), w] += sum_{q,u} S[(i,mo),(q,u)] A[(q,u), w]          (eqs. 34-35)
-GemmArgs g_state_times_A(const tpconv_plan* P, const PathH& p, const float* S, const float* W,
-                         float* out, int n0, int cn) {
-  const int RO = 2 * p.l_out + 1;
-  GemmArgs g = gemm_base();
-  g.M = cn * RO; g.N = p.c_out; g.K = P->K * p.c_in;
-  g.A = S + p.st_off; g.Am = idx2(RO, P->dev.state_per_node, (long long)P->K * p.c_in); g.Ak = idx1(1);
-  g.B = W + p.w_off; g.Bk = idx2(p.c_in, P->n_w, p.c_out); g.Bn = idx1(1);
-  g.C = out + (long long)n0 * P->dim_out + p.out_off; g.Cm = idx2(RO, P->dim_out, p.c_out); g.Cn = idx1(1);
-  g.accumulate = 1;
-  return g;
+struct Batch {
+  GemmBatch g{};
+  Batch(int splits, int accumulate, float* partial) {
+    g.splits = splits;
+    g.accumulate = accumulate;
+    g.partial = partial;
+  }
+  void problem(float* C, Idx2 Cm, Idx2 Cn, int M, int N) {
+    GemmProblem& p = g.pr[g.n_problems++];
+    p.C = C; p.Cm = Cm; p.Cn = Cn; p.M = M; p.N = N;
+    p.seg0 = g.n_segs; p.nseg = 0; p.Ktot = 0;
+  }
+  void seg(const float* A, Idx2 Am, Idx2 Ak, const float* B, Idx2 Bk, Idx2 Bn, int K) {
+    GemmSeg& s = g.sg[g.n_segs++];
+    s.A = A; s.Am = Am; s.Ak = Ak; s.B = B; s.Bk = Bk; s.Bn = Bn; s.K = K;
+    GemmProblem& p = g.pr[g.n_problems - 1];
+    ++p.nseg;
+    p.Ktot += K;
+  }
+};
+
+// m_g[(i,mo), w] = sum_{pi in g} sum_{q,u} S_pi[(i,mo),(q,u)] A_pi[(q,u), w]   (eqs. 34-35),
+// optionally + sum_pi S2_pi A2_pi (eq. 37: dm = dS A + S dA)
+cudaError_t gemm_state_times_A(const tpconv_plan* P, const float* S, const float* W, const float* S2,
+                               const float* W2, float* out, int n0, int cn, cudaStream_t st) {
+  Batch b(1, 0, nullptr);
+  for (int bo = 0; bo < (int)P->out.size(); ++bo) {
+    const Block& B = P->out[bo];
+    const int RO = 2 * B.l + 1;
+    bool any = false;
+    for (const PathH& p : P->paths) any = any || p.b_out == bo;
+    if (!any) continue;
+    b.problem(out + (long long)n0 * P->dim_out + B.offset, idx2(RO, P->dim_out, B.mul), idx1(1), cn * RO, B.mul);
+    for (const PathH& p : P->paths) {
+      if (p.b_out != bo) continue;
+      const Idx2 Am = idx2(RO, P->dev.state_per_node, (long long)P->K * p.c_in);
+      const Idx2 Bk = idx2(p.c_in, P->n_w, p.c_out);
+      if (S) b.seg(S + p.st_off, Am, idx1(1), W + p.w_off, Bk, idx1(1), P->K * p.c_in);
+      if (S2) b.seg(S2 + p.st_off, Am, idx1(1), W2 + p.w_off, Bk, idx1(1), P->K * p.c_in);
+    }
+  }
+  return launch_gemm(b.g, st);
 }
 
-// S_bar[(i,mo),(q,u)] = sum_w m_bar[(i,mo), w] A[(q,u), w]        (eq. 36)
-GemmArgs g_sbar(const tpconv_plan* P, const PathH& p, const float* gout, const float* W,
-                float* Sbar, int n0, int cn) {
-  const int RO = 2 * p.l_out + 1;
-  GemmArgs g = gemm_base();
-  g.M = cn * RO; g.N = P->K * p.c_in; g.K = p.c_out;
-  g.A = gout + (long long)n0 * P->dim_out + p.out_off; g.Am = idx2(RO, P->dim_out, p.c_out); g.Ak = idx1(1);
-  g.B = W + p.w_off; g.Bk = idx1(1); g.Bn = idx2(p.c_in, P->n_w, p.c_out);
-  g.C = Sbar + p.st_off; g.Cm = idx2(RO, P->dev.state_per_node, (long long)P->K * p.c_in); g.Cn = idx1(1);
-  g.accumulate = 0;
-  return g;
+// S_bar_pi[(i,mo),(q,u)] = sum_w m_bar[(i,mo), w] A_pi[(q,u), w]        (eq. 36)
+cudaError_t gemm_sbar(const tpconv_plan* P, const float* gout, const float* W, float* Sbar, int n0,
+                      int cn, cudaStream_t st) {
+  Batch b(1, 0, nullptr);
+  for (const PathH& p : P->paths) {
+    const int RO = 2 * p.l_out + 1;
+    b.problem(Sbar + p.st_off, idx2(RO, P->dev.state_per_node, (long long)P->K * p.c_in), idx1(1), cn * RO,
+              P->K * p.c_in);
+    b.seg(gout + (long long)n0 * P->dim_out + p.out_off, idx2(RO, P->dim_out, p.c_out), idx1(1), W + p.w_off,
+          idx1(1), idx2(p.c_in, P->n_w, p.c_out), p.c_out);
+  }
+  return launch_gemm(b.g, st);
 }
 
-// x_bar[(j,mi), u] += sum_{q,w} X[(j,mi),(q,w)] A[(q,u), w]      (mirrored eq. 21)
-GemmArgs g_xbar(const tpconv_plan* P, const PathH& p, const float* X, const float* W,
-                float* gx, int n0, int cn) {
-  const int RI = 2 * p.l_in + 1;
-  GemmArgs g = gemm_base();
-  g.M = cn * RI; g.N = p.c_in; g.K = P->K * p.c_out;
-  g.A = X + p.xst_off; g.Am = idx2(RI, P->dev.xstate_per_node, (long long)P->K * p.c_out); g.Ak = idx1(1);
-  g.B = W + p.w_off; g.Bk = idx2(p.c_out, P->n_w, 1); g.Bn = idx1(p.c_out);
-  g.C = gx + (long long)n0 * P->dim_in + p.in_off; g.Cm = idx2(RI, P->dim_in, p.c_in); g.Cn = idx1(1);
-  g.accumulate = 1;
-  return g;
+// x_bar[(j,mi), u] = sum_{pi from block} sum_{q,w} X_pi[(j,mi),(q,w)] A_pi[(q,u), w]
+// (mirrored eq. 21), optionally + X2 A2^T (eq. 30 with A_dot)
+cudaError_t gemm_xbar(const tpconv_plan* P, const float* X, const float* W, const float* X2, const float* W2,
+                      float* gx, int n0, int cn, cudaStream_t st) {
+  Batch b(1, 0, nullptr);
+  for (int bi = 0; bi < (int)P->in.size(); ++bi) {
+    const Block& B = P->in[bi];
+    const int RI = 2 * B.l + 1;
+    bool any = false;
+    for (const PathH& p : P->paths) any = any || p.b_in == bi;
+    if (!any) continue;
+    b.problem(gx + (long long)n0 * P->dim_in + B.offset, idx2(RI, P->dim_in, B.mul), idx1(1), cn * RI, B.mul);
+    for (const PathH& p : P->paths) {
+      if (p.b_in != bi) continue;
+      const Idx2 Am = idx2(RI, P->dev.xstate_per_node, (long long)P->K * p.c_out);
+      const Idx2 Bk = idx2(p.c_out, P->n_w, 1);
+      if (X) b.seg(X + p.xst_off, Am, idx1(1), W + p.w_off, Bk, idx1(p.c_out), P->K * p.c_out);
+      if (X2) b.seg(X2 + p.xst_off, Am, idx1(1), W2 + p.w_off, Bk, idx1(p.c_out), P->K * p.c_out);
+    }
+  }
+  return launch_gemm(b.g, st);
 }
 
-// A_bar[(q,u), w] += sum_{(j,mi)} x[(j,mi), u] X[(j,mi),(q,w)]    (mirrored eq. 19)
-GemmArgs g_abar_src(const tpconv_plan* P, const PathH& p, const float* x, const float* X,
-                    float* gW, int n0, int cn, float* part) {
-  const int RI = 2 * p.l_in + 1;
-  GemmArgs g = gemm_base();
-  g.M = p.c_in; g.N = P->K * p.c_out; g.K = cn * RI;
-  g.A = x + (long long)n0 * P->dim_in + p.in_off; g.Am = idx1(1); g.Ak = idx2(RI, P->dim_in, p.c_in);
-  g.B = X + p.xst_off; g.Bk = idx2(RI, P->dev.xstate_per_node, (long long)P->K * p.c_out); g.Bn = idx1(1);
-  g.C = gW + p.w_off; g.Cm = idx1(p.c_out); g.Cn = idx2(p.c_out, P->n_w, 1);
-  g.accumulate = 1;
-  g.splits = splits_for(g.K);
-  g.partial = part;
-  return g;
+// A_bar_pi[(q,u), w] (+)= sum_{(j,mi)} x[(j,mi), u] X_pi[(j,mi),(q,w)]     (mirrored eq. 19)
+cudaError_t gemm_abar_src(const tpconv_plan* P, const float* x, const float* X, float* gW, int n0, int cn,
+                          int accumulate, float* part, cudaStream_t st) {
+  Batch b(kSplits, accumulate, part);
+  for (const PathH& p : P->paths) {
+    const int RI = 2 * p.l_in + 1;
+    b.problem(gW + p.w_off, idx1(p.c_out), idx2(p.c_out, P->n_w, 1), p.c_in, P->K * p.c_out);
+    b.seg(x + (long long)n0 * P->dim_in + p.in_off, idx1(1), idx2(RI, P->dim_in, p.c_in), X + p.xst_off,
+          idx2(RI, P->dev.xstate_per_node, (long long)P->K * p.c_out), idx1(1), cn * RI);
+  }
+  return launch_gemm(b.g, st);
 }
 
-// A_bar[(q,u), w] += sum_{(i,mo)} dS[(i,mo),(q,u)] m_bar[(i,mo), w]   (eq. 39)
-GemmArgs g_abar_recv(const tpconv_plan* P, const PathH& p, const float* S, const float* gout,
-                     float* gW, int n0, int cn, float* part) {
-  const int RO = 2 * p.l_out + 1;
-  GemmArgs g = gemm_base();
-  g.M = P->K * p.c_in; g.N = p.c_out; g.K = cn * RO;
-  g.A = S + p.st_off; g.Am = idx1(1); g.Ak = idx2(RO, P->dev.state_per_node, (long long)P->K * p.c_in);
-  g.B = gout + (long long)n0 * P->dim_out + p.out_off; g.Bk = idx2(RO, P->dim_out, p.c_out); g.Bn = idx1(1);
-  g.C = gW + p.w_off; g.Cm = idx2(p.c_in, P->n_w, p.c_out); g.Cn = idx1(1);
-  g.accumulate = 1;
-  g.splits = splits_for(g.K);
-  g.partial = part;
-  return g;
+// A_bar_pi[(q,u), w] (+)= sum_{(i,mo)} dS_pi[(i,mo),(q,u)] m_bar[(i,mo), w]   (eq. 39)
+cudaError_t gemm_abar_recv(const tpconv_plan* P, const float* S, const float* gout, float* gW, int n0, int cn,
+                           int accumulate, float* part, cudaStream_t st) {
+  Batch b(kSplits, accumulate, part);
+  for (const PathH& p : P->paths) {
+    const int RO = 2 * p.l_out + 1;
+    b.problem(gW + p.w_off, idx2(p.c_in, P->n_w, p.c_out), idx1(1), P->K * p.c_in, p.c_out);
+    b.seg(S + p.st_off, idx1(1), idx2(RO, P->dev.state_per_node, (long long)P->K * p.c_in),
+          gout + (long long)n0 * P->dim_out + p.out_off, idx2(RO, P->dim_out, p.c_out), idx1(1), cn * RO);
+  }
+  return launch_gemm(b.g, st);
+}
+
+bool every_block_reached(const tpconv_plan* P, bool out_side) {
+  const int nb = (int)(out_side ? P->out.size() : P->in.size());
+  for (int b = 0; b < nb; ++b) {
+    bool any = false;
+    for (const PathH& p : P->paths) any = any || (out_side ? p.b_out : p.b_in) == b;
+    if (!any) return false;
+  }
+  return true;
 }
 
 float* fptr(void* ws, size_t off) { return reinterpret_cast<float*>(static_cast<char*>(ws) + off); }
@@ -548,17 +641,17 @@ tpconv_status tpconv_forward(tpconv_plan_t P, int64_t N, int64_t E, const float*
   cudaStream_t s = (cudaStream_t)stream;
   const int n = (int)N;
   if (P->mode == TPCONV_UVU) {
-    TPC_TRY(launch_uvu_fwd(P->dev, P->bp_out, P->t_bo, 0, x, nullptr, pos, nullptr, row_ptr, src, W,
+    TPC_RUN(PC_UVU_FWD, 1, launch_uvu_fwd(P->dev, P->bp_out, P->t_bo, 0, x, nullptr, pos, nullptr, row_ptr, src, W,
                            nullptr, n, out, s));
     return TPCONV_OK;
   }
-  TPC_TRY(cudaMemsetAsync(out, 0, sizeof(float) * (size_t)N * P->dim_out, s));
+  if (!every_block_reached(P, true)) TPC_TRY(cudaMemsetAsync(out, 0, sizeof(float) * (size_t)N * P->dim_out, s));
   float* S = fptr(ws, L.state_a);
   for (int n0 = 0; n0 < n; n0 += L.recv_chunk) {
     const int cn = std::min(L.recv_chunk, n - n0);
-    TPC_TRY(launch_uvw_state(P->dev, P->t_in, 0, x, nullptr, pos, nullptr, row_ptr, src, n0, cn, S,
+    TPC_RUN(PC_UVW_STATE, 1, launch_uvw_state(P->dev, P->t_in, 0, x, nullptr, pos, nullptr, row_ptr, src, n0, cn, S,
                              nullptr, s));
-    for (const PathH& p : P->paths) TPC_TRY(launch_gemm(g_state_times_A(P, p, S, W, out, n0, cn), s));
+    TPC_RUN(PC_GEMM, 1, gemm_state_times_A(P, S, W, nullptr, nullptr, out, n0, cn, s));
   }
   return TPCONV_OK;
 }
@@ -589,17 +682,17 @@ tpconv_status tpconv_backward(tpconv_plan_t P, int64_t N, int64_t E, const float
 
   if (P->mode == TPCONV_UVU) {
     if (grad_pos) {
-      TPC_TRY(launch_uvu_recv_bwd(P->dev, P->t_in, x, pos, row_ptr, src, W, grad_out, n, gbuf, s));
-      TPC_TRY(launch_pos_finish(n, row_ptr, t_ptr, t_eid, gbuf, grad_pos, s));
+      TPC_RUN(PC_UVU_RECV_BWD, 1, launch_uvu_recv_bwd(P->dev, P->t_in, x, pos, row_ptr, src, W, grad_out, n, gbuf, s));
+      TPC_RUN(PC_POS, 1, launch_pos_finish(n, row_ptr, t_ptr, t_eid, gbuf, grad_pos, s));
     }
     if (grad_W) {
       const int nr = std::min(kUvuRanges, n);
-      TPC_TRY(launch_uvu_gradw(P->dev, P->t_in, 0, x, nullptr, pos, nullptr, row_ptr, src, grad_out, n,
+      TPC_RUN(PC_UVU_GRADW, 1, launch_uvu_gradw(P->dev, P->t_in, 0, x, nullptr, pos, nullptr, row_ptr, src, grad_out, n,
                                nr, part, s));
-      TPC_TRY(launch_reduce_partials(part, nr, (long long)P->K * P->n_w, grad_W, 0, s));
+      TPC_RUN(PC_UVU_GRADW, 1, launch_reduce_partials(part, nr, (long long)P->K * P->n_w, grad_W, 0, s));
     }
     if (grad_x)
-      TPC_TRY(launch_uvu_src(P->dev, P->bp_in, P->t_bi, 0, pos, nullptr, t_ptr, t_eid, t_dst, W,
+      TPC_RUN(PC_UVU_SRC, 1, launch_uvu_src(P->dev, P->bp_in, P->t_bi, 0, pos, nullptr, t_ptr, t_eid, t_dst, W,
                              nullptr, grad_out, n, grad_x, s));
     return TPCONV_OK;
   }
@@ -608,22 +701,20 @@ tpconv_status tpconv_backward(tpconv_plan_t P, int64_t N, int64_t E, const float
   if (grad_pos) {
     for (int n0 = 0; n0 < n; n0 += L.recv_chunk) {
       const int cn = std::min(L.recv_chunk, n - n0);
-      for (const PathH& p : P->paths) TPC_TRY(launch_gemm(g_sbar(P, p, grad_out, W, state, n0, cn), s));
-      TPC_TRY(launch_uvw_recv_bwd(P->dev, P->t_in, x, pos, row_ptr, src, state, n0, cn, gbuf, s));
+      TPC_RUN(PC_GEMM, 1, gemm_sbar(P, grad_out, W, state, n0, cn, s));
+      TPC_RUN(PC_UVW_RECV_BWD, 1, launch_uvw_recv_bwd(P->dev, P->t_in, x, pos, row_ptr, src, state, n0, cn, gbuf, s));
     }
-    TPC_TRY(launch_pos_finish(n, row_ptr, t_ptr, t_eid, gbuf, grad_pos, s));
+    TPC_RUN(PC_POS, 1, launch_pos_finish(n, row_ptr, t_ptr, t_eid, gbuf, grad_pos, s));
   }
-  if (grad_x) TPC_TRY(cudaMemsetAsync(grad_x, 0, sizeof(float) * (size_t)N * P->dim_in, s));
-  if (grad_W) TPC_TRY(cudaMemsetAsync(grad_W, 0, sizeof(float) * (size_t)P->K * P->n_w, s));
+  if (grad_x && !every_block_reached(P, false))
+    TPC_TRY(cudaMemsetAsync(grad_x, 0, sizeof(float) * (size_t)N * P->dim_in, s));
   if (grad_x || grad_W) {
     for (int n0 = 0; n0 < n; n0 += L.src_chunk) {
       const int cn = std::min(L.src_chunk, n - n0);
-      TPC_TRY(launch_uvw_src_state(P->dev, P->t_out, 0, pos, nullptr, t_ptr, t_eid, t_dst, grad_out, n0,
+      TPC_RUN(PC_UVW_SRC, 1, launch_uvw_src_state(P->dev, P->t_out, 0, pos, nullptr, t_ptr, t_eid, t_dst, grad_out, n0,
                                    cn, state, nullptr, s));
-      for (const PathH& p : P->paths) {
-        if (grad_x) TPC_TRY(launch_gemm(g_xbar(P, p, state, W, grad_x, n0, cn), s));
-        if (grad_W) TPC_TRY(launch_gemm(g_abar_src(P, p, x, state, grad_W, n0, cn, part), s));
-      }
+      if (grad_x) TPC_RUN(PC_GEMM, 1, gemm_xbar(P, state, W, nullptr, nullptr, grad_x, n0, cn, s));
+      if (grad_W) TPC_RUN(PC_GEMM, 2, gemm_abar_src(P, x, state, grad_W, n0, cn, n0 > 0, part, s));
     }
   }
   return TPCONV_OK;
@@ -659,54 +750,98 @@ tpconv_status tpconv_double_backward(tpconv_plan_t P, int64_t N, int64_t E, cons
 
   if (P->mode == TPCONV_UVU) {
     if (grad_grad_out)
-      TPC_TRY(launch_uvu_fwd(P->dev, P->bp_out, P->t_bo, 1, x, gg_x, pos, gg_pos, row_ptr, src, W, gg_W,
+      TPC_RUN(PC_UVU_FWD, 1, launch_uvu_fwd(P->dev, P->bp_out, P->t_bo, 1, x, gg_x, pos, gg_pos, row_ptr, src, W, gg_W,
                              n, grad_grad_out, s));
     if (grad_W) {
       const int nr = std::min(kUvuRanges, n);
-      TPC_TRY(launch_uvu_gradw(P->dev, P->t_in, 1, x, gg_x, pos, gg_pos, row_ptr, src, grad_out, n, nr,
+      TPC_RUN(PC_UVU_GRADW, 1, launch_uvu_gradw(P->dev, P->t_in, 1, x, gg_x, pos, gg_pos, row_ptr, src, grad_out, n, nr,
                                part, s));
-      TPC_TRY(launch_reduce_partials(part, nr, (long long)P->K * P->n_w, grad_W, 0, s));
+      TPC_RUN(PC_UVU_GRADW, 1, launch_reduce_partials(part, nr, (long long)P->K * P->n_w, grad_W, 0, s));
     }
     if (grad_x)
-      TPC_TRY(launch_uvu_src(P->dev, P->bp_in, P->t_bi, 1, pos, gg_pos, t_ptr, t_eid, t_dst, W, gg_W,
+      TPC_RUN(PC_UVU_SRC, 1, launch_uvu_src(P->dev, P->bp_in, P->t_bi, 1, pos, gg_pos, t_ptr, t_eid, t_dst, W, gg_W,
                              grad_out, n, grad_x, s));
     return TPCONV_OK;
   }
 
   float* sa = fptr(ws, L.state_a);
   float* sb = fptr(ws, L.state_b);
-  if (grad_grad_out) TPC_TRY(cudaMemsetAsync(grad_grad_out, 0, sizeof(float) * (size_t)N * P->dim_out, s));
-  if (grad_W) TPC_TRY(cudaMemsetAsync(grad_W, 0, sizeof(float) * (size_t)P->K * P->n_w, s));
   const bool need_S = grad_grad_out && gg_W;
+  const bool gout_direct = grad_grad_out && (tan_xp || need_S) && every_block_reached(P, true);
+  if (grad_grad_out && !gout_direct)
+    TPC_TRY(cudaMemsetAsync(grad_grad_out, 0, sizeof(float) * (size_t)N * P->dim_out, s));
+  if (grad_W && !tan_xp) TPC_TRY(cudaMemsetAsync(grad_W, 0, sizeof(float) * (size_t)P->K * P->n_w, s));
   if ((grad_grad_out || grad_W) && (tan_xp || need_S)) {
     for (int n0 = 0; n0 < n; n0 += L.recv_chunk) {
       const int cn = std::min(L.recv_chunk, n - n0);
       // sa = dS (tangent of eq. 33), sb = S (needed for S dA in eq. 37)
-      TPC_TRY(launch_uvw_state(P->dev, P->t_in, 1, x, gg_x, pos, gg_pos, row_ptr, src, n0, cn,
+      TPC_RUN(PC_UVW_STATE_TAN, 1, launch_uvw_state(P->dev, P->t_in, 1, x, gg_x, pos, gg_pos, row_ptr, src, n0, cn,
                                need_S ? sb : nullptr, sa, s));
-      for (const PathH& p : P->paths) {
-        if (grad_grad_out && tan_xp) TPC_TRY(launch_gemm(g_state_times_A(P, p, sa, W, grad_grad_out, n0, cn), s));
-        if (need_S) TPC_TRY(launch_gemm(g_state_times_A(P, p, sb, gg_W, grad_grad_out, n0, cn), s));
-        if (grad_W && tan_xp) TPC_TRY(launch_gemm(g_abar_recv(P, p, sa, grad_out, grad_W, n0, cn, part), s));
-      }
+      if (grad_grad_out)
+        TPC_RUN(PC_GEMM, 1, gemm_state_times_A(P, tan_xp ? sa : nullptr, W, need_S ? sb : nullptr, gg_W, grad_grad_out, n0,
+                                   cn, s));
+      if (grad_W && tan_xp) TPC_RUN(PC_GEMM, 2, gemm_abar_recv(P, sa, grad_out, grad_W, n0, cn, n0 > 0, part, s));
     }
   }
   if (grad_x) {
-    TPC_TRY(cudaMemsetAsync(grad_x, 0, sizeof(float) * (size_t)N * P->dim_in, s));
+    const bool direct = (gg_pos || gg_W) && every_block_reached(P, false);
+    if (!direct) TPC_TRY(cudaMemsetAsync(grad_x, 0, sizeof(float) * (size_t)N * P->dim_in, s));
     if (gg_pos || gg_W) {
       for (int n0 = 0; n0 < n; n0 += L.src_chunk) {
         const int cn = std::min(L.src_chunk, n - n0);
         // sa = X' (tangent of the source state), sb = X
-        TPC_TRY(launch_uvw_src_state(P->dev, P->t_out, 1, pos, gg_pos, t_ptr, t_eid, t_dst, grad_out, n0,
+        TPC_RUN(PC_UVW_SRC_TAN, 1, launch_uvw_src_state(P->dev, P->t_out, 1, pos, gg_pos, t_ptr, t_eid, t_dst, grad_out, n0,
                                      cn, gg_W ? sb : nullptr, sa, s));
-        for (const PathH& p : P->paths) {
-          if (gg_pos) TPC_TRY(launch_gemm(g_xbar(P, p, sa, W, grad_x, n0, cn), s));
-          if (gg_W) TPC_TRY(launch_gemm(g_xbar(P, p, sb, gg_W, grad_x, n0, cn), s));
-        }
+        TPC_RUN(PC_GEMM, 1, gemm_xbar(P, gg_pos ? sa : nullptr, W, gg_W ? sb : nullptr, gg_W, grad_x, n0, cn, s));
       }
     }
   }
   return TPCONV_OK;
+}
+
+tpconv_status tpconv_profile_begin(int32_t max_records) {
+  if (max_records < 1 || max_records > (1 << 20)) return TPCONV_ERR_INVALID_ARG;
+  Prof& P = prof();
+  std::lock_guard<std::mutex> g(P.mu);
+  const size_t want = size_t(2) * max_records;
+  while (P.pool.size() < want) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return TPCONV_ERR_CUDA;
+    P.pool.push_back(e);
+  }
+  P.cat.assign(max_records, 0);
+  P.used = 0;
+  for (long long& v : P.launches) v = 0;
+  P.on = true;
+  return TPCONV_OK;
+}
+
+tpconv_status tpconv_profile_end(double* ms, int64_t* launches, int32_t n) {
+  if (n < 0 || n > PC_COUNT) return TPCONV_ERR_INVALID_ARG;
+  Prof& P = prof();
+  std::lock_guard<std::mutex> g(P.mu);
+  double tot[PC_COUNT] = {};
+  tpconv_status st = TPCONV_OK;
+  for (size_t r = 0; r < P.used; ++r) {
+    float t = 0.f;
+    if (cudaEventSynchronize(P.pool[2 * r + 1]) != cudaSuccess ||
+        cudaEventElapsedTime(&t, P.pool[2 * r], P.pool[2 * r + 1]) != cudaSuccess) {
+      st = TPCONV_ERR_CUDA;
+      continue;
+    }
+    tot[P.cat[r]] += t;
+  }
+  for (int c = 0; c < n; ++c) {
+    if (ms) ms[c] = tot[c];
+    if (launches) launches[c] = P.launches[c];
+  }
+  P.on = false;
+  P.used = 0;
+  return st;
+}
+
+const char* tpconv_profile_category_name(int32_t c) {
+  return (c >= 0 && c < PC_COUNT) ? kProfNames[c] : "unknown";
 }
 
 }  // extern "C"

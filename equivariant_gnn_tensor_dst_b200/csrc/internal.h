@@ -59,14 +59,35 @@ struct Idx2 {
 inline Idx2 idx1(long long s) { return Idx2{0x7fffffff, 0, s}; }
 inline Idx2 idx2(int d, long long s1, long long s2) { return Idx2{d, s1, s2}; }
 
-struct GemmArgs {
+// Grouped, multi-segment GEMM.  Problem p computes
+//   C_p(m, n) (+)= sum over its segments s of sum_k A_s(m, k) B_s(k, n)
+// with every operand addressed through two-level affine maps, so node rows of the
+// ir_mul tensors, the weight matrix and workspace states are read in place.  Problems
+// write disjoint outputs; one launch covers all problems.  With splits > 1 each
+// problem's contraction is split and reduced in a fixed order from `partial`.
+constexpr int MAX_GEMM_PROBLEMS = 64;
+constexpr int MAX_GEMM_SEGS = 128;
+
+struct GemmSeg {
   const float* A; Idx2 Am, Ak;   // A(m, k)
   const float* B; Idx2 Bk, Bn;   // B(k, n)
+  int K;
+};
+
+struct GemmProblem {
   float* C; Idx2 Cm, Cn;         // C(m, n)
-  int M, N, K;
-  int accumulate;                // C += AB (1) or C = AB (0)
-  float* partial;                // split-K scratch [splits][M][N] (splits > 1)
-  int splits;
+  int M, N;
+  int seg0, nseg;                // segments [seg0, seg0 + nseg)
+  int Ktot;                      // sum of the segments' K
+  int tile0;                     // first global tile of this problem
+  long long part_off;            // offset of this problem in `partial` (splits * M * N floats)
+};
+
+struct GemmBatch {
+  int n_problems, n_segs, splits, total_tiles, accumulate;
+  float* partial;
+  GemmProblem pr[MAX_GEMM_PROBLEMS];
+  GemmSeg sg[MAX_GEMM_SEGS];
 };
 
 // Per-(KP, MODE) kernel runners.  Each is explicitly instantiated in its own
@@ -107,7 +128,7 @@ cudaError_t run_uvu_src(const DevPlan& P, const BlockPaths& BP, const Tasks& T, 
                         cudaStream_t s);
 
 // kernel launchers (dispatch on K and mode; defined in launch.cu and k_misc.cu)
-cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
+cudaError_t launch_gemm(GemmBatch& g, cudaStream_t s);  // fills tile0 / total_tiles
 
 cudaError_t launch_uvw_state(const DevPlan& P, const Tasks& T, int mode, const float* x,
                              const float* xdot, const float* pos, const float* posdot,

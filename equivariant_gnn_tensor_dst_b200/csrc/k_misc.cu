@@ -21,87 +21,111 @@ __device__ __forceinline__ long long ix(const Idx2& f, int i) {
 
 constexpr int GBM = 64, GBN = 64, GBK = 16;
 
-__global__ void __launch_bounds__(256) k_gemm(GemmArgs g) {
+__global__ void __launch_bounds__(256) k_gemm(const __grid_constant__ GemmBatch g) {
   __shared__ float As[GBK][GBM + 4];
   __shared__ float Bs[GBK][GBN + 4];
+  const int tile = blockIdx.x;
+  int pi = 0;
+  while (pi + 1 < g.n_problems && g.pr[pi + 1].tile0 <= tile) ++pi;
+  const GemmProblem& P = g.pr[pi];
+  const int lt = tile - P.tile0;
+  const int tn = (P.N + GBN - 1) / GBN;
+  const int m0 = (lt / tn) * GBM, n0 = (lt % tn) * GBN;
+  const int split = blockIdx.y;
+  const int kper = (P.Ktot + g.splits - 1) / g.splits;
+  const int kb = split * kper, ke = min(P.Ktot, kb + kper);
   const int tid = threadIdx.x;
-  const int m0 = blockIdx.y * GBM, n0 = blockIdx.x * GBN;
-  const int split = blockIdx.z;
-  const int kper = ((g.K + g.splits - 1) / g.splits + GBK - 1) / GBK * GBK;
-  const int kb = split * kper;
-  const int ke = min(g.K, kb + kper);
   const int tx = tid & 15, ty = tid >> 4;
   float acc[4][4];
 #pragma unroll
   for (int a = 0; a < 4; ++a)
 #pragma unroll
     for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
-  for (int k0 = kb; k0 < ke; k0 += GBK) {
+  int kbase = 0;
+  for (int si = 0; si < P.nseg; ++si) {
+    const GemmSeg& S = g.sg[P.seg0 + si];
+    const int lo = max(kb - kbase, 0), hi = min(ke - kbase, S.K);
+    kbase += S.K;
+    for (int k0 = lo; k0 < hi; k0 += GBK) {
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int idx = tid + r * 256;
-      const int kk = idx & 15, mm = idx >> 4;
-      const int m = m0 + mm, k = k0 + kk;
-      As[kk][mm] = (m < g.M && k < ke) ? __ldg(g.A + ix(g.Am, m) + ix(g.Ak, k)) : 0.f;
+      for (int r = 0; r < 4; ++r) {
+        const int idx = tid + r * 256;
+        const int kk = idx & 15, mm = idx >> 4;
+        const int m = m0 + mm, k = k0 + kk;
+        As[kk][mm] = (m < P.M && k < hi) ? __ldg(S.A + ix(S.Am, m) + ix(S.Ak, k)) : 0.f;
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int idx = tid + r * 256;
+        const int nn = idx & 63, kk = idx >> 6;
+        const int n = n0 + nn, k = k0 + kk;
+        Bs[kk][nn] = (n < P.N && k < hi) ? __ldg(S.B + ix(S.Bk, k) + ix(S.Bn, n)) : 0.f;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int kk = 0; kk < GBK; ++kk) {
+        float av[4], bv[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) { av[t] = As[kk][ty * 4 + t]; bv[t] = Bs[kk][tx * 4 + t]; }
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc[p][q] = fmaf(av[p], bv[q], acc[p][q]);
+      }
+      __syncthreads();
     }
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int idx = tid + r * 256;
-      const int nn = idx & 63, kk = idx >> 6;
-      const int n = n0 + nn, k = k0 + kk;
-      Bs[kk][nn] = (n < g.N && k < ke) ? __ldg(g.B + ix(g.Bk, k) + ix(g.Bn, n)) : 0.f;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < GBK; ++kk) {
-      float a[4], b[4];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) { a[t] = As[kk][ty * 4 + t]; b[t] = Bs[kk][tx * 4 + t]; }
-#pragma unroll
-      for (int p = 0; p < 4; ++p)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[p][q] = fmaf(a[p], b[q], acc[p][q]);
-    }
-    __syncthreads();
   }
 #pragma unroll
   for (int p = 0; p < 4; ++p) {
     const int m = m0 + ty * 4 + p;
-    if (m >= g.M) continue;
+    if (m >= P.M) continue;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int n = n0 + tx * 4 + q;
-      if (n >= g.N) continue;
+      if (n >= P.N) continue;
       if (g.splits > 1) {
-        g.partial[((long long)split * g.M + m) * g.N + n] = acc[p][q];
+        g.partial[P.part_off + ((long long)split * P.M + m) * P.N + n] = acc[p][q];
       } else {
-        float* c = g.C + ix(g.Cm, m) + ix(g.Cn, n);
+        float* c = P.C + ix(P.Cm, m) + ix(P.Cn, n);
         *c = g.accumulate ? *c + acc[p][q] : acc[p][q];
       }
     }
   }
 }
 
-__global__ void k_gemm_reduce(GemmArgs g) {
+// one thread per output element of every problem; fixed-order sum over splits
+__global__ void k_gemm_reduce(const __grid_constant__ GemmBatch g, long long total) {
   const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  const long long total = (long long)g.M * g.N;
   if (t >= total) return;
-  const int m = (int)(t / g.N), n = (int)(t % g.N);
+  int pi = 0;
+  long long base = 0;
+  while (pi < g.n_problems && t >= base + (long long)g.pr[pi].M * g.pr[pi].N) {
+    base += (long long)g.pr[pi].M * g.pr[pi].N;
+    ++pi;
+  }
+  const GemmProblem& P = g.pr[pi];
+  const long long loc = t - base;
+  const long long mn = (long long)P.M * P.N;
+  const int m = (int)(loc / P.N), n = (int)(loc % P.N);
   float s = 0.f;
-  for (int p = 0; p < g.splits; ++p) s += g.partial[(long long)p * total + t];
-  float* c = g.C + ix(g.Cm, m) + ix(g.Cn, n);
+  for (int sp = 0; sp < g.splits; ++sp) s += g.partial[P.part_off + sp * mn + loc];
+  float* c = P.C + ix(P.Cm, m) + ix(P.Cn, n);
   *c = g.accumulate ? *c + s : s;
 }
 
-cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
-  if (g.M <= 0 || g.N <= 0) return cudaSuccess;
-  if (g.K <= 0) return cudaSuccess;  // nothing to add (outputs are pre-cleared by callers)
-  dim3 grid((g.N + GBN - 1) / GBN, (g.M + GBM - 1) / GBM, g.splits);
-  k_gemm<<<grid, 256, 0, s>>>(g);
-  if (g.splits > 1) {
-    const long long total = (long long)g.M * g.N;
-    k_gemm_reduce<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(g);
+cudaError_t launch_gemm(GemmBatch& g, cudaStream_t s) {
+  int tiles = 0;
+  long long elems = 0;
+  for (int p = 0; p < g.n_problems; ++p) {
+    g.pr[p].tile0 = tiles;
+    g.pr[p].part_off = elems * g.splits;
+    tiles += ((g.pr[p].M + GBM - 1) / GBM) * ((g.pr[p].N + GBN - 1) / GBN);
+    elems += (long long)g.pr[p].M * g.pr[p].N;
   }
+  g.total_tiles = tiles;
+  if (tiles == 0) return cudaSuccess;
+  k_gemm<<<dim3(tiles, g.splits), 256, 0, s>>>(g);
+  if (g.splits > 1) k_gemm_reduce<<<(unsigned)((elems + 255) / 256), 256, 0, s>>>(g, elems);
   return cudaGetLastError();
 }
 

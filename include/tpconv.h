@@ -186,6 +186,19 @@ tpconv_status tpconv_double_backward(tpconv_plan_t plan, int64_t N, int64_t E, c
                                      float* grad_W, float* grad_grad_out, float* grad_pos,
                                      void* ws, size_t ws_bytes, struct CUstream_st* stream);
 
+/* Profiling (off by default; host-side bookkeeping only).  While enabled, every kernel
+ * the library launches is bracketed by a pair of CUDA events on its stream and
+ * attributed to a category (tpconv_profile_category_name).  tpconv_profile_begin
+ * clears the records (capacity: max_records launches; later launches are counted but
+ * not timed).  tpconv_profile_end waits for the recorded events, writes per-category
+ * total device milliseconds and launch counts into ms[n] / launches[n] (either may be
+ * NULL; n <= TPCONV_PROF_CATEGORIES) and disables recording.  Not for use during
+ * stream capture.                                                                     */
+#define TPCONV_PROF_CATEGORIES 12
+tpconv_status tpconv_profile_begin(int32_t max_records);
+tpconv_status tpconv_profile_end(double* ms, int64_t* launches, int32_t n);
+const char* tpconv_profile_category_name(int32_t category);
+
 #ifdef __cplusplus
 }
 #endif

@@ -89,7 +89,8 @@ def receivers_of(row_ptr):
 
 def _edge_batches(n_edges, n_w, edges):
     ids = np.arange(n_edges) if edges is None else np.asarray(edges, dtype=np.int64)
-    step = max(1, int(2 ** 25 // max(1, n_w)))
+    # temporaries stay below ~16 MB so the allocator reuses memory across batches
+    step = max(1, int(2 ** 21 // max(1, n_w)))
     for s in range(0, ids.shape[0], step):
         yield ids[s:s + step]
 
@@ -127,6 +128,15 @@ def _geometry(plan, pos, src, dst, eb, need_grad):
 
 def _f64(a):
     return None if a is None else np.asarray(a, dtype=np.float64)
+
+
+def _radial_project(phi, A):
+    """Eq. 12: w_{e,c} = sum_q phi_{e,q} A_{q,c}, written out as a sum over q (a BLAS
+    matmul with this very short inner dimension is pathologically slow in OpenBLAS)."""
+    w = np.zeros((phi.shape[0], A.shape[1]))
+    for q in range(A.shape[0]):
+        w += phi[:, q:q + 1] * A[q][None, :]
+    return w
 
 
 def _wslice(plan, p, w):
@@ -172,7 +182,7 @@ def forward(plan, x, pos, row_ptr, src, A, edges=None):
         if eb.size == 0:
             continue
         Y, _, phi, _ = _geometry(plan, pos, src, dst, eb, False)
-        w = phi @ A                                     # eqs. 12-13: W = phi A
+        w = _radial_project(phi, A)                     # eqs. 12-13: W = phi A
         xs = x[src[eb]]
         z = np.zeros((eb.size, plan.dim_out))
         for p, c in zip(plan.paths, plan.coupling):
@@ -201,7 +211,7 @@ def backward(plan, x, pos, row_ptr, src, A, grad_out, edges=None):
         if eb.size == 0:
             continue
         Y, dY, phi, dphi = _geometry(plan, pos, src, dst, eb, True)
-        w = phi @ A
+        w = _radial_project(phi, A)
         xs = x[src[eb]]
         mb_rows = mbar[dst[eb]]
         h = np.zeros((eb.size, plan.n_w))
@@ -250,8 +260,8 @@ def double_backward(plan, x, pos, row_ptr, src, A, grad_out, gg_x=None, gg_pos=N
         rdot = pd[src[eb]] - pd[dst[eb]]
         Ydot = np.einsum("esk,ek->es", dY, rdot)
         phidot = np.einsum("eqk,ek->eq", dphi, rdot)
-        w = phi @ A
-        wdot = phidot @ A + phi @ Ad                                              # eq. 23
+        w = _radial_project(phi, A)
+        wdot = _radial_project(phidot, A) + _radial_project(phi, Ad)            # eq. 23
         xs, xds = x[src[eb]], xd[src[eb]]
         mb_rows = mbar[dst[eb]]
         h = np.zeros((eb.size, plan.n_w))
