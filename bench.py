@@ -45,6 +45,12 @@ def _workload_config(c, E):
             "pass": "forward + backward (x, pos, W)", "l2": "flushed between timed steps"}
 
 
+def _config_line(c, g):
+    d = _workload_config(c, g.n_edges)
+    d["nodes"] = g.n_nodes
+    return d
+
+
 def _dist():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -146,7 +152,7 @@ def run_native(args):
     c = workloads.CONFIGS[CFG]
     plan = binding.Plan(c.irreps_in, c.sh_lmax, c.irreps_out, c.mode, c.radial, c.num_basis, c.r_cut,
                         c.r_min, c.r_max)
-    g, rng = workloads.make_graph(c, seed=1000 + CFG + 7919 * rank)
+    g, rng = workloads.make_graph(c, n_nodes=args.nodes, seed=1000 + CFG + 7919 * rank)
     N, E = g.n_nodes, g.n_edges
     x_h = workloads.normal(rng, (N, plan.dim_in))
     W_h = workloads.weights(rng, c.num_basis, plan.fan_in_per_column())
@@ -283,7 +289,7 @@ def run_native(args):
         line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-                "config": _workload_config(c, E), "impl": "native",
+                "config": _config_line(c, g), "impl": "native",
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": gpu_launches,
                 "gpu_launches_per_step": gpu_launches / args.steps, "clocks": clocks,
                 "workspace_bytes": {"declared": int(ws_bytes), "peak_alloc_delta": int(peak_delta)},
@@ -374,6 +380,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--nodes", type=int, default=None,
+                    help="resize the workload (same density and degree); for profiling small cases")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "native":
         args.warmup = 3
