@@ -47,6 +47,7 @@ SIGNATURES = {
     "tpconv_profile_begin": (ctypes.c_int, [ctypes.c_int32]),
     "tpconv_profile_end": (ctypes.c_int, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_c_i64), ctypes.c_int32]),
     "tpconv_profile_category_name": (ctypes.c_char_p, [ctypes.c_int32]),
+    "tpconv_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int32)]),
 }
 PROF_CATEGORIES = 12
 
@@ -278,3 +279,10 @@ def tpconv_profile_end():
     cnt = (_c_i64 * n)()
     check(lib().tpconv_profile_end(ms, cnt, n), "tpconv_profile_end")
     return {lib().tpconv_profile_category_name(c).decode(): (ms[c], cnt[c]) for c in range(n)}
+
+
+def tpconv_device_error():
+    """Read and clear the library's device error word (0 = no bounded wait gave up)."""
+    v = ctypes.c_int32()
+    check(lib().tpconv_device_error(ctypes.byref(v)), "tpconv_device_error")
+    return v.value

@@ -204,6 +204,15 @@ int chunk_nodes(size_t budget, long long per_node_floats, int arrays, long long 
   return (int)c;
 }
 
+// floats of one split-K slice: the largest of the weight gradient, a receiver range of
+// outputs and a source range of input gradients
+long long part_floats(const tpconv_plan* P, const Layout& L) {
+  long long a = (long long)P->K * P->n_w;
+  a = std::max(a, (long long)L.recv_chunk * P->dim_out);
+  a = std::max(a, (long long)L.src_chunk * P->dim_in);
+  return a;
+}
+
 Layout make_layout(const tpconv_plan* P, long long N, long long E, uint32_t pass) {
   Layout L;
   size_t off = 0;
@@ -224,7 +233,7 @@ Layout make_layout(const tpconv_plan* P, long long N, long long E, uint32_t pass
     if (pass != TPCONV_PASS_FORWARD) {
       L.has_part = true;
       L.part = off;
-      off += align256(size_t(4) * kSplits * P->K * (long long)P->n_w);
+      off += align256(size_t(4) * kSplits * part_floats(P, L));
     }
   } else {
     if (pass != TPCONV_PASS_FORWARD) {
@@ -509,6 +518,17 @@ struct Batch {
     g.accumulate = accumulate;
     g.partial = partial;
   }
+  // Use split-K when the output tiles alone would leave SMs idle (needs `partial`).
+  cudaError_t launch(cudaStream_t st, float* part = nullptr) {
+    if (g.splits == 1 && part) {
+      const int tiles = gemm_tiles(g);
+      if (tiles > 0 && tiles < 2 * 148) {
+        g.splits = std::min(kSplits, (2 * 148 + tiles - 1) / tiles);
+        g.partial = part;
+      }
+    }
+    return launch_gemm(g, st);
+  }
   void problem(float* C, Idx2 Cm, Idx2 Cn, int M, int N) {
     GemmProblem& p = g.pr[g.n_problems++];
     p.C = C; p.Cm = Cm; p.Cn = Cn; p.M = M; p.N = N;
@@ -526,7 +546,7 @@ struct Batch {
 // m_g[(i,mo), w] = sum_{pi in g} sum_{q,u} S_pi[(i,mo),(q,u)] A_pi[(q,u), w]   (eqs. 34-35),
 // optionally + sum_pi S2_pi A2_pi (eq. 37: dm = dS A + S dA)
 cudaError_t gemm_state_times_A(const tpconv_plan* P, const float* S, const float* W, const float* S2,
-                               const float* W2, float* out, int n0, int cn, cudaStream_t st) {
+                               const float* W2, float* out, int n0, int cn, float* part, cudaStream_t st) {
   Batch b(1, 0, nullptr);
   for (int bo = 0; bo < (int)P->out.size(); ++bo) {
     const Block& B = P->out[bo];
@@ -543,7 +563,7 @@ cudaError_t gemm_state_times_A(const tpconv_plan* P, const float* S, const float
       if (S2) b.seg(S2 + p.st_off, Am, idx1(1), W2 + p.w_off, Bk, idx1(1), P->K * p.c_in);
     }
   }
-  return launch_gemm(b.g, st);
+  return b.launch(st, part);
 }
 
 // S_bar_pi[(i,mo),(q,u)] = sum_w m_bar[(i,mo), w] A_pi[(q,u), w]        (eq. 36)
@@ -563,7 +583,7 @@ cudaError_t gemm_sbar(const tpconv_plan* P, const float* gout, const float* W, f
 // x_bar[(j,mi), u] = sum_{pi from block} sum_{q,w} X_pi[(j,mi),(q,w)] A_pi[(q,u), w]
 // (mirrored eq. 21), optionally + X2 A2^T (eq. 30 with A_dot)
 cudaError_t gemm_xbar(const tpconv_plan* P, const float* X, const float* W, const float* X2, const float* W2,
-                      float* gx, int n0, int cn, cudaStream_t st) {
+                      float* gx, int n0, int cn, float* part, cudaStream_t st) {
   Batch b(1, 0, nullptr);
   for (int bi = 0; bi < (int)P->in.size(); ++bi) {
     const Block& B = P->in[bi];
@@ -580,18 +600,19 @@ cudaError_t gemm_xbar(const tpconv_plan* P, const float* X, const float* W, cons
       if (X2) b.seg(X2 + p.xst_off, Am, idx1(1), W2 + p.w_off, Bk, idx1(p.c_out), P->K * p.c_out);
     }
   }
-  return launch_gemm(b.g, st);
+  return b.launch(st, part);
 }
 
 // A_bar_pi[(q,u), w] (+)= sum_{(j,mi)} x[(j,mi), u] X_pi[(j,mi),(q,w)]     (mirrored eq. 19)
+// computed as its transpose, rows (q,w) and columns u, so the wide side fills the MMA rows
 cudaError_t gemm_abar_src(const tpconv_plan* P, const float* x, const float* X, float* gW, int n0, int cn,
                           int accumulate, float* part, cudaStream_t st) {
   Batch b(kSplits, accumulate, part);
   for (const PathH& p : P->paths) {
     const int RI = 2 * p.l_in + 1;
-    b.problem(gW + p.w_off, idx1(p.c_out), idx2(p.c_out, P->n_w, 1), p.c_in, P->K * p.c_out);
-    b.seg(x + (long long)n0 * P->dim_in + p.in_off, idx1(1), idx2(RI, P->dim_in, p.c_in), X + p.xst_off,
-          idx2(RI, P->dev.xstate_per_node, (long long)P->K * p.c_out), idx1(1), cn * RI);
+    b.problem(gW + p.w_off, idx2(p.c_out, P->n_w, 1), idx1(p.c_out), P->K * p.c_out, p.c_in);
+    b.seg(X + p.xst_off, idx1(1), idx2(RI, P->dev.xstate_per_node, (long long)P->K * p.c_out),
+          x + (long long)n0 * P->dim_in + p.in_off, idx2(RI, P->dim_in, p.c_in), idx1(1), cn * RI);
   }
   return launch_gemm(b.g, st);
 }
@@ -651,7 +672,7 @@ tpconv_status tpconv_forward(tpconv_plan_t P, int64_t N, int64_t E, const float*
     const int cn = std::min(L.recv_chunk, n - n0);
     TPC_RUN(PC_UVW_STATE, 1, launch_uvw_state(P->dev, P->t_in, 0, x, nullptr, pos, nullptr, row_ptr, src, n0, cn, S,
                              nullptr, s));
-    TPC_RUN(PC_GEMM, 1, gemm_state_times_A(P, S, W, nullptr, nullptr, out, n0, cn, s));
+    TPC_RUN(PC_GEMM, 1, gemm_state_times_A(P, S, W, nullptr, nullptr, out, n0, cn, nullptr, s));
   }
   return TPCONV_OK;
 }
@@ -713,7 +734,7 @@ tpconv_status tpconv_backward(tpconv_plan_t P, int64_t N, int64_t E, const float
       const int cn = std::min(L.src_chunk, n - n0);
       TPC_RUN(PC_UVW_SRC, 1, launch_uvw_src_state(P->dev, P->t_out, 0, pos, nullptr, t_ptr, t_eid, t_dst, grad_out, n0,
                                    cn, state, nullptr, s));
-      if (grad_x) TPC_RUN(PC_GEMM, 1, gemm_xbar(P, state, W, nullptr, nullptr, grad_x, n0, cn, s));
+      if (grad_x) TPC_RUN(PC_GEMM, 1, gemm_xbar(P, state, W, nullptr, nullptr, grad_x, n0, cn, part, s));
       if (grad_W) TPC_RUN(PC_GEMM, 2, gemm_abar_src(P, x, state, grad_W, n0, cn, n0 > 0, part, s));
     }
   }
@@ -779,7 +800,7 @@ tpconv_status tpconv_double_backward(tpconv_plan_t P, int64_t N, int64_t E, cons
                                need_S ? sb : nullptr, sa, s));
       if (grad_grad_out)
         TPC_RUN(PC_GEMM, 1, gemm_state_times_A(P, tan_xp ? sa : nullptr, W, need_S ? sb : nullptr, gg_W, grad_grad_out, n0,
-                                   cn, s));
+                                   cn, part, s));
       if (grad_W && tan_xp) TPC_RUN(PC_GEMM, 2, gemm_abar_recv(P, sa, grad_out, grad_W, n0, cn, n0 > 0, part, s));
     }
   }
@@ -792,7 +813,7 @@ tpconv_status tpconv_double_backward(tpconv_plan_t P, int64_t N, int64_t E, cons
         // sa = X' (tangent of the source state), sb = X
         TPC_RUN(PC_UVW_SRC_TAN, 1, launch_uvw_src_state(P->dev, P->t_out, 1, pos, gg_pos, t_ptr, t_eid, t_dst, grad_out, n0,
                                      cn, gg_W ? sb : nullptr, sa, s));
-        TPC_RUN(PC_GEMM, 1, gemm_xbar(P, gg_pos ? sa : nullptr, W, gg_W ? sb : nullptr, gg_W, grad_x, n0, cn, s));
+        TPC_RUN(PC_GEMM, 1, gemm_xbar(P, gg_pos ? sa : nullptr, W, gg_W ? sb : nullptr, gg_W, grad_x, n0, cn, part, s));
       }
     }
   }
@@ -838,6 +859,14 @@ tpconv_status tpconv_profile_end(double* ms, int64_t* launches, int32_t n) {
   P.on = false;
   P.used = 0;
   return st;
+}
+
+tpconv_status tpconv_device_error(int32_t* out) {
+  if (!out) return TPCONV_ERR_INVALID_ARG;
+  int v = 0;
+  if (read_and_clear_device_error(&v) != cudaSuccess) return TPCONV_ERR_CUDA;
+  *out = v;
+  return TPCONV_OK;
 }
 
 const char* tpconv_profile_category_name(int32_t c) {

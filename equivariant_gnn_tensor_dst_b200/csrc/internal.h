@@ -128,7 +128,12 @@ cudaError_t run_uvu_src(const DevPlan& P, const BlockPaths& BP, const Tasks& T, 
                         cudaStream_t s);
 
 // kernel launchers (dispatch on K and mode; defined in launch.cu and k_misc.cu)
-cudaError_t launch_gemm(GemmBatch& g, cudaStream_t s);  // fills tile0 / total_tiles
+cudaError_t launch_gemm(GemmBatch& g, cudaStream_t s);     // tensor cores; fills tile0 / total_tiles
+cudaError_t launch_gemm_simt(GemmBatch& g, cudaStream_t s);  // fp32 SIMT tiles (reference kernel)
+cudaError_t launch_gemm_tc(GemmBatch& g, int* err, cudaStream_t s);
+int gemm_tiles(const GemmBatch& g);                             // output tiles of the tensor-core kernel
+int* device_error_word();                                       // set by bounded waits that give up
+cudaError_t read_and_clear_device_error(int* host_value);
 
 cudaError_t launch_uvw_state(const DevPlan& P, const Tasks& T, int mode, const float* x,
                              const float* xdot, const float* pos, const float* posdot,

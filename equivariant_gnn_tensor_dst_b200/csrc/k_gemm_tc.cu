@@ -1,0 +1,332 @@
+// Channel contractions on the 5th-generation tensor cores (tcgen05, accumulator in TMEM).
+//
+// Sobek, section 4: the receiver state S is contracted with the radial parameters A
+// as one matrix product per output group (m = S A, eqs. 34-35); backward uses
+// S_bar = m_bar A^T and A_bar = S^T m_bar (eq. 36), double backward eqs. 37-39, and the
+// source side the mirrored x_bar = X A^T and A_bar = x^T X.  These are the only dense
+// contractions of the method.
+//
+// fp32 accuracy from TF32 tensor cores: every operand value a is split as
+// a = hi + lo with hi = tf32(a) (round to nearest) and lo = tf32(a - hi); each k-step
+// issues hi*hi + hi*lo + lo*hi into the same fp32 accumulator ("3xTF32", the
+// decomposition of Ootomo and Yokota, 2022), which keeps the relative error near
+// 2^-21 instead of TF32's 2^-11.
+//
+// Structure: one CTA of 128 threads per 128 x NT output tile (NT = 64 or 128) and
+// split-K slice.  All threads stage operand tiles from global memory through the same
+// two-level affine index maps as the rest of the library (so ir_mul node rows, weight
+// columns and workspace states are read in place), split them and store them in the
+// canonical K-major, no-swizzle core-matrix layout (8 rows x 16 bytes per core
+// matrix).  Two stages: while thread 0's MMAs of stage s run asynchronously, the CTA
+// fills stage s+1; a tcgen05.commit per stage arrives on that stage's mbarrier.  The
+// epilogue reads the TMEM accumulator with tcgen05.ld (one TMEM lane = one output row)
+// and writes C (or the split-K partial) through the output map.  Every mbarrier wait is
+// bounded; a wait that gives up sets *err and the kernel still releases its TMEM.
+#include <cuda_runtime.h>
+#include <cstdint>
+#include "internal.h"
+
+namespace tpc {
+
+namespace {
+
+constexpr int TC_M = 128;
+constexpr int TC_K = 32;           // k elements per stage (8 core-matrix columns)
+constexpr int TC_THREADS = 128;
+constexpr unsigned kWaitLimit = 1u << 20;
+
+__device__ __forceinline__ long long ixd(const Idx2& f, int i) {
+  return (long long)(i / f.d) * f.s1 + (long long)(i % f.d) * f.s2;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ float to_tf32(float a) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(a));
+  return __uint_as_float(r);
+}
+
+// byte offset of element (row, k) inside a [rows x 32] K-major no-swizzle tile
+__device__ __forceinline__ uint32_t tile_off(int row, int k) {
+  return (uint32_t)((row >> 3) * 1024 + (k >> 2) * 128 + (row & 7) * 16 + (k & 3) * 4);
+}
+
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
+  // start address, LBO = 128 B (next k core matrix), SBO = 1024 B (next 8-row group),
+  // descriptor version 1, no swizzle
+  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)(128 >> 4) << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         (1ull << 46);
+}
+
+template <int NT>
+__host__ __device__ constexpr uint32_t instr_desc() {
+  // D fp32 (bits 4-5 = 1), A and B tf32 (bits 7-9, 10-12 = 2), both K-major,
+  // N >> 3 at bits 17-22, M >> 4 at bits 24-28
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(NT >> 3) << 17) | ((uint32_t)(TC_M >> 4) << 24);
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  for (unsigned it = 0; it < kWaitLimit; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+
+// Stage the rows [r0, r0 + nrows) x k in [kt, kt + 32) of an operand X(r, k) into
+// hi/lo tiles.  Thread t owns row (t % rows_per_pass) and a contiguous k range.
+__device__ __forceinline__ void stage_operand(const float* __restrict__ base, const Idx2& mr,
+                                              const Idx2& mk, int r0, int rmax, int kt, int khi,
+                                              int nrows, char* hi, char* lo) {
+  const int t = threadIdx.x;
+  const int kparts = TC_THREADS / nrows;            // 1 (nrows = 128) or 2 (nrows = 64)
+  const int row = t % nrows;
+  const int kw = TC_K / kparts;
+  const int kbeg = (t / nrows) * kw;
+  const int r = r0 + row;
+  const bool rok = r < rmax;
+  const long long rbase = rok ? ixd(mr, r) : 0;
+  // contiguous k inside the stage when the k map does not cross a block boundary
+  const bool lin = (kt % mk.d) + TC_K <= mk.d;
+  const long long kbase = ixd(mk, kt);
+#pragma unroll 4
+  for (int k4 = kbeg; k4 < kbeg + kw; k4 += 4) {
+    float v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int k = kt + k4 + j;
+      float a = 0.f;
+      if (rok && k < khi) {
+        const long long ko = lin ? kbase + (long long)(k4 + j) * mk.s2 : ixd(mk, k);
+        a = __ldg(base + rbase + ko);
+      }
+      v[j] = a;
+    }
+    float4 h, l;
+    h.x = to_tf32(v[0]); l.x = to_tf32(v[0] - h.x);
+    h.y = to_tf32(v[1]); l.y = to_tf32(v[1] - h.y);
+    h.z = to_tf32(v[2]); l.z = to_tf32(v[2] - h.z);
+    h.w = to_tf32(v[3]); l.w = to_tf32(v[3] - h.w);
+    const uint32_t off = tile_off(row, k4);
+    *reinterpret_cast<float4*>(hi + off) = h;
+    *reinterpret_cast<float4*>(lo + off) = l;
+  }
+}
+
+template <int NT>
+struct TcSmem {
+  static constexpr int A_BYTES = TC_M * TC_K * 4;
+  static constexpr int B_BYTES = NT * TC_K * 4;
+  static constexpr int STAGE = 2 * A_BYTES + 2 * B_BYTES;
+  static constexpr int TOTAL = 2 * STAGE + 2048;  // + alignment slack, barriers, TMEM address
+};
+
+template <int NT>
+__global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ GemmBatch g, int* err) {
+  extern __shared__ char smem_raw[];
+  char* smem = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  char* stage_base[2] = {smem, smem + TcSmem<NT>::STAGE};
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * TcSmem<NT>::STAGE);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + 2 * TcSmem<NT>::STAGE + 64);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // locate (problem, m tile, n tile)
+  const int tile = blockIdx.x;
+  int pi = 0;
+  while (pi + 1 < g.n_problems && g.pr[pi + 1].tile0 <= tile) ++pi;
+  const GemmProblem& P = g.pr[pi];
+  const int lt = tile - P.tile0;
+  const int tn = (P.N + NT - 1) / NT;
+  const int m0 = (lt / tn) * TC_M, n0 = (lt % tn) * NT;
+  const int split = blockIdx.y;
+  const int kper = (P.Ktot + g.splits - 1) / g.splits;
+  const int kb = split * kper, ke = min(P.Ktot, kb + kper);
+
+  if (tid == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[0])));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[1])));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(NT));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *tmem_slot;
+
+  constexpr uint32_t IDESC = instr_desc<NT>();
+  uint32_t phase[2] = {0u, 0u};
+  int it = 0;
+  bool ok = true;
+  int kbase = 0;
+  for (int si = 0; si < P.nseg; ++si) {
+    const GemmSeg& S = g.sg[P.seg0 + si];
+    const int lo = max(kb - kbase, 0), hi = min(ke - kbase, S.K);
+    kbase += S.K;
+    for (int kt = lo; kt < hi; kt += TC_K) {
+      const int st = it & 1;
+      if (it >= 2) {  // stage st was read by the MMAs committed two iterations ago
+        ok = mbar_wait(smem_u32(&bars[st]), phase[st]) && ok;
+        phase[st] ^= 1u;
+      }
+      char* sb = stage_base[st];
+      stage_operand(S.A, S.Am, S.Ak, m0, P.M, kt, hi, TC_M, sb, sb + TcSmem<NT>::A_BYTES);
+      stage_operand(S.B, S.Bn, S.Bk, n0, P.N, kt, hi, NT, sb + 2 * TcSmem<NT>::A_BYTES,
+                    sb + 2 * TcSmem<NT>::A_BYTES + TcSmem<NT>::B_BYTES);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      __syncthreads();
+      if (tid == 0) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t a_hi = smem_u32(sb), a_lo = a_hi + TcSmem<NT>::A_BYTES;
+        const uint32_t b_hi = a_hi + 2 * TcSmem<NT>::A_BYTES, b_lo = b_hi + TcSmem<NT>::B_BYTES;
+#pragma unroll
+        for (int ks = 0; ks < TC_K / 8; ++ks) {
+          const uint32_t koff = ks * 256;  // two 16-byte core-matrix columns per K=8 step
+          const uint64_t dah = smem_desc(a_hi + koff), dal = smem_desc(a_lo + koff);
+          const uint64_t dbh = smem_desc(b_hi + koff), dbl = smem_desc(b_lo + koff);
+          const uint32_t acc0 = (it > 0 || ks > 0) ? 1u : 0u;
+          asm volatile(
+              "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+              "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
+              "l"(dah), "l"(dbh), "r"(IDESC), "r"(acc0));
+          asm volatile(
+              "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+              "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
+              "l"(dah), "l"(dbl), "r"(IDESC), "r"(1u));
+          asm volatile(
+              "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+              "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
+              "l"(dal), "l"(dbh), "r"(IDESC), "r"(1u));
+        }
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                         smem_u32(&bars[st]))
+                     : "memory");
+      }
+      ++it;
+    }
+  }
+  // wait for the last commit (tcgen05 operations complete in issue order)
+  if (it > 0) {
+    const int st = (it - 1) & 1;
+    ok = mbar_wait(smem_u32(&bars[st]), phase[st]) && ok;
+  }
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+
+  // epilogue: TMEM lane (32 * warp + lane) holds output row m0 + 32 * warp + lane
+  const int m = m0 + warp * 32 + lane;
+  const bool mok = m < P.M;
+  const long long cm = mok ? ixd(P.Cm, m) : 0;
+#pragma unroll 1
+  for (int c0 = 0; c0 < NT; c0 += 32) {
+    uint32_t r[32];
+    const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0;
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+    if (mok) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int n = n0 + c0 + j;
+        if (n >= P.N) break;
+        const float v = (it > 0) ? __uint_as_float(r[j]) : 0.f;
+        if (g.splits > 1) {
+          g.partial[P.part_off + ((long long)split * P.M + m) * P.N + n] = v;
+        } else {
+          float* c = P.C + cm + ixd(P.Cn, n);
+          *c = g.accumulate ? *c + v : v;
+        }
+      }
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 0) {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(NT));
+  }
+  if (!ok && tid == 0 && err) atomicExch(err, 1);
+}
+
+}  // namespace
+
+__global__ void k_gemm_tc_reduce(const __grid_constant__ GemmBatch g, long long total) {
+  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= total) return;
+  int pi = 0;
+  long long base = 0;
+  while (pi < g.n_problems && t >= base + (long long)g.pr[pi].M * g.pr[pi].N) {
+    base += (long long)g.pr[pi].M * g.pr[pi].N;
+    ++pi;
+  }
+  const GemmProblem& P = g.pr[pi];
+  const long long loc = t - base;
+  const long long mn = (long long)P.M * P.N;
+  const int m = (int)(loc / P.N), n = (int)(loc % P.N);
+  float s = 0.f;
+  for (int sp = 0; sp < g.splits; ++sp) s += g.partial[P.part_off + sp * mn + loc];
+  float* c = P.C + ixd(P.Cm, m) + ixd(P.Cn, n);
+  *c = g.accumulate ? *c + s : s;
+}
+
+template <int NT>
+static cudaError_t run_tc(GemmBatch& g, int* err, cudaStream_t s) {
+  static bool attr_set = false;  // per device-agnostic process; the attribute is per function
+  const int smem = TcSmem<NT>::TOTAL;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  int tiles = 0;
+  long long elems = 0;
+  for (int p = 0; p < g.n_problems; ++p) {
+    g.pr[p].tile0 = tiles;
+    g.pr[p].part_off = elems * g.splits;
+    tiles += ((g.pr[p].M + TC_M - 1) / TC_M) * ((g.pr[p].N + NT - 1) / NT);
+    elems += (long long)g.pr[p].M * g.pr[p].N;
+  }
+  g.total_tiles = tiles;
+  if (tiles == 0) return cudaSuccess;
+  k_gemm_tc<NT><<<dim3(tiles, g.splits), TC_THREADS, smem, s>>>(g, err);
+  if (g.splits > 1) k_gemm_tc_reduce<<<(unsigned)((elems + 255) / 256), 256, 0, s>>>(g, elems);
+  return cudaGetLastError();
+}
+
+int gemm_tiles(const GemmBatch& g) {
+  int maxN = 0;
+  for (int p = 0; p < g.n_problems; ++p) maxN = maxN > g.pr[p].N ? maxN : g.pr[p].N;
+  const int nt = maxN <= 64 ? 64 : 128;
+  int tiles = 0;
+  for (int p = 0; p < g.n_problems; ++p) tiles += ((g.pr[p].M + TC_M - 1) / TC_M) * ((g.pr[p].N + nt - 1) / nt);
+  return tiles;
+}
+
+cudaError_t launch_gemm_tc(GemmBatch& g, int* err, cudaStream_t s) {
+  int maxN = 0;
+  for (int p = 0; p < g.n_problems; ++p) maxN = maxN > g.pr[p].N ? maxN : g.pr[p].N;
+  if (maxN <= 64) return run_tc<64>(g, err, s);
+  return run_tc<128>(g, err, s);
+}
+
+}  // namespace tpc

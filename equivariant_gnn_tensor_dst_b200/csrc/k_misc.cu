@@ -113,7 +113,7 @@ __global__ void k_gemm_reduce(const __grid_constant__ GemmBatch g, long long tot
   *c = g.accumulate ? *c + s : s;
 }
 
-cudaError_t launch_gemm(GemmBatch& g, cudaStream_t s) {
+cudaError_t launch_gemm_simt(GemmBatch& g, cudaStream_t s) {
   int tiles = 0;
   long long elems = 0;
   for (int p = 0; p < g.n_problems; ++p) {
@@ -127,6 +127,25 @@ cudaError_t launch_gemm(GemmBatch& g, cudaStream_t s) {
   k_gemm<<<dim3(tiles, g.splits), 256, 0, s>>>(g);
   if (g.splits > 1) k_gemm_reduce<<<(unsigned)((elems + 255) / 256), 256, 0, s>>>(g, elems);
   return cudaGetLastError();
+}
+
+__device__ int g_tpc_error = 0;
+
+int* device_error_word() {
+  static int* p = nullptr;
+  if (!p) cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_tpc_error);
+  return p;
+}
+
+cudaError_t launch_gemm(GemmBatch& g, cudaStream_t s) { return launch_gemm_tc(g, device_error_word(), s); }
+
+cudaError_t read_and_clear_device_error(int* host_value) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return e;
+  e = cudaMemcpyFromSymbol(host_value, g_tpc_error, sizeof(int));
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_tpc_error, &zero, sizeof(int));
 }
 
 __global__ void k_reduce_partials(const float* __restrict__ partial, int n_parts, long long n,

@@ -140,9 +140,9 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32)
               const float* __restrict__ Wdot, int N, float* out) {
   __shared__ USmem<KP> sm;
   const long long gw = (long long)blockIdx.x * WARPS_PER_CTA + (threadIdx.x >> 5);
-  const int i = (int)(gw / T.n);
-  const int task = (int)(gw % T.n);
-  if (i >= N) return;
+  const int task = (int)(gw / N);   // task-major: co-resident warps share code
+  const int i = (int)(gw % N);
+  if (task >= T.n) return;
   const int bo = T.a[task];
   const int lane = threadIdx.x & 31;
   const int u = T.b[task] * 32 + lane;
@@ -380,9 +380,9 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32)
                 const float* __restrict__ gout, int N, int n_ranges, float* partial) {
   __shared__ USmem<KP> sm;
   const long long gw = (long long)blockIdx.x * WARPS_PER_CTA + (threadIdx.x >> 5);
-  const int range = (int)(gw / T.n);
-  const int task = (int)(gw % T.n);
-  if (range >= n_ranges) return;
+  const int task = (int)(gw / n_ranges);
+  const int range = (int)(gw % n_ranges);
+  if (task >= T.n) return;
   const int r0 = (int)((long long)N * range / n_ranges);
   const int r1 = (int)((long long)N * (range + 1) / n_ranges);
   const DevPath& p = P.p[T.a[task]];
@@ -466,9 +466,9 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32)
               float* grad_x) {
   __shared__ USmem<KP> sm;
   const long long gw = (long long)blockIdx.x * WARPS_PER_CTA + (threadIdx.x >> 5);
-  const int j = (int)(gw / T.n);
-  const int task = (int)(gw % T.n);
-  if (j >= N) return;
+  const int task = (int)(gw / N);
+  const int j = (int)(gw % N);
+  if (task >= T.n) return;
   const int bi = T.a[task];
   const int lane = threadIdx.x & 31;
   const int u = T.b[task] * 32 + lane;

@@ -169,10 +169,12 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32)
                 const int* __restrict__ row_ptr, const int* __restrict__ src, int node0,
                 int n_nodes, float* S, float* Sd) {
   __shared__ GeoSmem<KP> sm;
+  // task-major order: co-resident warps run the same (l_in, l_sh, l_out) body, which keeps
+  // the instruction working set small
   const long long gw = (long long)blockIdx.x * WARPS_PER_CTA + (threadIdx.x >> 5);
-  const int node_local = (int)(gw / T.n);
-  const int task = (int)(gw % T.n);
-  if (node_local >= n_nodes) return;
+  const int task = (int)(gw / n_nodes);
+  const int node_local = (int)(gw % n_nodes);
+  if (task >= T.n) return;
   const DevPath& p = P.p[T.a[task]];
   const int chunk = T.b[task];
   const int i = node0 + node_local;
@@ -189,10 +191,10 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32)
 
 template <int KP>
 struct RecvSmem {
-  int j[WARPS_PER_CTA][32];
-  float Y[WARPS_PER_CTA][32][16];
-  float phi[WARPS_PER_CTA][32][KP];
-  float accY[WARPS_PER_CTA][32][16];
+  int j[32];
+  float Y[32][16];
+  float phi[32][KP];
+  float accY[WARPS_PER_CTA][32][16];   // per-warp partial sums, combined in warp order
   float accphi[WARPS_PER_CTA][32][KP];
 };
 
@@ -219,15 +221,15 @@ __device__ __forceinline__ void uvw_recv_body(const DevPlan& P, const DevPath& p
   const int yw = reduce_multi_index<8>(lane), pw_ = reduce_multi_index<KP>(lane);
   const bool ywr = reduce_multi_writer<8>(lane), pwr = reduce_multi_writer<KP>(lane);
   for (int t = 0; t < ne; ++t) {
-    const long long row = (long long)sm.j[w][t] * P.dim_in;
+    const long long row = (long long)sm.j[t] * P.dim_in;
     float xv[RI];
 #pragma unroll
     for (int m = 0; m < RI; ++m) xv[m] = act ? __ldg(xb + row + m * p.c_in) : 0.f;
     float Y[RS], phi[KP];
 #pragma unroll
-    for (int k = 0; k < RS; ++k) Y[k] = sm.Y[w][t][LS * LS + k];
+    for (int k = 0; k < RS; ++k) Y[k] = sm.Y[t][LS * LS + k];
 #pragma unroll
-    for (int q = 0; q < KP; ++q) phi[q] = sm.phi[w][t][q];
+    for (int q = 0; q < KP; ++q) phi[q] = sm.phi[t][q];
     float C[RO];
     cg_couple<LI, LS, LO>(xv, Y, C);
     float pp[KP];
@@ -258,6 +260,8 @@ __device__ __forceinline__ void uvw_recv_body(const DevPlan& P, const DevPath& p
   }
 }
 
+// One CTA per receiver; its warps split the (path, channel chunk) tasks and keep
+// per-warp partial sums of phi_bar and Y_bar per edge, added in warp order.
 template <int KP>
 __global__ void __launch_bounds__(WARPS_PER_CTA * 32)
     k_uvw_recv_bwd(DevPlan P, Tasks T, const float* __restrict__ x, const float* __restrict__ pos,
@@ -265,27 +269,29 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32)
                    const float* __restrict__ Sbar, int node0, int n_nodes, float4* gbuf) {
   __shared__ RecvSmem<KP> sm;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int node_local = blockIdx.x * WARPS_PER_CTA + w;
+  const int node_local = blockIdx.x;
   if (node_local >= n_nodes) return;
   const int i = node0 + node_local;
   const int eb = __ldg(row_ptr + i), ee = __ldg(row_ptr + i + 1);
   for (int e0 = eb; e0 < ee; e0 += 32) {
     const int ne = min(32, ee - e0);
-    if (lane < ne) {
+    if (w == 0 && lane < ne) {
       const int j = __ldg(src + e0 + lane);
       const EdgeGeo g = edge_geo(pos, i, j);
       const Pow3 pw(g.ux, g.uy, g.uz);
       float Y[16], phi[KP], dphi[KP];
       sh_all(pw, Y);
       radial<KP, false>(P, g.d, phi, dphi);
-      sm.j[w][lane] = j;
+      sm.j[lane] = j;
 #pragma unroll
-      for (int k = 0; k < 16; ++k) { sm.Y[w][lane][k] = Y[k]; sm.accY[w][lane][k] = 0.f; }
+      for (int k = 0; k < 16; ++k) sm.Y[lane][k] = Y[k];
 #pragma unroll
-      for (int q = 0; q < KP; ++q) { sm.phi[w][lane][q] = phi[q]; sm.accphi[w][lane][q] = 0.f; }
+      for (int q = 0; q < KP; ++q) sm.phi[lane][q] = phi[q];
     }
-    __syncwarp();
-    for (int task = 0; task < T.n; ++task) {
+    for (int k = threadIdx.x; k < WARPS_PER_CTA * 32 * 16; k += blockDim.x) (&sm.accY[0][0][0])[k] = 0.f;
+    for (int k = threadIdx.x; k < WARPS_PER_CTA * 32 * KP; k += blockDim.x) (&sm.accphi[0][0][0])[k] = 0.f;
+    __syncthreads();
+    for (int task = w; task < T.n; task += WARPS_PER_CTA) {
       const DevPath& p = P.p[T.a[task]];
       const int chunk = T.b[task];
       dispatch_type(p.type, [&](auto tr) {
@@ -293,21 +299,31 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32)
         uvw_recv_body<TR::li, TR::ls, TR::lo, KP>(P, p, chunk, node_local, ne, x, Sbar, sm);
       });
     }
-    __syncwarp();
-    if (lane < ne) {
-      const int j = sm.j[w][lane];
+    __syncthreads();
+    if (w == 0 && lane < ne) {
+      const int j = sm.j[lane];
       const EdgeGeo g = edge_geo(pos, i, j);
       const Pow3 pw(g.ux, g.uy, g.uz);
       float phi[KP], dphi[KP], Yb[16];
       radial<KP, true>(P, g.d, phi, dphi);
 #pragma unroll
-      for (int k = 0; k < 16; ++k) Yb[k] = sm.accY[w][lane][k];
+      for (int k = 0; k < 16; ++k) {
+        float s = 0.f;
+#pragma unroll
+        for (int ww = 0; ww < WARPS_PER_CTA; ++ww) s += sm.accY[ww][lane][k];
+        Yb[k] = s;
+      }
       float vx = 0.f, vy = 0.f, vz = 0.f;
       sh_vjp_all(pw, Yb, vx, vy, vz);
       const float vr = vx * g.ux + vy * g.uy + vz * g.uz;
       float s = 0.f;
 #pragma unroll
-      for (int q = 0; q < KP; ++q) s = fmaf(sm.accphi[w][lane][q], dphi[q], s);
+      for (int q = 0; q < KP; ++q) {
+        float a = 0.f;
+#pragma unroll
+        for (int ww = 0; ww < WARPS_PER_CTA; ++ww) a += sm.accphi[ww][lane][q];
+        s = fmaf(a, dphi[q], s);
+      }
       float4 out;
       out.x = (vx - vr * g.ux) * g.inv_d + s * g.ux;
       out.y = (vy - vr * g.uy) * g.inv_d + s * g.uy;
@@ -315,7 +331,7 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32)
       out.w = 0.f;
       gbuf[e0 + lane] = out;
     }
-    __syncwarp();
+    __syncthreads();
   }
 }
 
@@ -411,10 +427,12 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32)
                     const int* __restrict__ t_dst, const float* __restrict__ gout, int node0,
                     int n_nodes, float* X, float* Xd) {
   __shared__ GeoSmem<KP> sm;
+  // task-major order: co-resident warps run the same (l_in, l_sh, l_out) body, which keeps
+  // the instruction working set small
   const long long gw = (long long)blockIdx.x * WARPS_PER_CTA + (threadIdx.x >> 5);
-  const int node_local = (int)(gw / T.n);
-  const int task = (int)(gw % T.n);
-  if (node_local >= n_nodes) return;
+  const int task = (int)(gw / n_nodes);
+  const int node_local = (int)(gw % n_nodes);
+  if (task >= T.n) return;
   const DevPath& p = P.p[T.a[task]];
   const int chunk = T.b[task];
   const int j = node0 + node_local;
@@ -447,7 +465,7 @@ template <int KP>
 cudaError_t run_uvw_recv_bwd(const DevPlan& P, const Tasks& T, const float* x, const float* pos,
                              const int* row_ptr, const int* src, const float* Sbar, int node0,
                              int n_nodes, float4* gbuf, cudaStream_t s) {
-  k_uvw_recv_bwd<KP><<<grid_for(n_nodes), WARPS_PER_CTA * 32, 0, s>>>(P, T, x, pos, row_ptr, src,
+  k_uvw_recv_bwd<KP><<<(unsigned)n_nodes, WARPS_PER_CTA * 32, 0, s>>>(P, T, x, pos, row_ptr, src,
                                                                      Sbar, node0, n_nodes, gbuf);
   return cudaGetLastError();
 }

@@ -195,6 +195,11 @@ tpconv_status tpconv_double_backward(tpconv_plan_t plan, int64_t N, int64_t E, c
  * NULL; n <= TPCONV_PROF_CATEGORIES) and disables recording.  Not for use during
  * stream capture.                                                                     */
 #define TPCONV_PROF_CATEGORIES 12
+
+/* Reads and clears the library's device error word (0 = fine; nonzero = a bounded wait
+ * inside a tensor-core kernel gave up, so results of that launch are invalid).
+ * Synchronises the current device; for tests and debugging.                        */
+tpconv_status tpconv_device_error(int32_t* out);
 tpconv_status tpconv_profile_begin(int32_t max_records);
 tpconv_status tpconv_profile_end(double* ms, int64_t* launches, int32_t n);
 const char* tpconv_profile_category_name(int32_t category);

@@ -308,3 +308,9 @@ def test_full_size_sampled(torch, cfg):
         assert rel_l2(gx2.cpu().numpy(), rx2) <= TOL
         assert rel_l2(gw2.cpu().numpy(), rw2) <= TOL
         assert rel_l2(gg2.cpu().numpy()[sample], rg2[sample]) <= TOL
+
+
+def test_no_device_error_after_runs(torch):
+    """Bounded waits inside the tensor-core kernels never gave up during this session."""
+    from equivariant_gnn_tensor_dst_b200 import binding
+    assert binding.tpconv_device_error() == 0
