@@ -537,6 +537,10 @@ struct Batch {
   void seg(const float* A, Idx2 Am, Idx2 Ak, const float* B, Idx2 Bk, Idx2 Bn, int K) {
     GemmSeg& s = g.sg[g.n_segs++];
     s.A = A; s.Am = Am; s.Ak = Ak; s.B = B; s.Bk = Bk; s.Bn = Bn; s.K = K;
+    // 16-byte vector loads along k: aligned base, row strides multiple of 4 floats,
+    // unit stride in k and k blocks (if any) of a multiple of 32
+    s.a_vec4 = ((reinterpret_cast<uintptr_t>(A) & 15u) == 0) && Am.s1 % 4 == 0 && Am.s2 % 4 == 0 &&
+               Ak.s2 == 1 && (Ak.d == 0x7fffffff || (Ak.d % 32 == 0 && Ak.s1 % 4 == 0));
     GemmProblem& p = g.pr[g.n_problems - 1];
     ++p.nseg;
     p.Ktot += K;

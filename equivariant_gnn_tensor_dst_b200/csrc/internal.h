@@ -72,6 +72,7 @@ struct GemmSeg {
   const float* A; Idx2 Am, Ak;   // A(m, k)
   const float* B; Idx2 Bk, Bn;   // B(k, n)
   int K;
+  int a_vec4;                    // A rows are 16-byte aligned and contiguous in k
 };
 
 struct GemmProblem {

@@ -83,41 +83,61 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   return false;
 }
 
-// Stage the rows [r0, r0 + nrows) x k in [kt, kt + 32) of an operand X(r, k) into
-// hi/lo tiles.  Thread t owns row (t % rows_per_pass) and a contiguous k range.
-__device__ __forceinline__ void stage_operand(const float* __restrict__ base, const Idx2& mr,
-                                              const Idx2& mk, int r0, int rmax, int kt, int khi,
-                                              int nrows, char* hi, char* lo) {
+// Operand staging is split in two halves so that the global loads of the next k-tile
+// are in flight while the current one is stored and its MMAs are issued.  Thread t
+// owns one operand row (row = t % nrows) and a contiguous range of kw = 32 / (128 /
+// nrows) k values.
+template <int KW>
+struct Frag {
+  float v[KW];
+};
+
+template <int KW>
+__device__ __forceinline__ void fetch_operand(const float* __restrict__ base, const Idx2& mr, const Idx2& mk,
+                                              int r0, int rmax, int kt, int khi, int nrows, bool vec4,
+                                              Frag<KW>& f) {
   const int t = threadIdx.x;
-  const int kparts = TC_THREADS / nrows;            // 1 (nrows = 128) or 2 (nrows = 64)
   const int row = t % nrows;
-  const int kw = TC_K / kparts;
-  const int kbeg = (t / nrows) * kw;
+  const int kbeg = (t / nrows) * KW;
   const int r = r0 + row;
   const bool rok = r < rmax;
   const long long rbase = rok ? ixd(mr, r) : 0;
-  // contiguous k inside the stage when the k map does not cross a block boundary
   const bool lin = (kt % mk.d) + TC_K <= mk.d;
   const long long kbase = ixd(mk, kt);
-#pragma unroll 4
-  for (int k4 = kbeg; k4 < kbeg + kw; k4 += 4) {
-    float v[4];
+  if (vec4 && lin && rok && ((kt & 3) == 0) && kt + kbeg + KW <= khi) {
+    const float4* p4 = reinterpret_cast<const float4*>(base + rbase + kbase + kbeg);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int k = kt + k4 + j;
-      float a = 0.f;
-      if (rok && k < khi) {
-        const long long ko = lin ? kbase + (long long)(k4 + j) * mk.s2 : ixd(mk, k);
-        a = __ldg(base + rbase + ko);
-      }
-      v[j] = a;
+    for (int q = 0; q < KW / 4; ++q) {
+      const float4 v = __ldg(p4 + q);
+      f.v[4 * q] = v.x; f.v[4 * q + 1] = v.y; f.v[4 * q + 2] = v.z; f.v[4 * q + 3] = v.w;
     }
+    return;
+  }
+#pragma unroll
+  for (int j = 0; j < KW; ++j) {
+    const int k = kt + kbeg + j;
+    float a = 0.f;
+    if (rok && k < khi) {
+      const long long ko = lin ? kbase + (long long)(kbeg + j) * mk.s2 : ixd(mk, k);
+      a = __ldg(base + rbase + ko);
+    }
+    f.v[j] = a;
+  }
+}
+
+template <int KW>
+__device__ __forceinline__ void store_operand(const Frag<KW>& f, int nrows, char* hi, char* lo) {
+  const int t = threadIdx.x;
+  const int row = t % nrows;
+  const int kbeg = (t / nrows) * KW;
+#pragma unroll
+  for (int q = 0; q < KW / 4; ++q) {
     float4 h, l;
-    h.x = to_tf32(v[0]); l.x = to_tf32(v[0] - h.x);
-    h.y = to_tf32(v[1]); l.y = to_tf32(v[1] - h.y);
-    h.z = to_tf32(v[2]); l.z = to_tf32(v[2] - h.z);
-    h.w = to_tf32(v[3]); l.w = to_tf32(v[3] - h.w);
-    const uint32_t off = tile_off(row, k4);
+    h.x = to_tf32(f.v[4 * q]);     l.x = to_tf32(f.v[4 * q] - h.x);
+    h.y = to_tf32(f.v[4 * q + 1]); l.y = to_tf32(f.v[4 * q + 1] - h.y);
+    h.z = to_tf32(f.v[4 * q + 2]); l.z = to_tf32(f.v[4 * q + 2] - h.z);
+    h.w = to_tf32(f.v[4 * q + 3]); l.w = to_tf32(f.v[4 * q + 3] - h.w);
+    const uint32_t off = tile_off(row, kbeg + 4 * q);
     *reinterpret_cast<float4*>(hi + off) = h;
     *reinterpret_cast<float4*>(lo + off) = l;
   }
@@ -149,7 +169,7 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
   const int tn = (P.N + NT - 1) / NT;
   const int m0 = (lt / tn) * TC_M, n0 = (lt % tn) * NT;
   const int split = blockIdx.y;
-  const int kper = (P.Ktot + g.splits - 1) / g.splits;
+  const int kper = ((P.Ktot + g.splits - 1) / g.splits + TC_K - 1) / TC_K * TC_K;
   const int kb = split * kper, ke = min(P.Ktot, kb + kper);
 
   if (tid == 0) {
@@ -168,56 +188,93 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
   const uint32_t tmem = *tmem_slot;
 
   constexpr uint32_t IDESC = instr_desc<NT>();
+  constexpr int KWB = TC_K / (TC_THREADS / NT);   // k values per thread for the B operand
   uint32_t phase[2] = {0u, 0u};
-  int it = 0;
   bool ok = true;
-  int kbase = 0;
-  for (int si = 0; si < P.nseg; ++si) {
-    const GemmSeg& S = g.sg[P.seg0 + si];
-    const int lo = max(kb - kbase, 0), hi = min(ke - kbase, S.K);
-    kbase += S.K;
-    for (int kt = lo; kt < hi; kt += TC_K) {
-      const int st = it & 1;
-      if (it >= 2) {  // stage st was read by the MMAs committed two iterations ago
-        ok = mbar_wait(smem_u32(&bars[st]), phase[st]) && ok;
-        phase[st] ^= 1u;
-      }
-      char* sb = stage_base[st];
-      stage_operand(S.A, S.Am, S.Ak, m0, P.M, kt, hi, TC_M, sb, sb + TcSmem<NT>::A_BYTES);
-      stage_operand(S.B, S.Bn, S.Bk, n0, P.N, kt, hi, NT, sb + 2 * TcSmem<NT>::A_BYTES,
-                    sb + 2 * TcSmem<NT>::A_BYTES + TcSmem<NT>::B_BYTES);
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-      __syncthreads();
-      if (tid == 0) {
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const uint32_t a_hi = smem_u32(sb), a_lo = a_hi + TcSmem<NT>::A_BYTES;
-        const uint32_t b_hi = a_hi + 2 * TcSmem<NT>::A_BYTES, b_lo = b_hi + TcSmem<NT>::B_BYTES;
-#pragma unroll
-        for (int ks = 0; ks < TC_K / 8; ++ks) {
-          const uint32_t koff = ks * 256;  // two 16-byte core-matrix columns per K=8 step
-          const uint64_t dah = smem_desc(a_hi + koff), dal = smem_desc(a_lo + koff);
-          const uint64_t dbh = smem_desc(b_hi + koff), dbl = smem_desc(b_lo + koff);
-          const uint32_t acc0 = (it > 0 || ks > 0) ? 1u : 0u;
-          asm volatile(
-              "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-              "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
-              "l"(dah), "l"(dbh), "r"(IDESC), "r"(acc0));
-          asm volatile(
-              "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-              "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
-              "l"(dah), "l"(dbl), "r"(IDESC), "r"(1u));
-          asm volatile(
-              "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-              "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
-              "l"(dal), "l"(dbh), "r"(IDESC), "r"(1u));
-        }
-        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                         smem_u32(&bars[st]))
-                     : "memory");
-      }
-      ++it;
+
+  // flat walk over the k-tiles of this split: (segment, kt) pairs
+  int seg = 0, kbase_seg = 0, kt = 0, khi = 0;
+  auto seg_range = [&](int si, int& lo, int& hi) {
+    const int K = g.sg[P.seg0 + si].K;
+    lo = max(kb - kbase_seg, 0);
+    hi = min(ke - kbase_seg, K);
+  };
+  // position on the first non-empty tile
+  bool have = false;
+  while (seg < P.nseg) {
+    int lo, hi;
+    seg_range(seg, lo, hi);
+    if (lo < hi) { kt = lo; khi = hi; have = true; break; }
+    kbase_seg += g.sg[P.seg0 + seg].K;
+    ++seg;
+  }
+  Frag<TC_K> fa;
+  Frag<KWB> fb;
+  if (have) {
+    const GemmSeg& S = g.sg[P.seg0 + seg];
+    fetch_operand<TC_K>(S.A, S.Am, S.Ak, m0, P.M, kt, khi, TC_M, S.a_vec4 != 0, fa);
+    fetch_operand<KWB>(S.B, S.Bn, S.Bk, n0, P.N, kt, khi, NT, false, fb);
+  }
+  int it = 0;
+  while (have) {
+    const int st = it & 1;
+    if (it >= 2) {  // stage st was read by the MMAs committed two iterations ago
+      ok = mbar_wait(smem_u32(&bars[st]), phase[st]) && ok;
+      phase[st] ^= 1u;
     }
+    char* sb = stage_base[st];
+    store_operand<TC_K>(fa, TC_M, sb, sb + TcSmem<NT>::A_BYTES);
+    store_operand<KWB>(fb, NT, sb + 2 * TcSmem<NT>::A_BYTES, sb + 2 * TcSmem<NT>::A_BYTES + TcSmem<NT>::B_BYTES);
+    // advance to the next tile and start its loads before this tile's MMAs
+    kt += TC_K;
+    if (kt >= khi) {
+      have = false;
+      kbase_seg += g.sg[P.seg0 + seg].K;
+      ++seg;
+      while (seg < P.nseg) {
+        int lo, hi;
+        seg_range(seg, lo, hi);
+        if (lo < hi) { kt = lo; khi = hi; have = true; break; }
+        kbase_seg += g.sg[P.seg0 + seg].K;
+        ++seg;
+      }
+    }
+    if (have) {
+      const GemmSeg& S = g.sg[P.seg0 + seg];
+      fetch_operand<TC_K>(S.A, S.Am, S.Ak, m0, P.M, kt, khi, TC_M, S.a_vec4 != 0, fa);
+      fetch_operand<KWB>(S.B, S.Bn, S.Bk, n0, P.N, kt, khi, NT, false, fb);
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (tid == 0) {
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t a_hi = smem_u32(sb), a_lo = a_hi + TcSmem<NT>::A_BYTES;
+      const uint32_t b_hi = a_hi + 2 * TcSmem<NT>::A_BYTES, b_lo = b_hi + TcSmem<NT>::B_BYTES;
+#pragma unroll
+      for (int ks = 0; ks < TC_K / 8; ++ks) {
+        const uint32_t koff = ks * 256;  // two 16-byte core-matrix columns per K=8 step
+        const uint64_t dah = smem_desc(a_hi + koff), dal = smem_desc(a_lo + koff);
+        const uint64_t dbh = smem_desc(b_hi + koff), dbl = smem_desc(b_lo + koff);
+        const uint32_t acc0 = (it > 0 || ks > 0) ? 1u : 0u;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
+            "l"(dah), "l"(dbh), "r"(IDESC), "r"(acc0));
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
+            "l"(dah), "l"(dbl), "r"(IDESC), "r"(1u));
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
+            "l"(dal), "l"(dbh), "r"(IDESC), "r"(1u));
+      }
+      asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                       smem_u32(&bars[st]))
+                   : "memory");
+    }
+    ++it;
   }
   // wait for the last commit (tcgen05 operations complete in issue order)
   if (it > 0) {
@@ -226,10 +283,10 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
   }
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 
-  // epilogue: TMEM lane (32 * warp + lane) holds output row m0 + 32 * warp + lane
-  const int m = m0 + warp * 32 + lane;
-  const bool mok = m < P.M;
-  const long long cm = mok ? ixd(P.Cm, m) : 0;
+  // epilogue: TMEM lane (32 * warp + lane) holds output row m0 + 32 * warp + lane.
+  // Each 32-column slice goes through shared memory (row stride 33 floats, conflict
+  // free) so that a warp then stores 32 consecutive columns of one row.
+  float* ep = reinterpret_cast<float*>(stage_base[0]);   // all MMAs are complete here
 #pragma unroll 1
   for (int c0 = 0; c0 < NT; c0 += 32) {
     uint32_t r[32];
@@ -244,16 +301,21 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
           "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-    if (mok) {
+    __syncthreads();  // previous slice fully read out of `ep`
+    const int row = warp * 32 + lane;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int n = n0 + c0 + j;
-        if (n >= P.N) break;
-        const float v = (it > 0) ? __uint_as_float(r[j]) : 0.f;
+    for (int j = 0; j < 32; ++j) ep[row * 33 + j] = (it > 0) ? __uint_as_float(r[j]) : 0.f;
+    __syncthreads();
+#pragma unroll 4
+    for (int q = 0; q < 32; ++q) {
+      const int rr = q * 4 + warp;          // each warp stores one row slice per step
+      const int m = m0 + rr, n = n0 + c0 + lane;
+      if (m < P.M && n < P.N) {
+        const float v = ep[rr * 33 + lane];
         if (g.splits > 1) {
           g.partial[P.part_off + ((long long)split * P.M + m) * P.N + n] = v;
         } else {
-          float* c = P.C + cm + ixd(P.Cn, n);
+          float* c = P.C + ixd(P.Cm, m) + ixd(P.Cn, n);
           *c = g.accumulate ? *c + v : v;
         }
       }
