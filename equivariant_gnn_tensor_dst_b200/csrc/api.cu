@@ -197,44 +197,36 @@ struct Layout {
   bool has_gbuf = false, has_part = false;
 };
 
-int chunk_nodes(size_t budget, long long per_node_floats, int arrays, long long N) {
-  if (per_node_floats <= 0 || N <= 0) return (int)std::max<long long>(N, 0);
-  long long c = (long long)(budget / (size_t(4) * per_node_floats * arrays));
+int chunk_for(size_t budget_floats, long long fixed, long long per_node, long long N) {
+  if (per_node <= 0 || N <= 0) return (int)std::max<long long>(N, 0);
+  long long avail = (long long)budget_floats - fixed;
+  long long c = avail > 0 ? avail / per_node : 1;
   c = std::max<long long>(1, std::min<long long>(c, N));
   return (int)c;
 }
 
-// floats of one split-K slice: the largest of the weight gradient, a receiver range of
-// outputs and a source range of input gradients
-long long part_floats(const tpconv_plan* P, const Layout& L) {
-  long long a = (long long)P->K * P->n_w;
-  a = std::max(a, (long long)L.recv_chunk * P->dim_out);
-  a = std::max(a, (long long)L.src_chunk * P->dim_in);
-  return a;
-}
-
+// Workspace of one pass.  The scratch budget covers the node states of a receiver (or
+// source) range and the split-K slices of the channel contractions; backward adds the
+// per-edge position-gradient staging (16 bytes per edge) on top.
 Layout make_layout(const tpconv_plan* P, long long N, long long E, uint32_t pass) {
   Layout L;
   size_t off = 0;
   const long long st = P->dev.state_per_node, xs = P->dev.xstate_per_node;
+  const size_t bf = P->budget / 4;
   if (P->mode == TPCONV_UVW) {
-    int arrays = (pass == TPCONV_PASS_DOUBLE_BACKWARD) ? 2 : 1;
-    L.recv_chunk = chunk_nodes(P->budget, st, arrays, N);
-    L.src_chunk = chunk_nodes(P->budget, xs, arrays, N);
-    size_t one = 0;
-    if (pass == TPCONV_PASS_FORWARD) {
-      one = align256(size_t(4) * L.recv_chunk * st);
-    } else {
-      one = std::max(align256(size_t(4) * L.recv_chunk * st), align256(size_t(4) * L.src_chunk * xs));
-    }
+    const int arrays = (pass == TPCONV_PASS_DOUBLE_BACKWARD) ? 2 : 1;
+    const long long fixed = (pass == TPCONV_PASS_FORWARD) ? 0 : (long long)kSplits * P->K * P->n_w;
+    L.recv_chunk = chunk_for(bf, fixed, arrays * st + (long long)kSplits * P->dim_out, N);
+    L.src_chunk = (pass == TPCONV_PASS_FORWARD) ? 0 : chunk_for(bf, fixed, arrays * xs + (long long)kSplits * P->dim_in, N);
+    const size_t one = std::max(align256(size_t(4) * L.recv_chunk * st), align256(size_t(4) * L.src_chunk * xs));
     L.state_a = off;
     off += one;
     if (arrays == 2) { L.state_b = off; off += one; }
-    if (pass != TPCONV_PASS_FORWARD) {
-      L.has_part = true;
-      L.part = off;
-      off += align256(size_t(4) * kSplits * part_floats(P, L));
-    }
+    long long pf = std::max((long long)L.recv_chunk * P->dim_out, (long long)L.src_chunk * P->dim_in);
+    if (pass != TPCONV_PASS_FORWARD) pf = std::max(pf, (long long)P->K * P->n_w);
+    L.has_part = true;
+    L.part = off;
+    off += align256(size_t(4) * kSplits * pf);
   } else {
     if (pass != TPCONV_PASS_FORWARD) {
       L.has_part = true;
@@ -676,7 +668,7 @@ tpconv_status tpconv_forward(tpconv_plan_t P, int64_t N, int64_t E, const float*
     const int cn = std::min(L.recv_chunk, n - n0);
     TPC_RUN(PC_UVW_STATE, 1, launch_uvw_state(P->dev, P->t_in, 0, x, nullptr, pos, nullptr, row_ptr, src, n0, cn, S,
                              nullptr, s));
-    TPC_RUN(PC_GEMM, 1, gemm_state_times_A(P, S, W, nullptr, nullptr, out, n0, cn, nullptr, s));
+    TPC_RUN(PC_GEMM, 2, gemm_state_times_A(P, S, W, nullptr, nullptr, out, n0, cn, fptr(ws, L.part), s));
   }
   return TPCONV_OK;
 }

@@ -7,12 +7,12 @@
 // contractions of the method.
 //
 // fp32 accuracy from TF32 tensor cores: every operand value a is split as
-// a = hi + lo with hi = tf32(a) (round to nearest) and lo = tf32(a - hi); each k-step
+// a = hi + lo with hi = a truncated to TF32 and lo = a - hi; each k-step
 // issues hi*hi + hi*lo + lo*hi into the same fp32 accumulator ("3xTF32", the
 // decomposition of Ootomo and Yokota, 2022), which keeps the relative error near
 // 2^-21 instead of TF32's 2^-11.
 //
-// Structure: one CTA of 128 threads per 128 x NT output tile (NT = 64 or 128) and
+// Structure: one CTA of 256 threads per 128 x NT output tile (NT = 64 or 128) and
 // split-K slice.  All threads stage operand tiles from global memory through the same
 // two-level affine index maps as the rest of the library (so ir_mul node rows, weight
 // columns and workspace states are read in place), split them and store them in the
@@ -32,7 +32,7 @@ namespace {
 
 constexpr int TC_M = 128;
 constexpr int TC_K = 32;           // k elements per stage (8 core-matrix columns)
-constexpr int TC_THREADS = 128;
+constexpr int TC_THREADS = 256;
 constexpr unsigned kWaitLimit = 1u << 20;
 
 __device__ __forceinline__ long long ixd(const Idx2& f, int i) {
@@ -43,11 +43,10 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ float to_tf32(float a) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(a));
-  return __uint_as_float(r);
-}
+// TF32 part of a float: keep sign, exponent and the top 10 mantissa bits.  The residual
+// a - hi is exact in fp32; the tensor core reads it as TF32 (dropping its low bits),
+// which leaves an error below 2^-21 |a|.
+__device__ __forceinline__ float tf32_hi(float a) { return __uint_as_float(__float_as_uint(a) & 0xffffe000u); }
 
 // byte offset of element (row, k) inside a [rows x 32] K-major no-swizzle tile
 __device__ __forceinline__ uint32_t tile_off(int row, int k) {
@@ -133,10 +132,10 @@ __device__ __forceinline__ void store_operand(const Frag<KW>& f, int nrows, char
 #pragma unroll
   for (int q = 0; q < KW / 4; ++q) {
     float4 h, l;
-    h.x = to_tf32(f.v[4 * q]);     l.x = to_tf32(f.v[4 * q] - h.x);
-    h.y = to_tf32(f.v[4 * q + 1]); l.y = to_tf32(f.v[4 * q + 1] - h.y);
-    h.z = to_tf32(f.v[4 * q + 2]); l.z = to_tf32(f.v[4 * q + 2] - h.z);
-    h.w = to_tf32(f.v[4 * q + 3]); l.w = to_tf32(f.v[4 * q + 3] - h.w);
+    h.x = tf32_hi(f.v[4 * q]);     l.x = f.v[4 * q] - h.x;
+    h.y = tf32_hi(f.v[4 * q + 1]); l.y = f.v[4 * q + 1] - h.y;
+    h.z = tf32_hi(f.v[4 * q + 2]); l.z = f.v[4 * q + 2] - h.z;
+    h.w = tf32_hi(f.v[4 * q + 3]); l.w = f.v[4 * q + 3] - h.w;
     const uint32_t off = tile_off(row, kbeg + 4 * q);
     *reinterpret_cast<float4*>(hi + off) = h;
     *reinterpret_cast<float4*>(lo + off) = l;
@@ -188,7 +187,8 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
   const uint32_t tmem = *tmem_slot;
 
   constexpr uint32_t IDESC = instr_desc<NT>();
-  constexpr int KWB = TC_K / (TC_THREADS / NT);   // k values per thread for the B operand
+  constexpr int KWA = TC_K / (TC_THREADS / TC_M);  // k values per thread for the A operand
+  constexpr int KWB = TC_K / (TC_THREADS / NT);    // k values per thread for the B operand
   uint32_t phase[2] = {0u, 0u};
   bool ok = true;
 
@@ -208,11 +208,11 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
     kbase_seg += g.sg[P.seg0 + seg].K;
     ++seg;
   }
-  Frag<TC_K> fa;
+  Frag<KWA> fa;
   Frag<KWB> fb;
   if (have) {
     const GemmSeg& S = g.sg[P.seg0 + seg];
-    fetch_operand<TC_K>(S.A, S.Am, S.Ak, m0, P.M, kt, khi, TC_M, S.a_vec4 != 0, fa);
+    fetch_operand<KWA>(S.A, S.Am, S.Ak, m0, P.M, kt, khi, TC_M, S.a_vec4 != 0, fa);
     fetch_operand<KWB>(S.B, S.Bn, S.Bk, n0, P.N, kt, khi, NT, false, fb);
   }
   int it = 0;
@@ -223,7 +223,7 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
       phase[st] ^= 1u;
     }
     char* sb = stage_base[st];
-    store_operand<TC_K>(fa, TC_M, sb, sb + TcSmem<NT>::A_BYTES);
+    store_operand<KWA>(fa, TC_M, sb, sb + TcSmem<NT>::A_BYTES);
     store_operand<KWB>(fb, NT, sb + 2 * TcSmem<NT>::A_BYTES, sb + 2 * TcSmem<NT>::A_BYTES + TcSmem<NT>::B_BYTES);
     // advance to the next tile and start its loads before this tile's MMAs
     kt += TC_K;
@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
     }
     if (have) {
       const GemmSeg& S = g.sg[P.seg0 + seg];
-      fetch_operand<TC_K>(S.A, S.Am, S.Ak, m0, P.M, kt, khi, TC_M, S.a_vec4 != 0, fa);
+      fetch_operand<KWA>(S.A, S.Am, S.Ak, m0, P.M, kt, khi, TC_M, S.a_vec4 != 0, fa);
       fetch_operand<KWB>(S.B, S.Bn, S.Bk, n0, P.N, kt, khi, NT, false, fb);
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -283,14 +283,29 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
   }
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 
-  // epilogue: TMEM lane (32 * warp + lane) holds output row m0 + 32 * warp + lane.
-  // Each 32-column slice goes through shared memory (row stride 33 floats, conflict
-  // free) so that a warp then stores 32 consecutive columns of one row.
+  // epilogue.  TMEM lane r holds output row m0 + r; warp w may read lane quadrant w % 4
+  // and takes the column half w / 4 of every 64-column slice.  Values pass through
+  // shared memory (row stride 65 floats, conflict free) so that each warp then stores
+  // consecutive columns of one row; row and column offsets of the output map are
+  // tabulated once.
   float* ep = reinterpret_cast<float*>(stage_base[0]);   // all MMAs are complete here
+  long long* rowoff = reinterpret_cast<long long*>(stage_base[1]);
+  long long* coloff = rowoff + TC_M;
+  __syncthreads();
+  for (int t = tid; t < TC_M; t += TC_THREADS) {
+    const int m = m0 + t;
+    rowoff[t] = m < P.M ? (g.splits > 1 ? ((long long)split * P.M + m) * P.N : ixd(P.Cm, m)) : 0;
+  }
+  for (int t = tid; t < NT; t += TC_THREADS) {
+    const int n = n0 + t;
+    coloff[t] = n < P.N ? (g.splits > 1 ? (long long)n : ixd(P.Cn, n)) : 0;
+  }
+  float* const outbase = g.splits > 1 ? g.partial + P.part_off : P.C;
+  const int quad = warp & 3, half = warp >> 2;
 #pragma unroll 1
-  for (int c0 = 0; c0 < NT; c0 += 32) {
+  for (int c0 = 0; c0 < NT; c0 += 64) {
     uint32_t r[32];
-    const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0;
+    const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(c0 + half * 32);
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
         "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
@@ -301,22 +316,25 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
           "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-    __syncthreads();  // previous slice fully read out of `ep`
-    const int row = warp * 32 + lane;
+    __syncthreads();  // previous slice read out of `ep`; offset tables written
+    const int row = quad * 32 + lane;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) ep[row * 33 + j] = (it > 0) ? __uint_as_float(r[j]) : 0.f;
+    for (int j = 0; j < 32; ++j) ep[row * 65 + half * 32 + j] = (it > 0) ? __uint_as_float(r[j]) : 0.f;
     __syncthreads();
+    const int ncols = min(64, NT - c0);
 #pragma unroll 4
-    for (int q = 0; q < 32; ++q) {
-      const int rr = q * 4 + warp;          // each warp stores one row slice per step
-      const int m = m0 + rr, n = n0 + c0 + lane;
-      if (m < P.M && n < P.N) {
-        const float v = ep[rr * 33 + lane];
-        if (g.splits > 1) {
-          g.partial[P.part_off + ((long long)split * P.M + m) * P.N + n] = v;
-        } else {
-          float* c = P.C + ixd(P.Cm, m) + ixd(P.Cn, n);
-          *c = g.accumulate ? *c + v : v;
+    for (int q = 0; q < TC_M / 8; ++q) {
+      const int rr = q * 8 + warp;                       // 8 warps store 8 rows per step
+      const int m = m0 + rr;
+      if (m >= P.M) continue;
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int cc = h2 * 32 + lane;
+        const int n = n0 + c0 + cc;
+        if (cc < ncols && n < P.N) {
+          const float v = ep[rr * 65 + cc];
+          float* c = outbase + rowoff[rr] + coloff[c0 + cc];
+          *c = (g.accumulate && g.splits == 1) ? *c + v : v;
         }
       }
     }
