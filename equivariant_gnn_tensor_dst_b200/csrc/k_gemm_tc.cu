@@ -82,19 +82,24 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   return false;
 }
 
-// Operand staging is split in two halves so that the global loads of the next k-tile
-// are in flight while the current one is stored and its MMAs are issued.  Thread t
-// owns one operand row (row = t % nrows) and a contiguous range of kw = 32 / (128 /
-// nrows) k values.
-template <int KW>
-struct Frag {
-  float v[KW];
-};
+// Asynchronous operand staging: raw fp32 tiles go straight from global to shared memory
+// with cp.async (zero-filled outside the operand) into a ring of RING stages, already in
+// the canonical core-matrix layout.  A conversion pass then splits a landed stage into
+// the hi and lo buffers read by the MMAs.  Thread t owns row t % nrows of an operand
+// tile and the contiguous k range [(t / nrows) * KW, +KW).
+__device__ __forceinline__ void cp_async4(uint32_t dst, const float* src, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(valid ? 4 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const float* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
+}
 
 template <int KW>
-__device__ __forceinline__ void fetch_operand(const float* __restrict__ base, const Idx2& mr, const Idx2& mk,
+__device__ __forceinline__ void issue_operand(const float* __restrict__ base, const Idx2& mr, const Idx2& mk,
                                               int r0, int rmax, int kt, int khi, int nrows, bool vec4,
-                                              Frag<KW>& f) {
+                                              uint32_t dst) {
   const int t = threadIdx.x;
   const int row = t % nrows;
   const int kbeg = (t / nrows) * KW;
@@ -103,42 +108,18 @@ __device__ __forceinline__ void fetch_operand(const float* __restrict__ base, co
   const long long rbase = rok ? ixd(mr, r) : 0;
   const bool lin = (kt % mk.d) + TC_K <= mk.d;
   const long long kbase = ixd(mk, kt);
-  if (vec4 && lin && rok && ((kt & 3) == 0) && kt + kbeg + KW <= khi) {
-    const float4* p4 = reinterpret_cast<const float4*>(base + rbase + kbase + kbeg);
+  if (vec4 && lin && ((kt & 3) == 0) && kt + kbeg + KW <= khi) {
 #pragma unroll
-    for (int q = 0; q < KW / 4; ++q) {
-      const float4 v = __ldg(p4 + q);
-      f.v[4 * q] = v.x; f.v[4 * q + 1] = v.y; f.v[4 * q + 2] = v.z; f.v[4 * q + 3] = v.w;
-    }
+    for (int q = 0; q < KW / 4; ++q)
+      cp_async16(dst + tile_off(row, kbeg + 4 * q), base + rbase + kbase + kbeg + 4 * q, rok);
     return;
   }
 #pragma unroll
   for (int j = 0; j < KW; ++j) {
     const int k = kt + kbeg + j;
-    float a = 0.f;
-    if (rok && k < khi) {
-      const long long ko = lin ? kbase + (long long)(kbeg + j) * mk.s2 : ixd(mk, k);
-      a = __ldg(base + rbase + ko);
-    }
-    f.v[j] = a;
-  }
-}
-
-template <int KW>
-__device__ __forceinline__ void store_operand(const Frag<KW>& f, int nrows, char* hi, char* lo) {
-  const int t = threadIdx.x;
-  const int row = t % nrows;
-  const int kbeg = (t / nrows) * KW;
-#pragma unroll
-  for (int q = 0; q < KW / 4; ++q) {
-    float4 h, l;
-    h.x = tf32_hi(f.v[4 * q]);     l.x = f.v[4 * q] - h.x;
-    h.y = tf32_hi(f.v[4 * q + 1]); l.y = f.v[4 * q + 1] - h.y;
-    h.z = tf32_hi(f.v[4 * q + 2]); l.z = f.v[4 * q + 2] - h.z;
-    h.w = tf32_hi(f.v[4 * q + 3]); l.w = f.v[4 * q + 3] - h.w;
-    const uint32_t off = tile_off(row, kbeg + 4 * q);
-    *reinterpret_cast<float4*>(hi + off) = h;
-    *reinterpret_cast<float4*>(lo + off) = l;
+    const bool ok = rok && k < khi;
+    const long long ko = !ok ? 0 : (lin ? kbase + (long long)(kbeg + j) * mk.s2 : ixd(mk, k));
+    cp_async4(dst + tile_off(row, kbeg + j), base + (ok ? rbase + ko : 0), ok);
   }
 }
 
@@ -146,17 +127,21 @@ template <int NT>
 struct TcSmem {
   static constexpr int A_BYTES = TC_M * TC_K * 4;
   static constexpr int B_BYTES = NT * TC_K * 4;
-  static constexpr int STAGE = 2 * A_BYTES + 2 * B_BYTES;
-  static constexpr int TOTAL = 2 * STAGE + 2048;  // + alignment slack, barriers, TMEM address
+  static constexpr int RAW = A_BYTES + B_BYTES;      // one raw fp32 stage: [A | B]
+  static constexpr int RING = NT <= 64 ? 4 : 3;      // raw stages in flight
+  static constexpr int SPLIT = 2 * RAW;              // one MMA buffer: hi [A | B], lo [A | B]
+  static constexpr int TOTAL = RING * RAW + 2 * SPLIT + 2048;  // + alignment, barriers, TMEM address
 };
 
 template <int NT>
 __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ GemmBatch g, int* err) {
   extern __shared__ char smem_raw[];
   char* smem = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  char* stage_base[2] = {smem, smem + TcSmem<NT>::STAGE};
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * TcSmem<NT>::STAGE);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + 2 * TcSmem<NT>::STAGE + 64);
+  using SM = TcSmem<NT>;
+  char* ring = smem;                                  // RING raw stages
+  char* split_buf[2] = {smem + SM::RING * SM::RAW, smem + SM::RING * SM::RAW + SM::SPLIT};
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::RING * SM::RAW + 2 * SM::SPLIT);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::RING * SM::RAW + 2 * SM::SPLIT + 64);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // locate (problem, m tile, n tile)
@@ -192,65 +177,78 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
   uint32_t phase[2] = {0u, 0u};
   bool ok = true;
 
-  // flat walk over the k-tiles of this split: (segment, kt) pairs
-  int seg = 0, kbase_seg = 0, kt = 0, khi = 0;
-  auto seg_range = [&](int si, int& lo, int& hi) {
-    const int K = g.sg[P.seg0 + si].K;
-    lo = max(kb - kbase_seg, 0);
-    hi = min(ke - kbase_seg, K);
+  // The k-tiles of this split, as (segment, kt) pairs, walked by a cursor.
+  struct Cursor { int seg, kbase, kt, khi; bool have; };
+  auto advance_to_valid = [&](Cursor& c) {
+    while (c.seg < P.nseg) {
+      const int K = g.sg[P.seg0 + c.seg].K;
+      const int lo = max(kb - c.kbase, 0), hi = min(ke - c.kbase, K);
+      if (c.kt < lo) c.kt = lo;
+      if (c.kt < hi) { c.khi = hi; c.have = true; return; }
+      c.kbase += K;
+      ++c.seg;
+      c.kt = 0;
+    }
+    c.have = false;
   };
-  // position on the first non-empty tile
-  bool have = false;
-  while (seg < P.nseg) {
-    int lo, hi;
-    seg_range(seg, lo, hi);
-    if (lo < hi) { kt = lo; khi = hi; have = true; break; }
-    kbase_seg += g.sg[P.seg0 + seg].K;
-    ++seg;
+  Cursor ld{0, 0, 0, 0, false};
+  advance_to_valid(ld);
+  auto issue_tile = [&](int slot) {
+    // always commit a group (possibly empty) so that group counting stays uniform
+    if (ld.have) {
+      const GemmSeg& S = g.sg[P.seg0 + ld.seg];
+      const uint32_t dst = smem_u32(ring + slot * SM::RAW);
+      issue_operand<KWA>(S.A, S.Am, S.Ak, m0, P.M, ld.kt, ld.khi, TC_M, S.a_vec4 != 0, dst);
+      issue_operand<KWB>(S.B, S.Bn, S.Bk, n0, P.N, ld.kt, ld.khi, NT, false, dst + SM::A_BYTES);
+      ld.kt += TC_K;
+      advance_to_valid(ld);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  // number of k-tiles of this split
+  int ntiles = 0;
+  {
+    Cursor c{0, 0, 0, 0, false};
+    advance_to_valid(c);
+    while (c.have) { ++ntiles; c.kt += TC_K; advance_to_valid(c); }
   }
-  Frag<KWA> fa;
-  Frag<KWB> fb;
-  if (have) {
-    const GemmSeg& S = g.sg[P.seg0 + seg];
-    fetch_operand<KWA>(S.A, S.Am, S.Ak, m0, P.M, kt, khi, TC_M, S.a_vec4 != 0, fa);
-    fetch_operand<KWB>(S.B, S.Bn, S.Bk, n0, P.N, kt, khi, NT, false, fb);
-  }
+#pragma unroll 1
+  for (int s = 0; s < SM::RING - 1; ++s) issue_tile(s);
+
   int it = 0;
-  while (have) {
+#pragma unroll 1
+  for (; it < ntiles; ++it) {
+    issue_tile((it + SM::RING - 1) % SM::RING);
+    asm volatile("cp.async.wait_group %0;" ::"n"(SM::RING - 1) : "memory");
+    __syncthreads();                                   // stage `it` landed for every thread
     const int st = it & 1;
-    if (it >= 2) {  // stage st was read by the MMAs committed two iterations ago
+    if (it >= 2) {  // split buffer st was read by the MMAs committed two iterations ago
       ok = mbar_wait(smem_u32(&bars[st]), phase[st]) && ok;
       phase[st] ^= 1u;
     }
-    char* sb = stage_base[st];
-    store_operand<KWA>(fa, TC_M, sb, sb + TcSmem<NT>::A_BYTES);
-    store_operand<KWB>(fb, NT, sb + 2 * TcSmem<NT>::A_BYTES, sb + 2 * TcSmem<NT>::A_BYTES + TcSmem<NT>::B_BYTES);
-    // advance to the next tile and start its loads before this tile's MMAs
-    kt += TC_K;
-    if (kt >= khi) {
-      have = false;
-      kbase_seg += g.sg[P.seg0 + seg].K;
-      ++seg;
-      while (seg < P.nseg) {
-        int lo, hi;
-        seg_range(seg, lo, hi);
-        if (lo < hi) { kt = lo; khi = hi; have = true; break; }
-        kbase_seg += g.sg[P.seg0 + seg].K;
-        ++seg;
+    {
+      const float4* raw = reinterpret_cast<const float4*>(ring + (it % SM::RING) * SM::RAW);
+      float4* hi = reinterpret_cast<float4*>(split_buf[st]);
+      float4* lo = reinterpret_cast<float4*>(split_buf[st] + SM::RAW);
+#pragma unroll 2
+      for (int i = tid; i < SM::RAW / 16; i += TC_THREADS) {
+        const float4 v = raw[i];
+        float4 h, l;
+        h.x = tf32_hi(v.x); l.x = v.x - h.x;
+        h.y = tf32_hi(v.y); l.y = v.y - h.y;
+        h.z = tf32_hi(v.z); l.z = v.z - h.z;
+        h.w = tf32_hi(v.w); l.w = v.w - h.w;
+        hi[i] = h;
+        lo[i] = l;
       }
-    }
-    if (have) {
-      const GemmSeg& S = g.sg[P.seg0 + seg];
-      fetch_operand<KWA>(S.A, S.Am, S.Ak, m0, P.M, kt, khi, TC_M, S.a_vec4 != 0, fa);
-      fetch_operand<KWB>(S.B, S.Bn, S.Bk, n0, P.N, kt, khi, NT, false, fb);
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     if (tid == 0) {
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t a_hi = smem_u32(sb), a_lo = a_hi + TcSmem<NT>::A_BYTES;
-      const uint32_t b_hi = a_hi + 2 * TcSmem<NT>::A_BYTES, b_lo = b_hi + TcSmem<NT>::B_BYTES;
+      const uint32_t a_hi = smem_u32(split_buf[st]), b_hi = a_hi + SM::A_BYTES;
+      const uint32_t a_lo = a_hi + SM::RAW, b_lo = a_lo + SM::A_BYTES;
 #pragma unroll
       for (int ks = 0; ks < TC_K / 8; ++ks) {
         const uint32_t koff = ks * 256;  // two 16-byte core-matrix columns per K=8 step
@@ -274,8 +272,8 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
                        smem_u32(&bars[st]))
                    : "memory");
     }
-    ++it;
   }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
   // wait for the last commit (tcgen05 operations complete in issue order)
   if (it > 0) {
     const int st = (it - 1) & 1;
@@ -288,8 +286,8 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
   // shared memory (row stride 65 floats, conflict free) so that each warp then stores
   // consecutive columns of one row; row and column offsets of the output map are
   // tabulated once.
-  float* ep = reinterpret_cast<float*>(stage_base[0]);   // all MMAs are complete here
-  long long* rowoff = reinterpret_cast<long long*>(stage_base[1]);
+  float* ep = reinterpret_cast<float*>(split_buf[0]);   // all MMAs are complete here
+  long long* rowoff = reinterpret_cast<long long*>(split_buf[1]);
   long long* coloff = rowoff + TC_M;
   __syncthreads();
   for (int t = tid; t < TC_M; t += TC_THREADS) {
