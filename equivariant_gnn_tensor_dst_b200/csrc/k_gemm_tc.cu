@@ -96,30 +96,58 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const float* src, bool 
                : "memory");
 }
 
+// Per-thread position of one operand inside the current segment.  The row offset is
+// computed once per segment; the k offset is tracked as (kq, kr) = (k / d, k % d) of the
+// operand's k map and advanced by additions, so that no division is executed per tile.
+struct OpCursor {
+  const float* row;     // base + row offset (nullptr: row outside the operand)
+  long long s1, s2;     // k map strides
+  int d;                // k map block
+  int kq, kr;           // (k / d, k % d) of the current tile start
+};
+
+__device__ __forceinline__ void op_enter(OpCursor& c, const float* base, const Idx2& mr, const Idx2& mk, int r,
+                                         int rmax, int kt) {
+  c.row = r < rmax ? base + ixd(mr, r) : nullptr;
+  c.s1 = mk.s1;
+  c.s2 = mk.s2;
+  c.d = mk.d;
+  c.kq = kt / mk.d;
+  c.kr = kt % mk.d;
+}
+
+__device__ __forceinline__ void op_step(OpCursor& c, int dk) {
+  c.kr += dk;
+  while (c.kr >= c.d) { c.kr -= c.d; ++c.kq; }
+}
+
+// Issue the cp.async copies of this thread's share of one operand tile.
 template <int KW>
-__device__ __forceinline__ void issue_operand(const float* __restrict__ base, const Idx2& mr, const Idx2& mk,
-                                              int r0, int rmax, int kt, int khi, int nrows, bool vec4,
-                                              uint32_t dst) {
-  const int t = threadIdx.x;
-  const int row = t % nrows;
-  const int kbeg = (t / nrows) * KW;
-  const int r = r0 + row;
-  const bool rok = r < rmax;
-  const long long rbase = rok ? ixd(mr, r) : 0;
-  const bool lin = (kt % mk.d) + TC_K <= mk.d;
-  const long long kbase = ixd(mk, kt);
+__device__ __forceinline__ void issue_operand(const OpCursor& c, const float* safe, int kt, int khi, int kbeg,
+                                              int row, bool vec4, uint32_t dst) {
+  const bool lin = c.kr + TC_K <= c.d;
+  const float* p = c.row ? c.row + (long long)c.kq * c.s1 + (long long)(c.kr + kbeg) * c.s2 : safe;
   if (vec4 && lin && ((kt & 3) == 0) && kt + kbeg + KW <= khi) {
 #pragma unroll
-    for (int q = 0; q < KW / 4; ++q)
-      cp_async16(dst + tile_off(row, kbeg + 4 * q), base + rbase + kbase + kbeg + 4 * q, rok);
+    for (int q = 0; q < KW / 4; ++q) cp_async16(dst + tile_off(row, kbeg + 4 * q), c.row ? p + 4 * q : safe, c.row != nullptr);
     return;
   }
+  if (lin) {
 #pragma unroll
+    for (int j = 0; j < KW; ++j) {
+      const bool ok = c.row && kt + kbeg + j < khi;
+      cp_async4(dst + tile_off(row, kbeg + j), ok ? p + (long long)j * c.s2 : safe, ok);
+    }
+    return;
+  }
+  // the tile crosses a block of the k map: step element by element
+  int q = c.kq, r = c.kr + kbeg;
+  while (r >= c.d) { r -= c.d; ++q; }
+#pragma unroll 1
   for (int j = 0; j < KW; ++j) {
-    const int k = kt + kbeg + j;
-    const bool ok = rok && k < khi;
-    const long long ko = !ok ? 0 : (lin ? kbase + (long long)(kbeg + j) * mk.s2 : ixd(mk, k));
-    cp_async4(dst + tile_off(row, kbeg + j), base + (ok ? rbase + ko : 0), ok);
+    const bool ok = c.row && kt + kbeg + j < khi;
+    cp_async4(dst + tile_off(row, kbeg + j), ok ? c.row + (long long)q * c.s1 + (long long)r * c.s2 : safe, ok);
+    if (++r == c.d) { r = 0; ++q; }
   }
 }
 
@@ -191,17 +219,31 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
     }
     c.have = false;
   };
+  const int rowA = tid % TC_M, kbegA = (tid / TC_M) * KWA;
+  const int rowB = tid % NT, kbegB = (tid / NT) * KWB;
   Cursor ld{0, 0, 0, 0, false};
+  OpCursor ca{}, cb{};
+  int cur_seg = -1;
   advance_to_valid(ld);
   auto issue_tile = [&](int slot) {
     // always commit a group (possibly empty) so that group counting stays uniform
     if (ld.have) {
       const GemmSeg& S = g.sg[P.seg0 + ld.seg];
+      if (ld.seg != cur_seg) {  // entering a segment: row offsets and k positions
+        op_enter(ca, S.A, S.Am, S.Ak, m0 + rowA, P.M, ld.kt);
+        op_enter(cb, S.B, S.Bn, S.Bk, n0 + rowB, P.N, ld.kt);
+        cur_seg = ld.seg;
+      }
       const uint32_t dst = smem_u32(ring + slot * SM::RAW);
-      issue_operand<KWA>(S.A, S.Am, S.Ak, m0, P.M, ld.kt, ld.khi, TC_M, S.a_vec4 != 0, dst);
-      issue_operand<KWB>(S.B, S.Bn, S.Bk, n0, P.N, ld.kt, ld.khi, NT, false, dst + SM::A_BYTES);
+      issue_operand<KWA>(ca, S.A, ld.kt, ld.khi, kbegA, rowA, S.a_vec4 != 0, dst);
+      issue_operand<KWB>(cb, S.B, ld.kt, ld.khi, kbegB, rowB, false, dst + SM::A_BYTES);
+      const int seg_before = ld.seg;
       ld.kt += TC_K;
       advance_to_valid(ld);
+      if (ld.have && ld.seg == seg_before) {
+        op_step(ca, TC_K);
+        op_step(cb, TC_K);
+      }
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
