@@ -17,7 +17,7 @@
 // two-level affine index maps as the rest of the library (so ir_mul node rows, weight
 // columns and workspace states are read in place), split them and store them in the
 // canonical K-major, no-swizzle core-matrix layout (8 rows x 16 bytes per core
-// matrix).  Two stages: while thread 0's MMAs of stage s run asynchronously, the CTA
+// matrix, row groups of a k column contiguous).  Two stages: while thread 0's MMAs of stage s run asynchronously, the CTA
 // fills stage s+1; a tcgen05.commit per stage arrives on that stage's mbarrier.  The
 // epilogue reads the TMEM accumulator with tcgen05.ld (one TMEM lane = one output row)
 // and writes C (or the split-K partial) through the output map.  Every mbarrier wait is
@@ -48,15 +48,20 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 // which leaves an error below 2^-21 |a|.
 __device__ __forceinline__ float tf32_hi(float a) { return __uint_as_float(__float_as_uint(a) & 0xffffe000u); }
 
-// byte offset of element (row, k) inside a [rows x 32] K-major no-swizzle tile
+// Byte offset of element (row, k) inside a [ROWS x 32] K-major no-swizzle tile.  The 8-row
+// core matrices of one 4-wide k column are contiguous (SBO = 128 B), so the tensor core
+// reads each k column of the tile as one contiguous block; k columns are ROWS * 16 B
+// apart (LBO).
+template <int ROWS>
 __device__ __forceinline__ uint32_t tile_off(int row, int k) {
-  return (uint32_t)((row >> 3) * 1024 + (k >> 2) * 128 + (row & 7) * 16 + (k & 3) * 4);
+  return (uint32_t)((k >> 2) * (ROWS * 16) + (row >> 3) * 128 + (row & 7) * 16 + (k & 3) * 4);
 }
 
+template <int ROWS>
 __device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
-  // start address, LBO = 128 B (next k core matrix), SBO = 1024 B (next 8-row group),
-  // descriptor version 1, no swizzle
-  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)(128 >> 4) << 16) | ((uint64_t)(1024 >> 4) << 32) |
+  // start address, LBO = ROWS * 16 B (next k core matrix), SBO = 128 B (next 8-row
+  // group), descriptor version 1, no swizzle
+  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((ROWS * 16) >> 4) << 16) | ((uint64_t)(128 >> 4) << 32) |
          (1ull << 46);
 }
 
@@ -122,21 +127,21 @@ __device__ __forceinline__ void op_step(OpCursor& c, int dk) {
 }
 
 // Issue the cp.async copies of this thread's share of one operand tile.
-template <int KW>
+template <int KW, int ROWS>
 __device__ __forceinline__ void issue_operand(const OpCursor& c, const float* safe, int kt, int khi, int kbeg,
                                               int row, bool vec4, uint32_t dst) {
   const bool lin = c.kr + TC_K <= c.d;
   const float* p = c.row ? c.row + (long long)c.kq * c.s1 + (long long)(c.kr + kbeg) * c.s2 : safe;
   if (vec4 && lin && ((kt & 3) == 0) && kt + kbeg + KW <= khi) {
 #pragma unroll
-    for (int q = 0; q < KW / 4; ++q) cp_async16(dst + tile_off(row, kbeg + 4 * q), c.row ? p + 4 * q : safe, c.row != nullptr);
+    for (int q = 0; q < KW / 4; ++q) cp_async16(dst + tile_off<ROWS>(row, kbeg + 4 * q), c.row ? p + 4 * q : safe, c.row != nullptr);
     return;
   }
   if (lin) {
 #pragma unroll
     for (int j = 0; j < KW; ++j) {
       const bool ok = c.row && kt + kbeg + j < khi;
-      cp_async4(dst + tile_off(row, kbeg + j), ok ? p + (long long)j * c.s2 : safe, ok);
+      cp_async4(dst + tile_off<ROWS>(row, kbeg + j), ok ? p + (long long)j * c.s2 : safe, ok);
     }
     return;
   }
@@ -146,7 +151,7 @@ __device__ __forceinline__ void issue_operand(const OpCursor& c, const float* sa
 #pragma unroll 1
   for (int j = 0; j < KW; ++j) {
     const bool ok = c.row && kt + kbeg + j < khi;
-    cp_async4(dst + tile_off(row, kbeg + j), ok ? c.row + (long long)q * c.s1 + (long long)r * c.s2 : safe, ok);
+    cp_async4(dst + tile_off<ROWS>(row, kbeg + j), ok ? c.row + (long long)q * c.s1 + (long long)r * c.s2 : safe, ok);
     if (++r == c.d) { r = 0; ++q; }
   }
 }
@@ -235,8 +240,8 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
         cur_seg = ld.seg;
       }
       const uint32_t dst = smem_u32(ring + slot * SM::RAW);
-      issue_operand<KWA>(ca, S.A, ld.kt, ld.khi, kbegA, rowA, S.a_vec4 != 0, dst);
-      issue_operand<KWB>(cb, S.B, ld.kt, ld.khi, kbegB, rowB, false, dst + SM::A_BYTES);
+      issue_operand<KWA, TC_M>(ca, S.A, ld.kt, ld.khi, kbegA, rowA, S.a_vec4 != 0, dst);
+      issue_operand<KWB, NT>(cb, S.B, ld.kt, ld.khi, kbegB, rowB, false, dst + SM::A_BYTES);
       const int seg_before = ld.seg;
       ld.kt += TC_K;
       advance_to_valid(ld);
@@ -293,9 +298,10 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
       const uint32_t a_lo = a_hi + SM::RAW, b_lo = a_lo + SM::A_BYTES;
 #pragma unroll
       for (int ks = 0; ks < TC_K / 8; ++ks) {
-        const uint32_t koff = ks * 256;  // two 16-byte core-matrix columns per K=8 step
-        const uint64_t dah = smem_desc(a_hi + koff), dal = smem_desc(a_lo + koff);
-        const uint64_t dbh = smem_desc(b_hi + koff), dbl = smem_desc(b_lo + koff);
+        // one K=8 step spans two 4-wide k columns
+        const uint32_t ka = ks * 2 * (TC_M * 16), kbo = ks * 2 * (NT * 16);
+        const uint64_t dah = smem_desc<TC_M>(a_hi + ka), dal = smem_desc<TC_M>(a_lo + ka);
+        const uint64_t dbh = smem_desc<NT>(b_hi + kbo), dbl = smem_desc<NT>(b_lo + kbo);
         const uint32_t acc0 = (it > 0 || ks > 0) ? 1u : 0u;
         asm volatile(
             "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
