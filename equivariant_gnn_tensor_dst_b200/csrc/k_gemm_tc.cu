@@ -10,15 +10,18 @@
 // a = hi + lo with hi = a truncated to TF32 and lo = a - hi; each k-step
 // issues hi*hi + hi*lo + lo*hi into the same fp32 accumulator ("3xTF32", the
 // decomposition of Ootomo and Yokota, 2022), which keeps the relative error near
-// 2^-21 instead of TF32's 2^-11.
+// 2^-21 instead of TF32's 2^-11.  The TF32 MMA reads only the top 19 bits of each
+// 32-bit operand, so the raw fp32 tile itself serves as "hi"; only "lo" is computed.
 //
 // Structure: one CTA of 256 threads per 128 x NT output tile (NT = 64 or 128) and
-// split-K slice.  All threads stage operand tiles from global memory through the same
-// two-level affine index maps as the rest of the library (so ir_mul node rows, weight
-// columns and workspace states are read in place), split them and store them in the
-// canonical K-major, no-swizzle core-matrix layout (8 rows x 16 bytes per core
-// matrix, row groups of a k column contiguous).  Two stages: while thread 0's MMAs of stage s run asynchronously, the CTA
-// fills stage s+1; a tcgen05.commit per stage arrives on that stage's mbarrier.  The
+// split-K slice.  Operand tiles are copied from global memory with cp.async through
+// the same two-level affine index maps as the rest of the library (so ir_mul node
+// rows, weight columns and workspace states are read in place) straight into the
+// canonical K-major, no-swizzle core-matrix layout (8 rows x 16 bytes per core matrix,
+// row groups of a k column contiguous).  Two raw stages: the copies of tile t+1 are in
+// flight while tile t is split and multiplied; every thread splits exactly the
+// elements it copied, so one barrier per tile suffices.  A tcgen05.commit per tile
+// arrives on an mbarrier that frees the raw stage and the lo buffer.  The
 // epilogue reads the TMEM accumulator with tcgen05.ld (one TMEM lane = one output row)
 // and writes C (or the split-K partial) through the output map.  Every mbarrier wait is
 // bounded; a wait that gives up sets *err and the kernel still releases its TMEM.
@@ -160,10 +163,9 @@ template <int NT>
 struct TcSmem {
   static constexpr int A_BYTES = TC_M * TC_K * 4;
   static constexpr int B_BYTES = NT * TC_K * 4;
-  static constexpr int RAW = A_BYTES + B_BYTES;      // one raw fp32 stage: [A | B]
-  static constexpr int RING = NT <= 64 ? 4 : 3;      // raw stages in flight
-  static constexpr int SPLIT = 2 * RAW;              // one MMA buffer: hi [A | B], lo [A | B]
-  static constexpr int TOTAL = RING * RAW + 2 * SPLIT + 2048;  // + alignment, barriers, TMEM address
+  static constexpr int RAW = A_BYTES + B_BYTES;      // one raw fp32 stage [A | B]; also the "hi" operand
+  static constexpr int RING = 2;                     // raw stages
+  static constexpr int TOTAL = RING * RAW + RAW + 2048;  // + lo buffer, alignment, barriers, TMEM address
 };
 
 template <int NT>
@@ -171,10 +173,10 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
   extern __shared__ char smem_raw[];
   char* smem = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   using SM = TcSmem<NT>;
-  char* ring = smem;                                  // RING raw stages
-  char* split_buf[2] = {smem + SM::RING * SM::RAW, smem + SM::RING * SM::RAW + SM::SPLIT};
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::RING * SM::RAW + 2 * SM::SPLIT);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::RING * SM::RAW + 2 * SM::SPLIT + 64);
+  char* ring = smem;                                  // RING raw stages (the "hi" operands)
+  char* lo_buf = smem + SM::RING * SM::RAW;           // "lo" operand of the current tile
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::RING * SM::RAW + SM::RAW);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::RING * SM::RAW + SM::RAW + 64);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // locate (problem, m tile, n tile)
@@ -191,7 +193,6 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
 
   if (tid == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[0])));
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[1])));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
@@ -207,7 +208,6 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
   constexpr uint32_t IDESC = instr_desc<NT>();
   constexpr int KWA = TC_K / (TC_THREADS / TC_M);  // k values per thread for the A operand
   constexpr int KWB = TC_K / (TC_THREADS / NT);    // k values per thread for the B operand
-  uint32_t phase[2] = {0u, 0u};
   bool ok = true;
 
   // The k-tiles of this split, as (segment, kt) pairs, walked by a cursor.
@@ -259,34 +259,36 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
     advance_to_valid(c);
     while (c.have) { ++ntiles; c.kt += TC_K; advance_to_valid(c); }
   }
-#pragma unroll 1
-  for (int s = 0; s < SM::RING - 1; ++s) issue_tile(s);
-
+  issue_tile(0);
+  uint32_t phase = 0u;
   int it = 0;
 #pragma unroll 1
   for (; it < ntiles; ++it) {
-    issue_tile((it + SM::RING - 1) % SM::RING);
-    asm volatile("cp.async.wait_group %0;" ::"n"(SM::RING - 1) : "memory");
-    __syncthreads();                                   // stage `it` landed for every thread
-    const int st = it & 1;
-    if (it >= 2) {  // split buffer st was read by the MMAs committed two iterations ago
-      ok = mbar_wait(smem_u32(&bars[st]), phase[st]) && ok;
-      phase[st] ^= 1u;
+    // MMA(it-1) read raw stage (it+1) % 2 and the lo buffer: wait before reusing them
+    if (it >= 1) {
+      ok = mbar_wait(smem_u32(&bars[0]), phase) && ok;
+      phase ^= 1u;
     }
+    issue_tile((it + 1) % SM::RING);
+    asm volatile("cp.async.wait_group 1;" ::: "memory");   // this thread's copies of tile `it`
     {
-      const float4* raw = reinterpret_cast<const float4*>(ring + (it % SM::RING) * SM::RAW);
-      float4* hi = reinterpret_cast<float4*>(split_buf[st]);
-      float4* lo = reinterpret_cast<float4*>(split_buf[st] + SM::RAW);
-#pragma unroll 2
-      for (int i = tid; i < SM::RAW / 16; i += TC_THREADS) {
-        const float4 v = raw[i];
-        float4 h, l;
-        h.x = tf32_hi(v.x); l.x = v.x - h.x;
-        h.y = tf32_hi(v.y); l.y = v.y - h.y;
-        h.z = tf32_hi(v.z); l.z = v.z - h.z;
-        h.w = tf32_hi(v.w); l.w = v.w - h.w;
-        hi[i] = h;
-        lo[i] = l;
+      // split the elements this thread copied: lo = raw - tf32(raw)
+      const char* raw = ring + (it % SM::RING) * SM::RAW;
+#pragma unroll
+      for (int q = 0; q < KWA / 4; ++q) {
+        const uint32_t off = tile_off<TC_M>(rowA, kbegA + 4 * q);
+        const float4 v = *reinterpret_cast<const float4*>(raw + off);
+        float4 l;
+        l.x = v.x - tf32_hi(v.x); l.y = v.y - tf32_hi(v.y); l.z = v.z - tf32_hi(v.z); l.w = v.w - tf32_hi(v.w);
+        *reinterpret_cast<float4*>(lo_buf + off) = l;
+      }
+#pragma unroll
+      for (int q = 0; q < KWB / 4; ++q) {
+        const uint32_t off = SM::A_BYTES + tile_off<NT>(rowB, kbegB + 4 * q);
+        const float4 v = *reinterpret_cast<const float4*>(raw + off);
+        float4 l;
+        l.x = v.x - tf32_hi(v.x); l.y = v.y - tf32_hi(v.y); l.z = v.z - tf32_hi(v.z); l.w = v.w - tf32_hi(v.w);
+        *reinterpret_cast<float4*>(lo_buf + off) = l;
       }
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -294,8 +296,8 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
     __syncthreads();
     if (tid == 0) {
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t a_hi = smem_u32(split_buf[st]), b_hi = a_hi + SM::A_BYTES;
-      const uint32_t a_lo = a_hi + SM::RAW, b_lo = a_lo + SM::A_BYTES;
+      const uint32_t a_hi = smem_u32(ring + (it % SM::RING) * SM::RAW), b_hi = a_hi + SM::A_BYTES;
+      const uint32_t a_lo = smem_u32(lo_buf), b_lo = a_lo + SM::A_BYTES;
 #pragma unroll
       for (int ks = 0; ks < TC_K / 8; ++ks) {
         // one K=8 step spans two 4-wide k columns
@@ -317,16 +319,13 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
             "l"(dal), "l"(dbh), "r"(IDESC), "r"(1u));
       }
       asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                       smem_u32(&bars[st]))
+                       smem_u32(&bars[0]))
                    : "memory");
     }
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");
   // wait for the last commit (tcgen05 operations complete in issue order)
-  if (it > 0) {
-    const int st = (it - 1) & 1;
-    ok = mbar_wait(smem_u32(&bars[st]), phase[st]) && ok;
-  }
+  if (it > 0) ok = mbar_wait(smem_u32(&bars[0]), phase) && ok;
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 
   // epilogue.  TMEM lane r holds output row m0 + r; warp w may read lane quadrant w % 4
@@ -334,8 +333,8 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
   // shared memory (row stride 65 floats, conflict free) so that each warp then stores
   // consecutive columns of one row; row and column offsets of the output map are
   // tabulated once.
-  float* ep = reinterpret_cast<float*>(split_buf[0]);   // all MMAs are complete here
-  long long* rowoff = reinterpret_cast<long long*>(split_buf[1]);
+  float* ep = reinterpret_cast<float*>(ring);            // all MMAs are complete here
+  long long* rowoff = reinterpret_cast<long long*>(lo_buf);
   long long* coloff = rowoff + TC_M;
   __syncthreads();
   for (int t = tid; t < TC_M; t += TC_THREADS) {
