@@ -48,6 +48,7 @@ SIGNATURES = {
     "tpconv_profile_end": (ctypes.c_int, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_c_i64), ctypes.c_int32]),
     "tpconv_profile_category_name": (ctypes.c_char_p, [ctypes.c_int32]),
     "tpconv_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int32)]),
+    "tpconv_forward_no_alloc": (ctypes.c_int, [_c_p, _c_i64, _c_i64] + [_c_p] * 6 + [_c_p]),
 }
 PROF_CATEGORIES = 12
 

@@ -870,3 +870,82 @@ const char* tpconv_profile_category_name(int32_t c) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// forward with library-owned static scratch (no allocation anywhere)
+// ---------------------------------------------------------------------------
+
+static __device__ __align__(256) unsigned char g_static_scratch[TPCONV_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 256;
+std::mutex g_static_mu;
+void* g_static_addr[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device, looked up once per device.
+tpconv_status static_scratch_address(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return TPCONV_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return TPCONV_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> g(g_static_mu);
+  if (!g_static_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return TPCONV_ERR_CUDA;
+    g_static_addr[dev] = p;
+  }
+  *out = g_static_addr[dev];
+  return TPCONV_OK;
+}
+
+// Forward layout (uvw) sized for a fixed scratch: receiver ranges of node state plus
+// the split-K slices of the channel contraction.
+Layout forward_layout_for(const tpconv_plan* P, long long N, size_t bytes) {
+  Layout L;
+  const long long st = P->dev.state_per_node;
+  const long long per_node = st + (long long)kSplits * P->dim_out;
+  const long long fit = (long long)(bytes / 4) / per_node;
+  L.recv_chunk = (int)std::max<long long>(0, std::min<long long>(fit, N));
+  L.state_a = 0;
+  const size_t one = align256(size_t(4) * L.recv_chunk * st);
+  L.has_part = true;
+  L.part = one;
+  L.total = one + align256(size_t(4) * kSplits * (long long)L.recv_chunk * P->dim_out);
+  return L;
+}
+
+}  // namespace
+
+extern "C" tpconv_status tpconv_forward_no_alloc(tpconv_plan_t P, int64_t N, int64_t E, const float* x,
+                                                 const float* pos, const int32_t* row_ptr,
+                                                 const int32_t* src, const float* W, float* out,
+                                                 struct CUstream_st* stream) {
+  tpconv_status st = common_checks(P, N, E);
+  if (st != TPCONV_OK) return st;
+  if (N == 0) return TPCONV_OK;
+  st = check_ptrs({x, pos, row_ptr, W, out}, {src});
+  if (st != TPCONV_OK) return st;
+  if (E > 0 && !src) return TPCONV_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int n = (int)N;
+  if (P->mode == TPCONV_UVU) {  // channelwise forward keeps no scratch
+    TPC_RUN(PC_UVU_FWD, 1, launch_uvu_fwd(P->dev, P->bp_out, P->t_bo, 0, x, nullptr, pos, nullptr, row_ptr, src,
+                                          W, nullptr, n, out, s));
+    return TPCONV_OK;
+  }
+  const Layout L = forward_layout_for(P, N, TPCONV_STATIC_SCRATCH_BYTES);
+  if (L.recv_chunk < 1 || L.total > TPCONV_STATIC_SCRATCH_BYTES) return TPCONV_ERR_WORKSPACE_TOO_SMALL;
+  void* ws = nullptr;
+  st = static_scratch_address(&ws);
+  if (st != TPCONV_OK) return st;
+  // every element of the state and of the split-K slices is written before it is read
+  if (!every_block_reached(P, true)) TPC_TRY(cudaMemsetAsync(out, 0, sizeof(float) * (size_t)N * P->dim_out, s));
+  float* S = fptr(ws, L.state_a);
+  for (int n0 = 0; n0 < n; n0 += L.recv_chunk) {
+    const int cn = std::min(L.recv_chunk, n - n0);
+    TPC_RUN(PC_UVW_STATE, 1, launch_uvw_state(P->dev, P->t_in, 0, x, nullptr, pos, nullptr, row_ptr, src, n0, cn, S,
+                                              nullptr, s));
+    TPC_RUN(PC_GEMM, 2, gemm_state_times_A(P, S, W, nullptr, nullptr, out, n0, cn, fptr(ws, L.part), s));
+  }
+  return TPCONV_OK;
+}

@@ -186,6 +186,30 @@ tpconv_status tpconv_double_backward(tpconv_plan_t plan, int64_t N, int64_t E, c
                                      float* grad_W, float* grad_grad_out, float* grad_pos,
                                      void* ws, size_t ws_bytes, struct CUstream_st* stream);
 
+/* Forward without any allocation by the caller or the library, for callers that
+ * cannot obtain device memory themselves: for example a plug-in whose host application
+ * owns every device allocation, or code that must not call cudaMalloc because that
+ * call can synchronise the device in the middle of latency-critical work.
+ *
+ * Same inputs, outputs and result as tpconv_forward (eq. 11 with eq. 12, evaluated as
+ * eqs. 32-35), but the scratch lives in a fixed array of TPCONV_STATIC_SCRATCH_BYTES
+ * compiled into the library, which every GPU that loads the library keeps until the
+ * process exits.  The pages have no counterpart to this entry point.
+ *  - The first call on a device looks up that array's device address (once per device,
+ *    with the device current); make that first call before any stream capture.
+ *  - Plans whose per-receiver state does not fit the array even one receiver at a time
+ *    are rejected with TPCONV_ERR_WORKSPACE_TOO_SMALL; larger graphs are processed in
+ *    receiver ranges that fit.
+ *  - All calls share the one array and every call overwrites what it reads, so nothing
+ *    needs clearing between calls; calls whose executions overlap on the GPU (several
+ *    streams, or several host threads) race on the array and must be serialised by the
+ *    caller.                                                                            */
+#define TPCONV_STATIC_SCRATCH_BYTES (32u << 20)
+tpconv_status tpconv_forward_no_alloc(tpconv_plan_t plan, int64_t N, int64_t E, const float* x,
+                                      const float* pos, const int32_t* row_ptr,
+                                      const int32_t* src, const float* W, float* out,
+                                      struct CUstream_st* stream);
+
 /* Profiling (off by default; host-side bookkeeping only).  While enabled, every kernel
  * the library launches is bracketed by a pair of CUDA events on its stream and
  * attributed to a category (tpconv_profile_category_name).  tpconv_profile_begin
