@@ -166,6 +166,7 @@ def run_native(args):
     gp = torch.empty(N, 3, device=dev)
     gw = torch.empty(plan.num_basis, plan.weight_cols, device=dev)
     ws_bytes = plan.workspace_bytes(N, E, binding.PASS_FORWARD | binding.PASS_BACKWARD)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     torch.cuda.synchronize()
     mem0 = torch.cuda.memory_allocated(dev)
     torch.cuda.reset_peak_memory_stats(dev)
@@ -177,7 +178,6 @@ def run_native(args):
         binding.tpconv_backward(plan, x, pos, row_ptr, src, t_ptr, t_eid, t_dst, W, gout, ws=ws,
                                 outputs=(gx, gp, gw), stream=stream)
 
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     for _ in range(args.warmup):
         flush.zero_()
         step()
@@ -281,6 +281,8 @@ def run_native(args):
                "includes": "H2D of x, pos, CSR, W, grad_out; source-view build; forward; backward; "
                            "D2H of out, grad_x, grad_pos, grad_W"}
 
+    extras = run_extras(args, dev, flush) if (args.extras and rank == 0) else None
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.cpu_seconds)
@@ -296,10 +298,105 @@ def run_native(args):
                 "step_algorithmic_tflop": round(total_algo / 1e12, 4),
                 "step_tflops_achieved": round(total_algo / (ms_step / 1e3) / 1e12, 3),
                 "breakdown": breakdown}
+        if extras is not None:
+            line["extras"] = extras
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# further workloads (opt-in): every pass of the method on its own workload
+# ---------------------------------------------------------------------------
+
+def _timed(fn, flush, steps, warmup):
+    import torch
+    for _ in range(warmup):
+        flush.zero_()
+        fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in ev:
+        flush.zero_()
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in ev) / steps
+
+
+def run_extras(args, dev, flush):
+    """Per-pass edges/s on every workload of the method (forward, backward, double
+    backward; uvw and uvu; fixed and power-law degrees)."""
+    import torch
+
+    from equivariant_gnn_tensor_dst_b200 import binding
+    out = {}
+    steps, warm = max(5, min(args.steps, 20)), 3
+    for cfg in args.extras_cfgs:
+        c = workloads.CONFIGS[cfg]
+        t0 = time.time()
+        plan = binding.Plan(c.irreps_in, c.sh_lmax, c.irreps_out, c.mode, c.radial, c.num_basis, c.r_cut,
+                            c.r_min, c.r_max)
+        g, rng = workloads.make_graph(c)
+        N, E = g.n_nodes, g.n_edges
+        tt = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)  # noqa: E731
+        x = tt(workloads.normal(rng, (N, plan.dim_in)))
+        W = tt(workloads.weights(rng, c.num_basis, plan.fan_in_per_column()))
+        go = tt(workloads.normal(rng, (N, plan.dim_out)))
+        pos, rp, src = tt(g.pos), tt(g.row_ptr), tt(g.src)
+        views = binding.tpconv_csr_transpose(rp, src, N)
+        ws = binding.workspace(plan.workspace_bytes(N, E), dev)
+        o = torch.empty(N, plan.dim_out, device=dev)
+        gx = torch.empty(N, plan.dim_in, device=dev)
+        gp = torch.empty(N, 3, device=dev)
+        gw = torch.empty(plan.num_basis, plan.weight_cols, device=dev)
+        fwd = lambda: binding.tpconv_forward(plan, x, pos, rp, src, W, out=o, ws=ws)  # noqa: E731
+        bwd = lambda: binding.tpconv_backward(plan, x, pos, rp, src, *views, W, go, ws=ws,  # noqa: E731
+                                              outputs=(gx, gp, gw))
+        rec = {"workload": c.name, "nodes": N, "edges": E, "mode": c.mode,
+               "graph_seconds": round(time.time() - t0, 1)}
+        ms_f = _timed(fwd, flush, steps, warm)
+        ms_b = _timed(bwd, flush, steps, warm)
+        rec.update({"forward_ms": round(ms_f, 4), "forward_edges_per_s": round(E / ms_f * 1e3, 1),
+                    "backward_ms": round(ms_b, 4), "backward_edges_per_s": round(E / ms_b * 1e3, 1)})
+        if "dbl" in c.passes:
+            # force training: energy = sum of scalar outputs, F = -dE/dpos, loss |F - F_ref|^2,
+            # then d loss / d(W, x) by the double backward
+            mask = np.zeros(plan.dim_out, np.float32)
+            off = 0
+            for tok in c.irreps_out.split("+"):
+                mul, ir = tok.split("x")
+                l = int(ir[:-1])
+                if l == 0 and ir[-1] == "e":
+                    mask[off:off + int(mul)] = 1.0
+                off += int(mul) * (2 * l + 1)
+            mbar = tt(np.tile(mask, (N, 1)))
+            F_ref = tt(workloads.normal(rng, (N, 3)))
+            dx = torch.empty(N, plan.dim_in, device=dev)
+            dw = torch.empty(plan.num_basis, plan.weight_cols, device=dev)
+            gg = torch.empty(N, 3, device=dev)
+
+            def force_step():
+                binding.tpconv_forward(plan, x, pos, rp, src, W, out=o, ws=ws)
+                binding.tpconv_backward(plan, x, pos, rp, src, *views, W, mbar, ws=ws, outputs=(None, gp, None))
+                torch.mul(torch.add(gp, F_ref), 2.0, out=gg)   # d loss / d pos_bar = 2 (pos_bar + F_ref)
+                binding.tpconv_double_backward(plan, x, pos, rp, src, *views, W, mbar, gg_pos=gg, ws=ws,
+                                               outputs=(dx, dw, None))
+
+            def dbl_only():
+                binding.tpconv_double_backward(plan, x, pos, rp, src, *views, W, mbar, gg_pos=gg, ws=ws,
+                                               outputs=(dx, dw, None))
+            ms_s = _timed(force_step, flush, steps, warm)
+            ms_d = _timed(dbl_only, flush, steps, warm)
+            rec.update({"double_backward_ms": round(ms_d, 4),
+                        "double_backward_edges_per_s": round(E / ms_d * 1e3, 1),
+                        "force_step_ms": round(ms_s, 4), "force_step_edges_per_s": round(E / ms_s * 1e3, 1)})
+        out[str(cfg)] = rec
+        del ws
+        torch.cuda.empty_cache()
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -380,6 +477,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--extras", action="store_true",
+                    help="also time every pass on the other workloads (adds ~1-2 minutes)")
+    ap.add_argument("--extras-cfgs", type=int, nargs="*", default=[2, 3, 5, 4])
     ap.add_argument("--nodes", type=int, default=None,
                     help="resize the workload (same density and degree); for profiling small cases")
     args = ap.parse_args()
