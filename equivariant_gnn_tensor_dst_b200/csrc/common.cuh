@@ -185,6 +185,62 @@ __device__ __forceinline__ void cg_couple(const float* xv, const float* Y, float
   for (int n = 0; n < T::nnz; ++n) C[T::mo(n)] = fmaf(T::val(n) * Y[T::my(n)], xv[T::mi(n)], C[T::mo(n)]);
 }
 
+// Per-edge products cy[n] = c_n * Y[my_n] of one path (n < nnz, padded with zeros to a
+// multiple of 4); every lane then needs only these and its own x values.
+constexpr int CY_MAX = 44;   // max nnz over l <= 3 triples (42), padded to a multiple of 4
+
+template <int LI, int LS, int LO>
+struct CgInfo {
+  static constexpr int nnz = tpc_tab::CG<LI, LS, LO>::nnz;
+  static constexpr int n4 = (nnz + 3) / 4;
+};
+
+template <int LI, int LS, int LO>
+__device__ __forceinline__ void cg_products(const float* Y, float* cy) {
+  using T = tpc_tab::CG<LI, LS, LO>;
+  constexpr int n4 = CgInfo<LI, LS, LO>::n4;
+#pragma unroll
+  for (int n = 0; n < 4 * n4; ++n) cy[n] = n < T::nnz ? T::val(n < T::nnz ? n : 0) * Y[T::my(n < T::nnz ? n : 0)] : 0.f;
+}
+
+// C[mo] = sum_n cy[n] x[mi_n] with cy read from shared memory (broadcast)
+template <int LI, int LS, int LO>
+__device__ __forceinline__ void cg_couple_cy(const float* xv, const float* cy, float* C) {
+  using T = tpc_tab::CG<LI, LS, LO>;
+  constexpr int n4 = CgInfo<LI, LS, LO>::n4;
+#pragma unroll
+  for (int o = 0; o < 2 * LO + 1; ++o) C[o] = 0.f;
+#pragma unroll
+  for (int b = 0; b < n4; ++b) {
+    const float4 v = reinterpret_cast<const float4*>(cy)[b];
+    const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int n = 4 * b + k;
+      if (n < T::nnz) C[T::mo(n < T::nnz ? n : 0)] = fmaf(vv[k], xv[T::mi(n < T::nnz ? n : 0)], C[T::mo(n < T::nnz ? n : 0)]);
+    }
+  }
+}
+
+// U[mi] = sum_n cy[n] g[mo_n]   (adjoint in x, products from shared memory)
+template <int LI, int LS, int LO>
+__device__ __forceinline__ void cg_adj_x_cy(const float* cy, const float* g, float* U) {
+  using T = tpc_tab::CG<LI, LS, LO>;
+  constexpr int n4 = CgInfo<LI, LS, LO>::n4;
+#pragma unroll
+  for (int i = 0; i < 2 * LI + 1; ++i) U[i] = 0.f;
+#pragma unroll
+  for (int b = 0; b < n4; ++b) {
+    const float4 v = reinterpret_cast<const float4*>(cy)[b];
+    const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int n = 4 * b + k;
+      if (n < T::nnz) U[T::mi(n < T::nnz ? n : 0)] = fmaf(vv[k], g[T::mo(n < T::nnz ? n : 0)], U[T::mi(n < T::nnz ? n : 0)]);
+    }
+  }
+}
+
 // U[mi] = sum c Y[my] g[mo]  (adjoint in x)
 template <int LI, int LS, int LO>
 __device__ __forceinline__ void cg_adj_x(const float* Y, const float* g, float* U) {

@@ -21,21 +21,25 @@
 
 namespace tpc {
 
-template <int KP>
+// Per-warp edge data in shared memory (dynamic: the tangent variant exceeds 48 KB).
+template <int KP, bool TAN>
 struct GeoSmem {
+  static constexpr int WT = TAN ? WARPS_PER_CTA : 1;
   int j[WARPS_PER_CTA][32];
-  float Y[WARPS_PER_CTA][32][8];
-  float phi[WARPS_PER_CTA][32][KP];
-  float Yd[WARPS_PER_CTA][32][8];
-  float phid[WARPS_PER_CTA][32][KP];
+  alignas(16) float cy[WARPS_PER_CTA][32][CY_MAX];    // c_n * Y[my_n] per edge
+  alignas(16) float phi[WARPS_PER_CTA][32][KP];
+  alignas(16) float cyd[WT][32][CY_MAX];               // c_n * Y_dot[my_n] (tangent only)
+  alignas(16) float phid[WT][32][KP];
 };
 
-// lane-per-edge preparation for one path's harmonic block (and optional tangents)
-template <int LS, int KP, bool TAN>
+// lane-per-edge preparation for one path: coupling products c*Y, radial values (and
+// their tangents along r_dot)
+template <int LI, int LS, int LO, int KP, bool TAN>
 __device__ __forceinline__ void prep_edge(const DevPlan& P, const float* __restrict__ pos,
                                           const float* __restrict__ posdot, int i, int j,
-                                          int store, GeoSmem<KP>& sm, int w, int lane) {
+                                          int store, GeoSmem<KP, TAN>& sm, int w, int lane) {
   constexpr int RS = 2 * LS + 1;
+  constexpr int N4 = CgInfo<LI, LS, LO>::n4;
   const EdgeGeo g = edge_geo(pos, i, j);
   const Pow3 pw(g.ux, g.uy, g.uz);
   float Y[RS];
@@ -43,10 +47,14 @@ __device__ __forceinline__ void prep_edge(const DevPlan& P, const float* __restr
   float phi[KP], dphi[KP];
   radial<KP, TAN>(P, g.d, phi, dphi);
   sm.j[w][lane] = store;
+  float cy[4 * N4];
+  cg_products<LI, LS, LO>(Y, cy);
 #pragma unroll
-  for (int k = 0; k < RS; ++k) sm.Y[w][lane][k] = Y[k];
+  for (int b = 0; b < N4; ++b)
+    reinterpret_cast<float4*>(sm.cy[w][lane])[b] = make_float4(cy[4 * b], cy[4 * b + 1], cy[4 * b + 2], cy[4 * b + 3]);
 #pragma unroll
-  for (int q = 0; q < KP; ++q) sm.phi[w][lane][q] = phi[q];
+  for (int q = 0; q < KP; q += 4)
+    reinterpret_cast<float4*>(sm.phi[w][lane])[q / 4] = make_float4(phi[q], phi[q + 1], phi[q + 2], phi[q + 3]);
   if (TAN) {
     float vx = 0.f, vy = 0.f, vz = 0.f;
     if (posdot) {
@@ -60,10 +68,14 @@ __device__ __forceinline__ void prep_edge(const DevPlan& P, const float* __restr
     const float tz = (vz - s * g.uz) * g.inv_d;
     float Yd[RS];
     sh_block_dir<LS>(pw, tx, ty, tz, Yd);
+    cg_products<LI, LS, LO>(Yd, cy);
 #pragma unroll
-    for (int k = 0; k < RS; ++k) sm.Yd[w][lane][k] = Yd[k];
+    for (int b = 0; b < N4; ++b)
+      reinterpret_cast<float4*>(sm.cyd[w][lane])[b] = make_float4(cy[4 * b], cy[4 * b + 1], cy[4 * b + 2], cy[4 * b + 3]);
 #pragma unroll
-    for (int q = 0; q < KP; ++q) sm.phid[w][lane][q] = dphi[q] * s;
+    for (int q = 0; q < KP; q += 4)
+      reinterpret_cast<float4*>(sm.phid[w][lane])[q / 4] =
+          make_float4(dphi[q] * s, dphi[q + 1] * s, dphi[q + 2] * s, dphi[q + 3] * s);
   }
 }
 
@@ -79,7 +91,7 @@ __device__ __forceinline__ void uvw_state_body(const DevPlan& P, const DevPath& 
                                                const float* __restrict__ posdot,
                                                const int* __restrict__ row_ptr,
                                                const int* __restrict__ src, float* S, float* Sd,
-                                               GeoSmem<KP>& sm) {
+                                               GeoSmem<KP, MODE == 1>& sm) {
   constexpr int RI = 2 * LI + 1, RS = 2 * LS + 1, RO = 2 * LO + 1;
   constexpr bool TAN = MODE == 1;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -98,38 +110,54 @@ __device__ __forceinline__ void uvw_state_body(const DevPlan& P, const DevPath& 
     const int ne = min(32, ee - e0);
     if (lane < ne) {
       const int j = __ldg(src + e0 + lane);
-      prep_edge<LS, KP, TAN>(P, pos, posdot, i, j, j, sm, w, lane);
+      prep_edge<LI, LS, LO, KP, TAN>(P, pos, posdot, i, j, j, sm, w, lane);
     }
     __syncwarp();
+    // x of the next edge is loaded while the current one is consumed
+    float xn[RI], xdn[RI];
+    {
+      const long long row = (long long)sm.j[w][0] * P.dim_in;
+#pragma unroll
+      for (int m = 0; m < RI; ++m) {
+        xn[m] = act ? __ldg(xb + row + m * p.c_in) : 0.f;
+        xdn[m] = (TAN && xdb && act) ? __ldg(xdb + row + m * p.c_in) : 0.f;
+      }
+    }
     for (int t = 0; t < ne; ++t) {
-      const long long row = (long long)sm.j[w][t] * P.dim_in;
-      float xv[RI];
+      float xv[RI], xdv[RI];
 #pragma unroll
-      for (int m = 0; m < RI; ++m) xv[m] = act ? __ldg(xb + row + m * p.c_in) : 0.f;
-      float Y[RS], phi[KP];
+      for (int m = 0; m < RI; ++m) { xv[m] = xn[m]; xdv[m] = xdn[m]; }
+      if (t + 1 < ne) {
+        const long long row = (long long)sm.j[w][t + 1] * P.dim_in;
 #pragma unroll
-      for (int k = 0; k < RS; ++k) Y[k] = sm.Y[w][t][k];
+        for (int m = 0; m < RI; ++m) {
+          xn[m] = act ? __ldg(xb + row + m * p.c_in) : 0.f;
+          if (TAN && xdb) xdn[m] = act ? __ldg(xdb + row + m * p.c_in) : 0.f;
+        }
+      }
+      float phi[KP];
 #pragma unroll
-      for (int q = 0; q < KP; ++q) phi[q] = sm.phi[w][t][q];
+      for (int q = 0; q < KP; q += 4) {
+        const float4 v = reinterpret_cast<const float4*>(sm.phi[w][t])[q / 4];
+        phi[q] = v.x; phi[q + 1] = v.y; phi[q + 2] = v.z; phi[q + 3] = v.w;
+      }
       float C[RO];
-      cg_couple<LI, LS, LO>(xv, Y, C);
+      cg_couple_cy<LI, LS, LO>(xv, sm.cy[w][t], C);
       if (!TAN) {
 #pragma unroll
         for (int q = 0; q < KP; ++q)
 #pragma unroll
           for (int o = 0; o < RO; ++o) acc[q][o] = fmaf(phi[q], C[o], acc[q][o]);
       } else {
-        float Yd[RS], phid[KP], Cd[RO], C2[RO];
+        float phid[KP], Cd[RO], C2[RO];
 #pragma unroll
-        for (int k = 0; k < RS; ++k) Yd[k] = sm.Yd[w][t][k];
-#pragma unroll
-        for (int q = 0; q < KP; ++q) phid[q] = sm.phid[w][t][q];
-        cg_couple<LI, LS, LO>(xv, Yd, Cd);
+        for (int q = 0; q < KP; q += 4) {
+          const float4 v = reinterpret_cast<const float4*>(sm.phid[w][t])[q / 4];
+          phid[q] = v.x; phid[q + 1] = v.y; phid[q + 2] = v.z; phid[q + 3] = v.w;
+        }
+        cg_couple_cy<LI, LS, LO>(xv, sm.cyd[w][t], Cd);
         if (xdb) {
-          float xdv[RI];
-#pragma unroll
-          for (int m = 0; m < RI; ++m) xdv[m] = act ? __ldg(xdb + row + m * p.c_in) : 0.f;
-          cg_couple<LI, LS, LO>(xdv, Y, C2);
+          cg_couple_cy<LI, LS, LO>(xdv, sm.cy[w][t], C2);
 #pragma unroll
           for (int o = 0; o < RO; ++o) Cd[o] += C2[o];
         }
@@ -168,7 +196,8 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32)
                 const float* __restrict__ pos, const float* __restrict__ posdot,
                 const int* __restrict__ row_ptr, const int* __restrict__ src, int node0,
                 int n_nodes, float* S, float* Sd) {
-  __shared__ GeoSmem<KP> sm;
+  extern __shared__ __align__(16) char dyn_smem[];
+  GeoSmem<KP, MODE == 1>& sm = *reinterpret_cast<GeoSmem<KP, MODE == 1>*>(dyn_smem);
   // task-major order: co-resident warps run the same (l_in, l_sh, l_out) body, which keeps
   // the instruction working set small
   const long long gw = (long long)blockIdx.x * WARPS_PER_CTA + (threadIdx.x >> 5);
@@ -346,7 +375,7 @@ __device__ __forceinline__ void uvw_src_body(const DevPlan& P, const DevPath& p,
                                              const int* __restrict__ t_ptr,
                                              const int* __restrict__ t_dst,
                                              const float* __restrict__ gout, float* X, float* Xd,
-                                             GeoSmem<KP>& sm) {
+                                             GeoSmem<KP, MODE == 1>& sm) {
   constexpr int RI = 2 * LI + 1, RS = 2 * LS + 1, RO = 2 * LO + 1;
   constexpr bool TAN = MODE == 1;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -364,33 +393,45 @@ __device__ __forceinline__ void uvw_src_body(const DevPlan& P, const DevPath& p,
     // edge j -> i seen from its source: r = pos[j] - pos[i]; keep the receiver index
     if (lane < ne) {
       const int i = __ldg(t_dst + k0 + lane);
-      prep_edge<LS, KP, TAN>(P, pos, posdot, i, j, i, sm, w, lane);
+      prep_edge<LI, LS, LO, KP, TAN>(P, pos, posdot, i, j, i, sm, w, lane);
     }
     __syncwarp();
+    float mn[RO];
+    {
+      const long long row = (long long)sm.j[w][0] * P.dim_out;
+#pragma unroll
+      for (int o = 0; o < RO; ++o) mn[o] = act ? __ldg(gb + row + o * p.c_out) : 0.f;
+    }
     for (int t = 0; t < ne; ++t) {
-      const long long row = (long long)sm.j[w][t] * P.dim_out;
       float mb[RO];
 #pragma unroll
-      for (int o = 0; o < RO; ++o) mb[o] = act ? __ldg(gb + row + o * p.c_out) : 0.f;
-      float Y[RS], phi[KP];
+      for (int o = 0; o < RO; ++o) mb[o] = mn[o];
+      if (t + 1 < ne) {
+        const long long row = (long long)sm.j[w][t + 1] * P.dim_out;
 #pragma unroll
-      for (int k = 0; k < RS; ++k) Y[k] = sm.Y[w][t][k];
+        for (int o = 0; o < RO; ++o) mn[o] = act ? __ldg(gb + row + o * p.c_out) : 0.f;
+      }
+      float phi[KP];
 #pragma unroll
-      for (int q = 0; q < KP; ++q) phi[q] = sm.phi[w][t][q];
+      for (int q = 0; q < KP; q += 4) {
+        const float4 v = reinterpret_cast<const float4*>(sm.phi[w][t])[q / 4];
+        phi[q] = v.x; phi[q + 1] = v.y; phi[q + 2] = v.z; phi[q + 3] = v.w;
+      }
       float U[RI];
-      cg_adj_x<LI, LS, LO>(Y, mb, U);
+      cg_adj_x_cy<LI, LS, LO>(sm.cy[w][t], mb, U);
       if (!TAN) {
 #pragma unroll
         for (int q = 0; q < KP; ++q)
 #pragma unroll
           for (int m = 0; m < RI; ++m) acc[q][m] = fmaf(phi[q], U[m], acc[q][m]);
       } else {
-        float Yd[RS], phid[KP], Ud[RI];
+        float phid[KP], Ud[RI];
 #pragma unroll
-        for (int k = 0; k < RS; ++k) Yd[k] = sm.Yd[w][t][k];
-#pragma unroll
-        for (int q = 0; q < KP; ++q) phid[q] = sm.phid[w][t][q];
-        cg_adj_x<LI, LS, LO>(Yd, mb, Ud);
+        for (int q = 0; q < KP; q += 4) {
+          const float4 v = reinterpret_cast<const float4*>(sm.phid[w][t])[q / 4];
+          phid[q] = v.x; phid[q + 1] = v.y; phid[q + 2] = v.z; phid[q + 3] = v.w;
+        }
+        cg_adj_x_cy<LI, LS, LO>(sm.cyd[w][t], mb, Ud);
 #pragma unroll
         for (int q = 0; q < KP; ++q)
 #pragma unroll
@@ -426,7 +467,8 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32)
                     const float* __restrict__ posdot, const int* __restrict__ t_ptr,
                     const int* __restrict__ t_dst, const float* __restrict__ gout, int node0,
                     int n_nodes, float* X, float* Xd) {
-  __shared__ GeoSmem<KP> sm;
+  extern __shared__ __align__(16) char dyn_smem[];
+  GeoSmem<KP, MODE == 1>& sm = *reinterpret_cast<GeoSmem<KP, MODE == 1>*>(dyn_smem);
   // task-major order: co-resident warps run the same (l_in, l_sh, l_out) body, which keeps
   // the instruction working set small
   const long long gw = (long long)blockIdx.x * WARPS_PER_CTA + (threadIdx.x >> 5);
@@ -456,7 +498,14 @@ cudaError_t run_uvw_state(const DevPlan& P, const Tasks& T, const float* x, cons
                           const float* pos, const float* posdot, const int* row_ptr,
                           const int* src, int node0, int n_nodes, float* S, float* Sdot,
                           cudaStream_t s) {
-  k_uvw_state<KP, MODE><<<grid_for((long long)n_nodes * T.n), WARPS_PER_CTA * 32, 0, s>>>(
+  constexpr int smem = sizeof(GeoSmem<KP, MODE == 1>);
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_uvw_state<KP, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  k_uvw_state<KP, MODE><<<grid_for((long long)n_nodes * T.n), WARPS_PER_CTA * 32, smem, s>>>(
       P, T, x, xdot, pos, posdot, row_ptr, src, node0, n_nodes, S, Sdot);
   return cudaGetLastError();
 }
@@ -475,7 +524,14 @@ cudaError_t run_uvw_src_state(const DevPlan& P, const Tasks& T, const float* pos
                               const float* posdot, const int* t_ptr, const int* t_dst,
                               const float* grad_out, int node0, int n_nodes, float* X,
                               float* Xdot, cudaStream_t s) {
-  k_uvw_src_state<KP, MODE><<<grid_for((long long)n_nodes * T.n), WARPS_PER_CTA * 32, 0, s>>>(
+  constexpr int smem = sizeof(GeoSmem<KP, MODE == 1>);
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_uvw_src_state<KP, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  k_uvw_src_state<KP, MODE><<<grid_for((long long)n_nodes * T.n), WARPS_PER_CTA * 32, smem, s>>>(
       P, T, pos, posdot, t_ptr, t_dst, grad_out, node0, n_nodes, X, Xdot);
   return cudaGetLastError();
 }
