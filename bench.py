@@ -47,6 +47,10 @@ def _workload_config(c, E):
 
 def _config_line(c, g):
     d = _workload_config(c, g.n_edges)
+    if c.cfg != CFG:
+        d["workload"] = c.name
+        d.update({"irreps": c.irreps_in, "sh_lmax": c.sh_lmax, "mode": c.mode,
+                  "radial": f"{c.radial} K={c.num_basis} r_c={c.r_cut}"})
     d["nodes"] = g.n_nodes
     return d
 
@@ -149,10 +153,10 @@ def run_native(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    c = workloads.CONFIGS[CFG]
+    c = workloads.CONFIGS[args.cfg]
     plan = binding.Plan(c.irreps_in, c.sh_lmax, c.irreps_out, c.mode, c.radial, c.num_basis, c.r_cut,
                         c.r_min, c.r_max)
-    g, rng = workloads.make_graph(c, n_nodes=args.nodes, seed=1000 + CFG + 7919 * rank)
+    g, rng = workloads.make_graph(c, n_nodes=args.nodes, seed=1000 + args.cfg + 7919 * rank)
     N, E = g.n_nodes, g.n_edges
     x_h = workloads.normal(rng, (N, plan.dim_in))
     W_h = workloads.weights(rng, c.num_basis, plan.fan_in_per_column())
@@ -227,7 +231,10 @@ def run_native(args):
     kern = {k: v for k, v in prof.items() if v[1] > 0}
     gpu_launches = int(sum(v[1] for v in kern.values()))
     timed_ms = sum(v[0] for v in kern.values())
-    dom = max((k for k in kern if k in algo), key=lambda k: kern[k][0])
+    cand = [k for k in kern if k in algo] or list(kern)
+    dom = max(cand, key=lambda k: kern[k][0])
+    if dom not in algo:
+        algo[dom] = 0
     dom_ms_step = kern[dom][0] / args.steps
     achieved = algo[dom] / (dom_ms_step / 1e3) / 1e12
     roofline = {"bound": "alu", "kernel": dom, "achieved": round(achieved, 3),
@@ -480,6 +487,8 @@ def main():
     ap.add_argument("--extras", action="store_true",
                     help="also time every pass on the other workloads (adds ~1-2 minutes)")
     ap.add_argument("--extras-cfgs", type=int, nargs="*", default=[2, 3, 5, 4])
+    ap.add_argument("--cfg", type=int, default=CFG, choices=sorted(workloads.CONFIGS),
+                    help="workload of the timed step (default: the uvw forward+backward workload)")
     ap.add_argument("--nodes", type=int, default=None,
                     help="resize the workload (same density and degree); for profiling small cases")
     args = ap.parse_args()
