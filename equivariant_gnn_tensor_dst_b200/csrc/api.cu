@@ -42,7 +42,7 @@ struct PathH {
 
 constexpr size_t kDefaultBudget = size_t(128) << 20;  // the pages' 128 MiB scratch cap
 constexpr int kSplits = 8;  // split-K factor of the weight-gradient contractions
-constexpr int kUvuRanges = 64;
+constexpr int kUvuRanges = 256;  // receiver ranges of the uvu weight gradient (fixed-order partials)
 
 int triple_index(int a, int b, int c) {
   for (int t = 0; t < tpc_tab::NTRIPLES; ++t)
@@ -697,9 +697,13 @@ tpconv_status tpconv_backward(tpconv_plan_t P, int64_t N, int64_t E, const float
   float4* gbuf = reinterpret_cast<float4*>(static_cast<char*>(ws) + L.gbuf);
   float* part = fptr(ws, L.part);
 
+  // CTAs per receiver in the receiver backward: about four times the mean number of
+  // 32-edge chunks per receiver (at most 16), so that receivers far above the mean
+  // degree are shared
+  const int edge_split = (int)std::max<long long>(1, std::min<long long>(16, (4 * E / std::max<int64_t>(N, 1) + 31) / 32));
   if (P->mode == TPCONV_UVU) {
     if (grad_pos) {
-      TPC_RUN(PC_UVU_RECV_BWD, 1, launch_uvu_recv_bwd(P->dev, P->t_in, x, pos, row_ptr, src, W, grad_out, n, gbuf, s));
+      TPC_RUN(PC_UVU_RECV_BWD, 1, launch_uvu_recv_bwd(P->dev, P->t_in, x, pos, row_ptr, src, W, grad_out, n, gbuf, edge_split, s));
       TPC_RUN(PC_POS, 1, launch_pos_finish(n, row_ptr, t_ptr, t_eid, gbuf, grad_pos, s));
     }
     if (grad_W) {
@@ -719,7 +723,7 @@ tpconv_status tpconv_backward(tpconv_plan_t P, int64_t N, int64_t E, const float
     for (int n0 = 0; n0 < n; n0 += L.recv_chunk) {
       const int cn = std::min(L.recv_chunk, n - n0);
       TPC_RUN(PC_GEMM, 1, gemm_sbar(P, grad_out, W, state, n0, cn, s));
-      TPC_RUN(PC_UVW_RECV_BWD, 1, launch_uvw_recv_bwd(P->dev, P->t_in, x, pos, row_ptr, src, state, n0, cn, gbuf, s));
+      TPC_RUN(PC_UVW_RECV_BWD, 1, launch_uvw_recv_bwd(P->dev, P->t_in, x, pos, row_ptr, src, state, n0, cn, gbuf, edge_split, s));
     }
     TPC_RUN(PC_POS, 1, launch_pos_finish(n, row_ptr, t_ptr, t_eid, gbuf, grad_pos, s));
   }

@@ -102,7 +102,7 @@ cudaError_t run_uvw_state(const DevPlan& P, const Tasks& T, const float* x, cons
 template <int KP>
 cudaError_t run_uvw_recv_bwd(const DevPlan& P, const Tasks& T, const float* x, const float* pos,
                              const int* row_ptr, const int* src, const float* Sbar, int node0,
-                             int n_nodes, float4* gbuf, cudaStream_t s);
+                             int n_nodes, float4* gbuf, int edge_split, cudaStream_t s);
 template <int KP, int MODE>
 cudaError_t run_uvw_src_state(const DevPlan& P, const Tasks& T, const float* pos,
                               const float* posdot, const int* t_ptr, const int* t_dst,
@@ -116,7 +116,7 @@ cudaError_t run_uvu_fwd(const DevPlan& P, const BlockPaths& BP, const Tasks& T, 
 template <int KP>
 cudaError_t run_uvu_recv_bwd(const DevPlan& P, const Tasks& T, const float* x, const float* pos,
                              const int* row_ptr, const int* src, const float* W,
-                             const float* grad_out, int N, float4* gbuf, cudaStream_t s);
+                             const float* grad_out, int N, float4* gbuf, int edge_split, cudaStream_t s);
 template <int KP, int MODE>
 cudaError_t run_uvu_gradw(const DevPlan& P, const Tasks& T, const float* x, const float* xdot,
                           const float* pos, const float* posdot, const int* row_ptr,
@@ -143,7 +143,7 @@ cudaError_t launch_uvw_state(const DevPlan& P, const Tasks& T, int mode, const f
 cudaError_t launch_uvw_recv_bwd(const DevPlan& P, const Tasks& T, const float* x,
                                 const float* pos, const int* row_ptr, const int* src,
                                 const float* Sbar, int node0, int n_nodes, float4* gbuf,
-                                cudaStream_t s);
+                                int edge_split, cudaStream_t s);
 cudaError_t launch_uvw_src_state(const DevPlan& P, const Tasks& T, int mode,
                                  const float* pos, const float* posdot, const int* t_ptr,
                                  const int* t_eid, const int* t_dst, const float* grad_out,
@@ -157,7 +157,7 @@ cudaError_t launch_uvu_fwd(const DevPlan& P, const BlockPaths& BP, const Tasks& 
 cudaError_t launch_uvu_recv_bwd(const DevPlan& P, const Tasks& T, const float* x,
                                 const float* pos, const int* row_ptr, const int* src,
                                 const float* W, const float* grad_out, int N, float4* gbuf,
-                                cudaStream_t s);
+                                int edge_split, cudaStream_t s);
 cudaError_t launch_uvu_gradw(const DevPlan& P, const Tasks& T, int mode, const float* x,
                              const float* xdot, const float* pos, const float* posdot,
                              const int* row_ptr, const int* src, const float* grad_out,

@@ -173,10 +173,10 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32)
 
 template <int KP>
 struct URecvSmem {
-  int j[WARPS_PER_CTA][32];
-  float Y[WARPS_PER_CTA][32][16];
-  float phi[WARPS_PER_CTA][32][KP];
-  float accY[WARPS_PER_CTA][32][16];
+  int j[32];
+  float Y[32][16];
+  float phi[32][KP];
+  float accY[WARPS_PER_CTA][32][16];   // per-warp partial sums, combined in warp order
   float accphi[WARPS_PER_CTA][32][KP];
 };
 
@@ -200,12 +200,12 @@ __device__ __forceinline__ void uvu_recv_body(const DevPlan& P, const DevPath& p
   const int yw = reduce_multi_index<8>(lane), pw_ = reduce_multi_index<KP>(lane);
   const bool ywr = reduce_multi_writer<8>(lane), pwr = reduce_multi_writer<KP>(lane);
   for (int t = 0; t < ne; ++t) {
-    const long long row = (long long)sm.j[w][t] * P.dim_in;
+    const long long row = (long long)sm.j[t] * P.dim_in;
     float xv[RI], Y[RS], C[RO];
 #pragma unroll
     for (int k = 0; k < RI; ++k) xv[k] = act ? __ldg(xb + row + k * p.c_in) : 0.f;
 #pragma unroll
-    for (int k = 0; k < RS; ++k) Y[k] = sm.Y[w][t][LS * LS + k];
+    for (int k = 0; k < RS; ++k) Y[k] = sm.Y[t][LS * LS + k];
     cg_couple<LI, LS, LO>(xv, Y, C);
     float h = 0.f;
 #pragma unroll
@@ -214,7 +214,7 @@ __device__ __forceinline__ void uvu_recv_body(const DevPlan& P, const DevPath& p
     float pp[KP];
 #pragma unroll
     for (int q = 0; q < KP; ++q) {
-      we = fmaf(sm.phi[w][t][q], a[q], we);
+      we = fmaf(sm.phi[t][q], a[q], we);
       pp[q] = a[q] * h;                                        // eq. 20 (per channel)
     }
     float G[RO], py[8];
@@ -231,6 +231,8 @@ __device__ __forceinline__ void uvu_recv_body(const DevPlan& P, const DevPath& p
   }
 }
 
+// One CTA per (receiver, share of its 32-edge chunks); its warps split the (path,
+// channel chunk) tasks.
 template <int KP>
 __global__ void __launch_bounds__(WARPS_PER_CTA * 32)
     k_uvu_recv_bwd(DevPlan P, Tasks T, const float* __restrict__ x, const float* __restrict__ pos,
@@ -239,26 +241,28 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32)
                    float4* gbuf) {
   __shared__ URecvSmem<KP> sm;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int i = blockIdx.x * WARPS_PER_CTA + w;
+  const int i = blockIdx.x;
   if (i >= N) return;
   const int eb = __ldg(row_ptr + i), ee = __ldg(row_ptr + i + 1);
-  for (int e0 = eb; e0 < ee; e0 += 32) {
+  for (int e0 = eb + 32 * blockIdx.y; e0 < ee; e0 += 32 * gridDim.y) {
     const int ne = min(32, ee - e0);
-    if (lane < ne) {
+    if (w == 0 && lane < ne) {
       const int j = __ldg(src + e0 + lane);
       const EdgeGeo g = edge_geo(pos, i, j);
       const Pow3 pw(g.ux, g.uy, g.uz);
       float Y[16], phi[KP], dphi[KP];
       sh_all(pw, Y);
       radial<KP, false>(P, g.d, phi, dphi);
-      sm.j[w][lane] = j;
+      sm.j[lane] = j;
 #pragma unroll
-      for (int k = 0; k < 16; ++k) { sm.Y[w][lane][k] = Y[k]; sm.accY[w][lane][k] = 0.f; }
+      for (int k = 0; k < 16; ++k) sm.Y[lane][k] = Y[k];
 #pragma unroll
-      for (int q = 0; q < KP; ++q) { sm.phi[w][lane][q] = phi[q]; sm.accphi[w][lane][q] = 0.f; }
+      for (int q = 0; q < KP; ++q) sm.phi[lane][q] = phi[q];
     }
-    __syncwarp();
-    for (int task = 0; task < T.n; ++task) {
+    for (int k = threadIdx.x; k < WARPS_PER_CTA * 32 * 16; k += blockDim.x) (&sm.accY[0][0][0])[k] = 0.f;
+    for (int k = threadIdx.x; k < WARPS_PER_CTA * 32 * KP; k += blockDim.x) (&sm.accphi[0][0][0])[k] = 0.f;
+    __syncthreads();
+    for (int task = w; task < T.n; task += WARPS_PER_CTA) {
       const DevPath& p = P.p[T.a[task]];
       const int chunk = T.b[task];
       dispatch_type(p.type, [&](auto tr) {
@@ -266,21 +270,31 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32)
         uvu_recv_body<TR::li, TR::ls, TR::lo, KP>(P, p, chunk, i, ne, x, W, gout, sm);
       });
     }
-    __syncwarp();
-    if (lane < ne) {
-      const int j = sm.j[w][lane];
+    __syncthreads();
+    if (w == 0 && lane < ne) {
+      const int j = sm.j[lane];
       const EdgeGeo g = edge_geo(pos, i, j);
       const Pow3 pw(g.ux, g.uy, g.uz);
       float phi[KP], dphi[KP], Yb[16];
       radial<KP, true>(P, g.d, phi, dphi);
 #pragma unroll
-      for (int k = 0; k < 16; ++k) Yb[k] = sm.accY[w][lane][k];
+      for (int k = 0; k < 16; ++k) {
+        float s = 0.f;
+#pragma unroll
+        for (int ww = 0; ww < WARPS_PER_CTA; ++ww) s += sm.accY[ww][lane][k];
+        Yb[k] = s;
+      }
       float vx = 0.f, vy = 0.f, vz = 0.f;
       sh_vjp_all(pw, Yb, vx, vy, vz);
       const float vr = vx * g.ux + vy * g.uy + vz * g.uz;
       float s = 0.f;
 #pragma unroll
-      for (int q = 0; q < KP; ++q) s = fmaf(sm.accphi[w][lane][q], dphi[q], s);
+      for (int q = 0; q < KP; ++q) {
+        float a = 0.f;
+#pragma unroll
+        for (int ww = 0; ww < WARPS_PER_CTA; ++ww) a += sm.accphi[ww][lane][q];
+        s = fmaf(a, dphi[q], s);
+      }
       float4 o;
       o.x = (vx - vr * g.ux) * g.inv_d + s * g.ux;
       o.y = (vy - vr * g.uy) * g.inv_d + s * g.uy;
@@ -288,7 +302,7 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32)
       o.w = 0.f;
       gbuf[e0 + lane] = o;
     }
-    __syncwarp();
+    __syncthreads();
   }
 }
 
@@ -514,8 +528,8 @@ cudaError_t run_uvu_fwd(const DevPlan& P, const BlockPaths& BP, const Tasks& T, 
 template <int KP>
 cudaError_t run_uvu_recv_bwd(const DevPlan& P, const Tasks& T, const float* x, const float* pos,
                              const int* row_ptr, const int* src, const float* W,
-                             const float* grad_out, int N, float4* gbuf, cudaStream_t s) {
-  k_uvu_recv_bwd<KP><<<ugrid(N), WARPS_PER_CTA * 32, 0, s>>>(P, T, x, pos, row_ptr, src, W,
+                             const float* grad_out, int N, float4* gbuf, int edge_split, cudaStream_t s) {
+  k_uvu_recv_bwd<KP><<<dim3((unsigned)N, (unsigned)edge_split), WARPS_PER_CTA * 32, 0, s>>>(P, T, x, pos, row_ptr, src, W,
                                                             grad_out, N, gbuf);
   return cudaGetLastError();
 }
@@ -564,7 +578,7 @@ template cudaError_t run_uvu_src<TPC_UNIT_KP, TPC_UNIT_MODE>(
 #if TPC_UNIT_PART == TPC_PART_RECV
 template cudaError_t run_uvu_recv_bwd<TPC_UNIT_KP>(const DevPlan&, const Tasks&, const float*,
                                                    const float*, const int*, const int*,
-                                                   const float*, const float*, int, float4*,
+                                                   const float*, const float*, int, float4*, int,
                                                    cudaStream_t);
 #endif
 #endif

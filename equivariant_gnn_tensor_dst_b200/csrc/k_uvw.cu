@@ -289,8 +289,9 @@ __device__ __forceinline__ void uvw_recv_body(const DevPlan& P, const DevPath& p
   }
 }
 
-// One CTA per receiver; its warps split the (path, channel chunk) tasks and keep
-// per-warp partial sums of phi_bar and Y_bar per edge, added in warp order.
+// One CTA per (receiver, share of its 32-edge chunks); its warps split the (path,
+// channel chunk) tasks and keep per-warp partial sums of phi_bar and Y_bar per edge,
+// added in warp order.
 template <int KP>
 __global__ void __launch_bounds__(WARPS_PER_CTA * 32)
     k_uvw_recv_bwd(DevPlan P, Tasks T, const float* __restrict__ x, const float* __restrict__ pos,
@@ -302,7 +303,9 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32)
   if (node_local >= n_nodes) return;
   const int i = node0 + node_local;
   const int eb = __ldg(row_ptr + i), ee = __ldg(row_ptr + i + 1);
-  for (int e0 = eb; e0 < ee; e0 += 32) {
+  // the 32-edge chunks of one receiver are shared by gridDim.y CTAs (their per-edge
+  // results are independent), which keeps high-degree receivers off the critical path
+  for (int e0 = eb + 32 * blockIdx.y; e0 < ee; e0 += 32 * gridDim.y) {
     const int ne = min(32, ee - e0);
     if (w == 0 && lane < ne) {
       const int j = __ldg(src + e0 + lane);
@@ -513,8 +516,8 @@ cudaError_t run_uvw_state(const DevPlan& P, const Tasks& T, const float* x, cons
 template <int KP>
 cudaError_t run_uvw_recv_bwd(const DevPlan& P, const Tasks& T, const float* x, const float* pos,
                              const int* row_ptr, const int* src, const float* Sbar, int node0,
-                             int n_nodes, float4* gbuf, cudaStream_t s) {
-  k_uvw_recv_bwd<KP><<<(unsigned)n_nodes, WARPS_PER_CTA * 32, 0, s>>>(P, T, x, pos, row_ptr, src,
+                             int n_nodes, float4* gbuf, int edge_split, cudaStream_t s) {
+  k_uvw_recv_bwd<KP><<<dim3((unsigned)n_nodes, (unsigned)edge_split), WARPS_PER_CTA * 32, 0, s>>>(P, T, x, pos, row_ptr, src,
                                                                      Sbar, node0, n_nodes, gbuf);
   return cudaGetLastError();
 }
@@ -555,7 +558,7 @@ template cudaError_t run_uvw_src_state<TPC_UNIT_KP, TPC_UNIT_MODE>(
 #if TPC_UNIT_PART == TPC_PART_RECV
 template cudaError_t run_uvw_recv_bwd<TPC_UNIT_KP>(const DevPlan&, const Tasks&, const float*,
                                                    const float*, const int*, const int*,
-                                                   const float*, int, int, float4*,
+                                                   const float*, int, int, float4*, int,
                                                    cudaStream_t);
 #endif
 #endif

@@ -19,10 +19,11 @@ cudaError_t launch_uvw_state(const DevPlan& P, const Tasks& T, int mode, const f
 cudaError_t launch_uvw_recv_bwd(const DevPlan& P, const Tasks& T, const float* x,
                                 const float* pos, const int* row_ptr, const int* src,
                                 const float* Sbar, int node0, int n_nodes, float4* gbuf,
-                                cudaStream_t s) {
+                                int edge_split, cudaStream_t s) {
   if (n_nodes <= 0) return cudaSuccess;
-  if (P.K <= 8) return run_uvw_recv_bwd<8>(P, T, x, pos, row_ptr, src, Sbar, node0, n_nodes, gbuf, s);
-  return run_uvw_recv_bwd<16>(P, T, x, pos, row_ptr, src, Sbar, node0, n_nodes, gbuf, s);
+  if (edge_split < 1) edge_split = 1;
+  if (P.K <= 8) return run_uvw_recv_bwd<8>(P, T, x, pos, row_ptr, src, Sbar, node0, n_nodes, gbuf, edge_split, s);
+  return run_uvw_recv_bwd<16>(P, T, x, pos, row_ptr, src, Sbar, node0, n_nodes, gbuf, edge_split, s);
 }
 
 cudaError_t launch_uvw_src_state(const DevPlan& P, const Tasks& T, int mode,
@@ -47,10 +48,11 @@ cudaError_t launch_uvu_fwd(const DevPlan& P, const BlockPaths& BP, const Tasks& 
 cudaError_t launch_uvu_recv_bwd(const DevPlan& P, const Tasks& T, const float* x,
                                 const float* pos, const int* row_ptr, const int* src,
                                 const float* W, const float* grad_out, int N, float4* gbuf,
-                                cudaStream_t s) {
+                                int edge_split, cudaStream_t s) {
   if (N <= 0) return cudaSuccess;
-  if (P.K <= 8) return run_uvu_recv_bwd<8>(P, T, x, pos, row_ptr, src, W, grad_out, N, gbuf, s);
-  return run_uvu_recv_bwd<16>(P, T, x, pos, row_ptr, src, W, grad_out, N, gbuf, s);
+  if (edge_split < 1) edge_split = 1;
+  if (P.K <= 8) return run_uvu_recv_bwd<8>(P, T, x, pos, row_ptr, src, W, grad_out, N, gbuf, edge_split, s);
+  return run_uvu_recv_bwd<16>(P, T, x, pos, row_ptr, src, W, grad_out, N, gbuf, edge_split, s);
 }
 
 cudaError_t launch_uvu_gradw(const DevPlan& P, const Tasks& T, int mode, const float* x,
