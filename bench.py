@@ -35,6 +35,24 @@ UNIT = "edges/s"
 CFG = 2
 FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # SM count x FP32 lanes x FMA x max clock
 L2_FLUSH_BYTES = 256 << 20                          # > 126 MB L2
+TF32_PER_BF16 = 1.1 / 2.25                          # nominal dense TF32 / BF16 tensor rates
+SPLIT_MMAS = 3                                      # 3xTF32: three TF32 products per fp32 product
+# DRAM bytes per launch of each kernel category, averaged over one step of this workload
+# from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum); None when not
+# measured for the current kernels.
+TRAFFIC_BYTES_PER_LAUNCH = {}
+
+
+def measured_peaks():
+    """Peaks measured on this machine (MEASURED_PEAKS.json), else the recipe's fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16": float(d["bf16_tflops"]),
+                "source": "of measured (MEASURED_PEAKS.json: bf16 burst; the step keeps the SM clock at max)"}
+    except (OSError, ValueError, KeyError):
+        return {"hbm_gbs": 6650.0, "bf16": 1590.0, "source": "of fallback (6.65 TB/s, 1.59 PFLOP/s bf16 burst)"}
 
 
 def _workload_config(c, E):
@@ -62,13 +80,28 @@ def _dist():
     return ws, rank, local
 
 
+def reduce_over_ranks(total_ms, edges, device=None):
+    """Max of the timed milliseconds and sum of the processed edges over all ranks
+    (identity on a single rank).  Every rank must call it, in the same order."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(total_ms), float(edges)
+    dev = device if device is not None else torch.device("cpu")
+    t = torch.tensor([float(total_ms)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e = torch.tensor([float(edges)], dtype=torch.float64, device=dev)
+    dist.all_reduce(e, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(e.item())
+
+
 # ---------------------------------------------------------------------------
 # algorithmic operation counts (per edge and per node), from the plan's paths
 # ---------------------------------------------------------------------------
 
 def flop_model(plan):
     K = plan.num_basis
-    f = dict(state=0, recv=0, src=0, gemm_node=0)
+    f = dict(state=0, recv=0, src=0, gemm_node=0, gemm_node_bytes=0)
     for p in plan.paths():
         ri, ro = 2 * p["l_in"] + 1, 2 * p["l_out"] + 1
         nnz, ci, co = p["nnz"], p["c_in"], p["c_out"]
@@ -76,6 +109,11 @@ def flop_model(plan):
         f["recv"] += 2 * ci * (2 * nnz + 2 * K * ro)       # coupling, phi_bar, T_bar, Y_bar
         f["src"] += 2 * co * (nnz + K * ri)                # adjoint coupling + source state
         f["gemm_node"] += 2 * K * ci * co * (2 * ro + 2 * ri)  # S A, m_bar A^T, X A^T, x^T X
+        # fp32 operand bytes of the five channel contractions of a forward+backward step:
+        # m = S A (read S, write m), S_bar = m_bar A^T (read m_bar, write S_bar),
+        # A_bar += S^T m_bar (read S, m_bar), x_bar = X A^T (read X, write x_bar),
+        # A_bar += x^T X (read x, X); the weights stay in L2.
+        f["gemm_node_bytes"] += 4 * (3 * ro * K * ci + 3 * ro * co + 2 * ri * K * co + 2 * ri * ci)
     return f
 
 
@@ -211,36 +249,48 @@ def run_native(args):
     barrier()
     clocks = sampler.stop()
     total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
-        ee = torch.tensor([float(E)], device=dev, dtype=torch.float64)
-        dist.all_reduce(ee, op=dist.ReduceOp.SUM)
-        edges_all = float(ee.item())
-    else:
-        edges_all = float(E)
+    total_ms, edges_all = reduce_over_ranks(total_ms, E, dev)
     ms_step = total_ms / args.steps
     value = edges_all * args.steps / (total_ms / 1e3)
 
-    # live roofline of the dominant kernel category (CUDA events over the timed region)
+    # live roofline of every kernel category (CUDA events over the timed region)
     fm = flop_model(plan)
     algo = {"uvw_receiver_state": fm["state"] * E, "uvw_receiver_backward": fm["recv"] * E,
             "uvw_source_state": fm["src"] * E, "channel_gemm": fm["gemm_node"] * N}
+    peaks = measured_peaks()
+    tc_peak = peaks["bf16"] * TF32_PER_BF16 / SPLIT_MMAS
     kern = {k: v for k, v in prof.items() if v[1] > 0}
     gpu_launches = int(sum(v[1] for v in kern.values()))
     timed_ms = sum(v[0] for v in kern.values())
-    cand = [k for k in kern if k in algo] or list(kern)
-    dom = max(cand, key=lambda k: kern[k][0])
-    if dom not in algo:
-        algo[dom] = 0
-    dom_ms_step = kern[dom][0] / args.steps
-    achieved = algo[dom] / (dom_ms_step / 1e3) / 1e12
-    roofline = {"bound": "alu", "kernel": dom, "achieved": round(achieved, 3),
-                "peak": round(FP32_PEAK_TFLOPS, 1), "unit": "TFLOP/s",
-                "frac": round(achieved / FP32_PEAK_TFLOPS, 4), "traffic": None,
-                "peak_note": "derived: 148 SMs x 128 FP32 lanes x 2 flop x 1965 MHz"}
+    rooflines = {}
+    for k, (ms, n) in kern.items():
+        if k not in algo or ms <= 0:
+            continue
+        ach = algo[k] / (ms / args.steps / 1e3) / 1e12
+        if k == "channel_gemm":
+            # the channel contraction is bound by whichever of its tensor-core time and its
+            # HBM time is longer at the peaks
+            t_tc = algo[k] / (tc_peak * 1e12)
+            t_hbm = fm["gemm_node_bytes"] * N / (peaks["hbm_gbs"] * 1e9)
+            if t_tc >= t_hbm:
+                rl = {"bound": "tensor", "achieved": round(ach, 3), "peak": round(tc_peak, 1), "unit": "TFLOP/s",
+                      "peak_note": f"fp32 products via 3xTF32: bf16 x {TF32_PER_BF16:.3f} (nominal TF32/BF16) "
+                                   f"/ {SPLIT_MMAS}, bf16 {peaks['source']}"}
+            else:
+                gbs = fm["gemm_node_bytes"] * N / (ms / args.steps / 1e3) / 1e9
+                rl = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                      "peak_note": f"HBM copy bandwidth {peaks['source']}"}
+            rl["algorithmic_per_step"] = {"flop": algo[k], "bytes": fm["gemm_node_bytes"] * N}
+        else:
+            rl = {"bound": "alu", "achieved": round(ach, 3), "peak": round(FP32_PEAK_TFLOPS, 1), "unit": "TFLOP/s",
+                  "peak_note": "derived: 148 SMs x 128 FP32 lanes x 2 flop x 1965 MHz"}
+            rl["algorithmic_per_step"] = {"flop": algo[k]}
+        rl["frac"] = round(rl["achieved"] / rl["peak"], 4)
+        tb = TRAFFIC_BYTES_PER_LAUNCH.get(k)
+        rl["traffic"] = tb
+        rooflines[k] = rl
+    dom = max(rooflines, key=lambda k: kern[k][0])
+    roofline = dict(rooflines[dom], kernel=dom)
     breakdown = {k: {"ms_per_step": round(v[0] / args.steps, 4), "launches_per_step": v[1] / args.steps,
                      "share": round(v[0] / timed_ms, 4) if timed_ms else None} for k, v in kern.items()}
     total_algo = sum(algo.values())
@@ -277,12 +327,7 @@ def run_native(args):
             e2e_step()
         s1.record(stream)
         torch.cuda.synchronize()
-        e_ms = s0.elapsed_time(s1)
-        if world > 1:
-            import torch.distributed as dist
-            tt = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt.item())
+        e_ms, _ = reduce_over_ranks(s0.elapsed_time(s1), E, dev)
         e2e = {"value": round(edges_all * ne2e / (e_ms / 1e3), 1), "unit": UNIT, "h2d_bytes_per_step": int(bi),
                "d2h_bytes_per_step": int(bo), "steps": ne2e,
                "includes": "H2D of x, pos, CSR, W, grad_out; source-view build; forward; backward; "
@@ -304,7 +349,7 @@ def run_native(args):
                 "workspace_bytes": {"declared": int(ws_bytes), "peak_alloc_delta": int(peak_delta)},
                 "step_algorithmic_tflop": round(total_algo / 1e12, 4),
                 "step_tflops_achieved": round(total_algo / (ms_step / 1e3) / 1e12, 3),
-                "breakdown": breakdown}
+                "breakdown": breakdown, "rooflines": rooflines}
         if extras is not None:
             line["extras"] = extras
         print(json.dumps(line), flush=True)

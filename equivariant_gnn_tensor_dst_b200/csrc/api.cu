@@ -533,6 +533,11 @@ struct Batch {
     // unit stride in k and k blocks (if any) of a multiple of 32
     s.a_vec4 = ((reinterpret_cast<uintptr_t>(A) & 15u) == 0) && Am.s1 % 4 == 0 && Am.s2 % 4 == 0 &&
                Ak.s2 == 1 && (Ak.d == 0x7fffffff || (Ak.d % 32 == 0 && Ak.s1 % 4 == 0));
+    s.b_vec4 = ((reinterpret_cast<uintptr_t>(B) & 15u) == 0) && Bn.s1 % 4 == 0 && Bn.s2 % 4 == 0 &&
+               Bk.s2 == 1 && (Bk.d == 0x7fffffff || (Bk.d % 32 == 0 && Bk.s1 % 4 == 0));
+    // 16-byte vector loads along m: unit m stride and every k offset a multiple of 4 floats
+    s.a_mvec4 = ((reinterpret_cast<uintptr_t>(A) & 15u) == 0) && Am.d == 0x7fffffff && Am.s2 == 1 &&
+                Ak.s1 % 4 == 0 && Ak.s2 % 4 == 0;
     GemmProblem& p = g.pr[g.n_problems - 1];
     ++p.nseg;
     p.Ktot += K;

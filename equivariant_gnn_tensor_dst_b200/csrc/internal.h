@@ -73,6 +73,8 @@ struct GemmSeg {
   const float* B; Idx2 Bk, Bn;   // B(k, n)
   int K;
   int a_vec4;                    // A rows are 16-byte aligned and contiguous in k
+  int b_vec4;                    // B columns are 16-byte aligned and contiguous in k
+  int a_mvec4;                   // A is contiguous in m (unit m stride), 16-byte aligned at every k
 };
 
 struct GemmProblem {

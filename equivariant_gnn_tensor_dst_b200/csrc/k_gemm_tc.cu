@@ -10,20 +10,23 @@
 // a = hi + lo with hi = a truncated to TF32 and lo = a - hi; each k-step
 // issues hi*hi + hi*lo + lo*hi into the same fp32 accumulator ("3xTF32", the
 // decomposition of Ootomo and Yokota, 2022), which keeps the relative error near
-// 2^-21 instead of TF32's 2^-11.  The TF32 MMA reads only the top 19 bits of each
-// 32-bit operand, so the raw fp32 tile itself serves as "hi"; only "lo" is computed.
+// 2^-21 instead of TF32's 2^-11.
 //
 // Structure: one CTA of 256 threads per 128 x NT output tile (NT = 64 or 128) and
-// split-K slice.  Operand tiles are copied from global memory with cp.async through
-// the same two-level affine index maps as the rest of the library (so ir_mul node
-// rows, weight columns and workspace states are read in place) straight into the
-// canonical K-major, no-swizzle core-matrix layout (8 rows x 16 bytes per core matrix,
-// row groups of a k column contiguous).  Two raw stages: the copies of tile t+1 are in
-// flight while tile t is split and multiplied; every thread splits exactly the
-// elements it copied, so one barrier per tile suffices.  A tcgen05.commit per tile
-// arrives on an mbarrier that frees the raw stage and the lo buffer.  The
-// epilogue reads the TMEM accumulator with tcgen05.ld (one TMEM lane = one output row)
-// and writes C (or the split-K partial) through the output map.  Every mbarrier wait is
+// split-K slice, two CTAs per SM, warp-specialised around a ring of shared-memory stages
+// of 32 k values:
+//   - warps 0-3 (producers) copy the raw fp32 A and B tiles of a stage from global memory
+//     with cp.async, through the same two-level affine index maps as the rest of the
+//     library (ir_mul node rows, weight columns and workspace states are read in place);
+//     the copies arrive on the stage's "full" mbarrier when they land;
+//   - warps 4-7 (converters) split the stage: thread (quadrant w, lane) owns output row
+//     32 w + lane and writes hi(A) and lo(A) of its row into its TMEM lane (tcgen05.st);
+//     B is split in place in shared memory (raw -> hi, plus a lo copy); one converter
+//     thread then issues hi*hi + hi*lo + lo*hi (A from TMEM, B from shared memory) into
+//     the fp32 TMEM accumulator and commits them to the stage's "empty" mbarrier, which
+//     the producers wait on before refilling the stage.
+// The epilogue reads the accumulator with tcgen05.ld (one TMEM lane = one output row) and
+// writes C (or the split-K partial) through the output map.  Every mbarrier wait is
 // bounded; a wait that gives up sets *err and the kernel still releases its TMEM.
 #include <cuda_runtime.h>
 #include <cstdint>
@@ -90,11 +93,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   return false;
 }
 
-// Asynchronous operand staging: raw fp32 tiles go straight from global to shared memory
-// with cp.async (zero-filled outside the operand) into a ring of RING stages, already in
-// the canonical core-matrix layout.  A conversion pass then splits a landed stage into
-// the hi and lo buffers read by the MMAs.  Thread t owns row t % nrows of an operand
-// tile and the contiguous k range [(t / nrows) * KW, +KW).
+// Asynchronous operand staging: raw fp32 values go straight from global to shared memory
+// with cp.async, zero-filled outside the operand.
 __device__ __forceinline__ void cp_async4(uint32_t dst, const float* src, bool valid) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(valid ? 4 : 0)
                : "memory");
@@ -129,7 +129,8 @@ __device__ __forceinline__ void op_step(OpCursor& c, int dk) {
   while (c.kr >= c.d) { c.kr -= c.d; ++c.kq; }
 }
 
-// Issue the cp.async copies of this thread's share of one operand tile.
+// Issue the cp.async copies of one operand tile row owned by this thread: row `row`, k
+// range [kbeg, kbeg + KW), into the K-major core-matrix layout (tile_off).
 template <int KW, int ROWS>
 __device__ __forceinline__ void issue_operand(const OpCursor& c, const float* safe, int kt, int khi, int kbeg,
                                               int row, bool vec4, uint32_t dst) {
@@ -159,24 +160,59 @@ __device__ __forceinline__ void issue_operand(const OpCursor& c, const float* sa
   }
 }
 
+// Shared-memory plan: RING stages, each [A raw | B raw | B lo], 1 KB aligned, then the
+// mbarriers and the TMEM address.
+//   A raw (128 x 32 fp32) is read back only by the converter warps, one output row per
+//   thread, so its layout is chosen for conflict-free reads: k-contiguous operands are
+//   stored row-major with the 16-byte chunks of row r XOR-swizzled by r % 8 ("KM"),
+//   m-contiguous operands k-major, [k][128 m] ("MM").
+//   B raw / B lo (NT x 32) are in the tensor core's K-major no-swizzle core-matrix
+//   layout (tile_off); B raw doubles as the "hi" operand.
+// TMEM: columns [0, NT) the fp32 accumulator; stage s holds A hi in columns
+// NT + 64 s + [0, 32) and A lo in NT + 64 s + [32, 64).
 template <int NT>
 struct TcSmem {
   static constexpr int A_BYTES = TC_M * TC_K * 4;
   static constexpr int B_BYTES = NT * TC_K * 4;
-  static constexpr int RAW = A_BYTES + B_BYTES;      // one raw fp32 stage [A | B]; also the "hi" operand
-  static constexpr int RING = 2;                     // raw stages
-  static constexpr int TOTAL = RING * RAW + RAW + 2048;  // + lo buffer, alignment, barriers, TMEM address
+  static constexpr int STAGE = A_BYTES + 2 * B_BYTES;
+  static constexpr int RING = NT == 64 ? 3 : 2;       // stages (two CTAs share an SM)
+  static constexpr int BAR_OFF = RING * STAGE;
+  static constexpr int TOTAL = BAR_OFF + 128 + 1024;  // barriers, TMEM address; alignment slack
+  static constexpr int TMEM_COLS = 256;
+  static_assert(NT + 64 * RING <= TMEM_COLS, "TMEM columns");
 };
 
+constexpr int TC_PRODUCERS = 128;  // warps 0-3 copy operand tiles
+constexpr int TC_CONVERTERS = 128; // warps 4-7 split tiles, fill TMEM and issue the MMAs
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar) : "memory");
+}
+
+// A operands with unit m stride are staged k-major ("MM"), all others row-major ("KM")
+__device__ __forceinline__ bool a_is_mm(const GemmSeg& S) { return S.Am.d == 0x7fffffff && S.Am.s2 == 1; }
+
+// byte offset of 16-byte chunk c (k = 4c .. 4c + 3) of row r in a KM stage
+__device__ __forceinline__ uint32_t km_off(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
+
+// step a (k / d, k % d) position by dk
+__device__ __forceinline__ void kstep(int& kq, int& kr, int d, int dk) {
+  kr += dk;
+  while (kr >= d) { kr -= d; ++kq; }
+}
+
 template <int NT>
-__global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ GemmBatch g, int* err) {
+__global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant__ GemmBatch g, int* err) {
   extern __shared__ char smem_raw[];
   char* smem = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   using SM = TcSmem<NT>;
-  char* ring = smem;                                  // RING raw stages (the "hi" operands)
-  char* lo_buf = smem + SM::RING * SM::RAW;           // "lo" operand of the current tile
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::RING * SM::RAW + SM::RAW);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::RING * SM::RAW + SM::RAW + 64);
+  char* ring = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::BAR_OFF);  // stage copied (TC_PRODUCERS arrivals)
+  uint64_t* empty = full + SM::RING;                  // stage consumed by the MMAs (tcgen05.commit)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(empty + SM::RING);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // locate (problem, m tile, n tile)
@@ -192,12 +228,15 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
   const int kb = split * kper, ke = min(P.Ktot, kb + kper);
 
   if (tid == 0) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[0])));
+    for (int i = 0; i < SM::RING; ++i) {
+      mbar_init(smem_u32(&full[i]), TC_PRODUCERS);
+      mbar_init(smem_u32(&empty[i]), 1);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"(NT));
+                 "r"(SM::TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -206,8 +245,7 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
   const uint32_t tmem = *tmem_slot;
 
   constexpr uint32_t IDESC = instr_desc<NT>();
-  constexpr int KWA = TC_K / (TC_THREADS / TC_M);  // k values per thread for the A operand
-  constexpr int KWB = TC_K / (TC_THREADS / NT);    // k values per thread for the B operand
+  constexpr int KWB = TC_K / (TC_PRODUCERS / NT);    // k values per producer for the B operand
   bool ok = true;
 
   // The k-tiles of this split, as (segment, kt) pairs, walked by a cursor.
@@ -224,34 +262,6 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
     }
     c.have = false;
   };
-  const int rowA = tid % TC_M, kbegA = (tid / TC_M) * KWA;
-  const int rowB = tid % NT, kbegB = (tid / NT) * KWB;
-  Cursor ld{0, 0, 0, 0, false};
-  OpCursor ca{}, cb{};
-  int cur_seg = -1;
-  advance_to_valid(ld);
-  auto issue_tile = [&](int slot) {
-    // always commit a group (possibly empty) so that group counting stays uniform
-    if (ld.have) {
-      const GemmSeg& S = g.sg[P.seg0 + ld.seg];
-      if (ld.seg != cur_seg) {  // entering a segment: row offsets and k positions
-        op_enter(ca, S.A, S.Am, S.Ak, m0 + rowA, P.M, ld.kt);
-        op_enter(cb, S.B, S.Bn, S.Bk, n0 + rowB, P.N, ld.kt);
-        cur_seg = ld.seg;
-      }
-      const uint32_t dst = smem_u32(ring + slot * SM::RAW);
-      issue_operand<KWA, TC_M>(ca, S.A, ld.kt, ld.khi, kbegA, rowA, S.a_vec4 != 0, dst);
-      issue_operand<KWB, NT>(cb, S.B, ld.kt, ld.khi, kbegB, rowB, false, dst + SM::A_BYTES);
-      const int seg_before = ld.seg;
-      ld.kt += TC_K;
-      advance_to_valid(ld);
-      if (ld.have && ld.seg == seg_before) {
-        op_step(ca, TC_K);
-        op_step(cb, TC_K);
-      }
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-  };
   // number of k-tiles of this split
   int ntiles = 0;
   {
@@ -259,74 +269,217 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
     advance_to_valid(c);
     while (c.have) { ++ntiles; c.kt += TC_K; advance_to_valid(c); }
   }
-  issue_tile(0);
-  uint32_t phase = 0u;
-  int it = 0;
+
+  if (warp < TC_PRODUCERS / 32) {
+    // ---- producers: copy stage `it` once the MMAs of stage it - RING have released it;
+    // up to RING stages are in flight
+    const int p = tid;
+    const int rowB = p % NT, kbegB = (p / NT) * KWB;
+    Cursor ld{0, 0, 0, 0, false};
+    OpCursor cb{};
+    int cur_seg = -1;
+    bool a_mm = false, a_vec = false;
+    const float* arow[8];  // KM vector copies: rows 16 q + p / 8
+    const float* mrow = nullptr;  // MM copies: row base of this thread's m (or chunk of 4 m)
+    long long a_s1 = 0, a_s2 = 0;
+    int a_d = 1;
+    advance_to_valid(ld);
 #pragma unroll 1
-  for (; it < ntiles; ++it) {
-    // MMA(it-1) read raw stage (it+1) % 2 and the lo buffer: wait before reusing them
-    if (it >= 1) {
-      ok = mbar_wait(smem_u32(&bars[0]), phase) && ok;
-      phase ^= 1u;
+    for (int it = 0; it < ntiles; ++it) {
+      const int slot = it % SM::RING;
+      if (it >= SM::RING) ok = mbar_wait(smem_u32(&empty[slot]), ((it / SM::RING) - 1) & 1) && ok;
+      const GemmSeg& S = g.sg[P.seg0 + ld.seg];
+      if (ld.seg != cur_seg) {  // entering a segment: layout, row offsets, k map
+        cur_seg = ld.seg;
+        a_mm = a_is_mm(S);
+        a_vec = a_mm ? (S.a_mvec4 != 0 && (P.M & 3) == 0) : (S.a_vec4 != 0);
+        a_s1 = S.Ak.s1; a_s2 = S.Ak.s2; a_d = S.Ak.d;
+        if (a_mm) {
+          const int m = m0 + (a_vec ? 4 * (p & 31) : p);
+          mrow = m < P.M ? S.A + m : nullptr;
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int m = m0 + 16 * q + (p >> 3);
+            arow[q] = m < P.M ? S.A + ixd(S.Am, m) : nullptr;
+          }
+          mrow = m0 + p < P.M ? S.A + ixd(S.Am, m0 + p) : nullptr;
+        }
+        op_enter(cb, S.B, S.Bn, S.Bk, n0 + rowB, P.N, ld.kt);
+      }
+      char* st = ring + slot * SM::STAGE;
+      const uint32_t dA = smem_u32(st), dB = dA + SM::A_BYTES;
+      const int kt = ld.kt, khi = ld.khi;
+      int kq = kt / a_d, kr = kt % a_d;   // k map position of the tile start
+      if (!a_mm) {
+        const bool lin = kr + TC_K <= a_d;
+        if (a_vec && lin && ((kt & 3) == 0) && kt + TC_K <= khi) {
+          // 16-byte copies: a warp covers 4 rows x 128 contiguous bytes
+          const int c = p & 7;
+          const long long ko = (long long)kq * a_s1 + (long long)(kr + 4 * c);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int r = 16 * q + (p >> 3);
+            cp_async16(dA + km_off(r, c), arow[q] ? arow[q] + ko : S.A, arow[q] != nullptr);
+          }
+        } else {
+          // 4-byte copies, one row per thread
+          int q2 = kq, r2 = kr;
+#pragma unroll 1
+          for (int j = 0; j < TC_K; ++j) {
+            const bool v = mrow && kt + j < khi;
+            cp_async4(dA + km_off(p, j >> 2) + (j & 3) * 4, v ? mrow + (long long)q2 * a_s1 + (long long)r2 * a_s2 : S.A,
+                      v);
+            kstep(q2, r2, a_d, 1);
+          }
+        }
+      } else if (a_vec) {
+        // 16-byte copies of 4 consecutive m: thread p takes m chunk p % 32 of k rows
+        // 4 q + p / 32; a warp covers 512 contiguous bytes of one k row
+        int q2 = kq, r2 = kr;
+        kstep(q2, r2, a_d, p >> 5);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int kk = 4 * q + (p >> 5);
+          const bool v = mrow && kt + kk < khi;
+          cp_async16(dA + kk * 512 + (p & 31) * 16, v ? mrow + (long long)q2 * a_s1 + (long long)r2 * a_s2 : S.A, v);
+          kstep(q2, r2, a_d, 4);
+        }
+      } else {
+        // 4-byte copies, lanes along m
+        int q2 = kq, r2 = kr;
+#pragma unroll 1
+        for (int j = 0; j < TC_K; ++j) {
+          const bool v = mrow && kt + j < khi;
+          cp_async4(dA + j * 512 + p * 4, v ? mrow + (long long)q2 * a_s1 + (long long)r2 * a_s2 : S.A, v);
+          kstep(q2, r2, a_d, 1);
+        }
+      }
+      issue_operand<KWB, NT>(cb, S.B, kt, khi, kbegB, rowB, S.b_vec4 != 0, dB);
+      // the stage's full barrier completes when this thread's copies (and its earlier
+      // ones) have landed; nothing the copies write is read by the tensor core directly
+      asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&full[slot])) : "memory");
+      const int seg_before = ld.seg;
+      ld.kt += TC_K;
+      advance_to_valid(ld);
+      if (ld.have && ld.seg == seg_before) op_step(cb, TC_K);
     }
-    issue_tile((it + 1) % SM::RING);
-    asm volatile("cp.async.wait_group 1;" ::: "memory");   // this thread's copies of tile `it`
-    {
-      // split the elements this thread copied: lo = raw - tf32(raw)
-      const char* raw = ring + (it % SM::RING) * SM::RAW;
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  } else {
+    // ---- converters: thread (quadrant w, lane) owns output row m = 32 w + lane; it splits
+    // its 32 A values of the stage into hi / lo and stores them to its TMEM lane; the B
+    // residuals are split cooperatively in shared memory.  One thread then issues
+    // hi*hi + hi*lo + lo*hi for the stage's four K=8 steps (A from TMEM, B from shared
+    // memory) and commits them to the stage's empty barrier.
+    const int c = tid - TC_PRODUCERS;
+    const int quad = warp - TC_PRODUCERS / 32;
+    const int m = 32 * quad + lane;
+    const uint32_t tlane = tmem + ((uint32_t)(32 * quad) << 16);
+    Cursor cv{0, 0, 0, 0, false};  // the same walk as the producers: the A layout of each stage
+    advance_to_valid(cv);
+#pragma unroll 1
+    for (int it = 0; it < ntiles; ++it) {
+      const bool mm = a_is_mm(g.sg[P.seg0 + cv.seg]);
+      cv.kt += TC_K;
+      advance_to_valid(cv);
+      const int slot = it % SM::RING;
+      char* st = ring + slot * SM::STAGE;
+      ok = mbar_wait(smem_u32(&full[slot]), (it / SM::RING) & 1) && ok;
+      const uint32_t acol = (uint32_t)(NT + 64 * slot);
+      // two halves of 16 k values: split, then store hi and lo to this thread's TMEM lane
 #pragma unroll
-      for (int q = 0; q < KWA / 4; ++q) {
-        const uint32_t off = tile_off<TC_M>(rowA, kbegA + 4 * q);
-        const float4 v = *reinterpret_cast<const float4*>(raw + off);
-        float4 l;
-        l.x = v.x - tf32_hi(v.x); l.y = v.y - tf32_hi(v.y); l.z = v.z - tf32_hi(v.z); l.w = v.w - tf32_hi(v.w);
-        *reinterpret_cast<float4*>(lo_buf + off) = l;
-      }
+      for (int h = 0; h < 2; ++h) {
+        uint32_t hi[16], lo[16];
+        if (mm) {
+          const float* a = reinterpret_cast<const float*>(st);
 #pragma unroll
-      for (int q = 0; q < KWB / 4; ++q) {
-        const uint32_t off = SM::A_BYTES + tile_off<NT>(rowB, kbegB + 4 * q);
-        const float4 v = *reinterpret_cast<const float4*>(raw + off);
-        float4 l;
-        l.x = v.x - tf32_hi(v.x); l.y = v.y - tf32_hi(v.y); l.z = v.z - tf32_hi(v.z); l.w = v.w - tf32_hi(v.w);
-        *reinterpret_cast<float4*>(lo_buf + off) = l;
-      }
-    }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-    __syncthreads();
-    if (tid == 0) {
-      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t a_hi = smem_u32(ring + (it % SM::RING) * SM::RAW), b_hi = a_hi + SM::A_BYTES;
-      const uint32_t a_lo = smem_u32(lo_buf), b_lo = a_lo + SM::A_BYTES;
+          for (int k = 0; k < 16; ++k) {
+            const float v = a[(16 * h + k) * 128 + m];
+            const float t = tf32_hi(v);
+            hi[k] = __float_as_uint(t);
+            lo[k] = __float_as_uint(v - t);
+          }
+        } else {
 #pragma unroll
-      for (int ks = 0; ks < TC_K / 8; ++ks) {
-        // one K=8 step spans two 4-wide k columns
-        const uint32_t ka = ks * 2 * (TC_M * 16), kbo = ks * 2 * (NT * 16);
-        const uint64_t dah = smem_desc<TC_M>(a_hi + ka), dal = smem_desc<TC_M>(a_lo + ka);
-        const uint64_t dbh = smem_desc<NT>(b_hi + kbo), dbl = smem_desc<NT>(b_lo + kbo);
-        const uint32_t acc0 = (it > 0 || ks > 0) ? 1u : 0u;
+          for (int cc = 0; cc < 4; ++cc) {
+            const float4 v = *reinterpret_cast<const float4*>(st + km_off(m, 4 * h + cc));
+            const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float t = tf32_hi(vv[e]);
+              hi[4 * cc + e] = __float_as_uint(t);
+              lo[4 * cc + e] = __float_as_uint(vv[e] - t);
+            }
+          }
+        }
         asm volatile(
-            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-            "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
-            "l"(dah), "l"(dbh), "r"(IDESC), "r"(acc0));
+            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+                tlane + acol + 16u * h),
+            "r"(hi[0]), "r"(hi[1]), "r"(hi[2]), "r"(hi[3]), "r"(hi[4]), "r"(hi[5]), "r"(hi[6]), "r"(hi[7]),
+            "r"(hi[8]), "r"(hi[9]), "r"(hi[10]), "r"(hi[11]), "r"(hi[12]), "r"(hi[13]), "r"(hi[14]), "r"(hi[15])
+            : "memory");
         asm volatile(
-            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-            "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
-            "l"(dah), "l"(dbl), "r"(IDESC), "r"(1u));
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-            "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
-            "l"(dal), "l"(dbh), "r"(IDESC), "r"(1u));
+            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+                tlane + acol + 32u + 16u * h),
+            "r"(lo[0]), "r"(lo[1]), "r"(lo[2]), "r"(lo[3]), "r"(lo[4]), "r"(lo[5]), "r"(lo[6]), "r"(lo[7]),
+            "r"(lo[8]), "r"(lo[9]), "r"(lo[10]), "r"(lo[11]), "r"(lo[12]), "r"(lo[13]), "r"(lo[14]), "r"(lo[15])
+            : "memory");
       }
-      asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                       smem_u32(&bars[0]))
-                   : "memory");
+      // B split in place (layout-agnostic, elementwise): raw -> hi, plus the residual lo.
+      // Every value the tensor core reads from shared memory is thus written by a
+      // converter thread, which orders it before the MMAs with its own proxy fence.
+      char* braw = st + SM::A_BYTES;
+      char* blo = st + SM::A_BYTES + SM::B_BYTES;
+#pragma unroll
+      for (int q = c; q < SM::B_BYTES / 16; q += TC_CONVERTERS) {
+        const float4 v = *reinterpret_cast<const float4*>(braw + q * 16);
+        float4 h, l;
+        h.x = tf32_hi(v.x); h.y = tf32_hi(v.y); h.z = tf32_hi(v.z); h.w = tf32_hi(v.w);
+        l.x = v.x - h.x; l.y = v.y - h.y; l.z = v.z - h.z; l.w = v.w - h.w;
+        *reinterpret_cast<float4*>(braw + q * 16) = h;
+        *reinterpret_cast<float4*>(blo + q * 16) = l;
+      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      asm volatile("bar.sync 1, %0;" ::"n"(TC_CONVERTERS) : "memory");
+      if (c == 0) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t b_hi = smem_u32(braw), b_lo = smem_u32(blo);
+#pragma unroll
+        for (int ks = 0; ks < TC_K / 8; ++ks) {
+          // one K=8 step: 8 TMEM columns of A, two 4-wide k columns of B
+          const uint32_t ahi = tmem + acol + 8 * ks, alo = ahi + 32;
+          const uint32_t kbo = ks * 2 * (NT * 16);
+          const uint64_t dbh = smem_desc<NT>(b_hi + kbo), dbl = smem_desc<NT>(b_lo + kbo);
+          const uint32_t acc0 = (it > 0 || ks > 0) ? 1u : 0u;
+          asm volatile(
+              "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+              "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem),
+              "r"(ahi), "l"(dbh), "r"(IDESC), "r"(acc0));
+          asm volatile(
+              "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+              "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem),
+              "r"(ahi), "l"(dbl), "r"(IDESC), "r"(1u));
+          asm volatile(
+              "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+              "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem),
+              "r"(alo), "l"(dbh), "r"(IDESC), "r"(1u));
+        }
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                         smem_u32(&empty[slot]))
+                     : "memory");
+      }
     }
   }
-  asm volatile("cp.async.wait_group 0;" ::: "memory");
-  // wait for the last commit (tcgen05 operations complete in issue order)
-  if (it > 0) ok = mbar_wait(smem_u32(&bars[0]), phase) && ok;
+  // the last commit completes after every MMA of the tile (tcgen05 operations complete
+  // in issue order)
+  if (ntiles > 0) {
+    const int j = ntiles - 1;
+    ok = mbar_wait(smem_u32(&empty[j % SM::RING]), (j / SM::RING) & 1) && ok;
+  }
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const int it = ntiles;
 
   // epilogue.  TMEM lane r holds output row m0 + r; warp w may read lane quadrant w % 4
   // and takes the column half w / 4 of every 64-column slice.  Values pass through
@@ -334,7 +487,7 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
   // consecutive columns of one row; row and column offsets of the output map are
   // tabulated once.
   float* ep = reinterpret_cast<float*>(ring);            // all MMAs are complete here
-  long long* rowoff = reinterpret_cast<long long*>(lo_buf);
+  long long* rowoff = reinterpret_cast<long long*>(ring + 65536);
   long long* coloff = rowoff + TC_M;
   __syncthreads();
   for (int t = tid; t < TC_M; t += TC_THREADS) {
@@ -388,7 +541,7 @@ __global__ void __launch_bounds__(TC_THREADS) k_gemm_tc(const __grid_constant__ 
   __syncthreads();
   if (warp == 0) {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(NT));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TcSmem<NT>::TMEM_COLS));
   }
   if (!ok && tid == 0 && err) atomicExch(err, 1);
 }
