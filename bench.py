@@ -108,7 +108,8 @@ def flop_model(plan):
         f["state"] += 2 * ci * (nnz + K * ro)              # eq. 32 coupling + eq. 33 outer product
         f["recv"] += 2 * ci * (2 * nnz + 2 * K * ro)       # coupling, phi_bar, T_bar, Y_bar
         f["src"] += 2 * co * (nnz + K * ri)                # adjoint coupling + source state
-        f["gemm_node"] += 2 * K * ci * co * (2 * ro + 2 * ri)  # S A, m_bar A^T, X A^T, x^T X
+        # S A, m_bar A^T, S^T m_bar (receiver side); X A^T, x^T X (source side)
+        f["gemm_node"] += 2 * K * ci * co * (3 * ro + 2 * ri)
         # fp32 operand bytes of the five channel contractions of a forward+backward step:
         # m = S A (read S, write m), S_bar = m_bar A^T (read m_bar, write S_bar),
         # A_bar += S^T m_bar (read S, m_bar), x_bar = X A^T (read X, write x_bar),
@@ -255,7 +256,8 @@ def run_native(args):
 
     # live roofline of every kernel category (CUDA events over the timed region)
     fm = flop_model(plan)
-    algo = {"uvw_receiver_state": fm["state"] * E, "uvw_receiver_backward": fm["recv"] * E,
+    # the receiver state runs in the forward pass and again in the backward pass
+    algo = {"uvw_receiver_state": 2 * fm["state"] * E, "uvw_receiver_backward": fm["recv"] * E,
             "uvw_source_state": fm["src"] * E, "channel_gemm": fm["gemm_node"] * N}
     peaks = measured_peaks()
     tc_peak = peaks["bf16"] * TF32_PER_BF16 / SPLIT_MMAS

@@ -503,25 +503,44 @@ tpconv_status check_ws(const Layout& L, void* ws, size_t ws_bytes) {
   return TPCONV_OK;
 }
 
+// A grouped GEMM under construction.  Problems are collected into a GemmBatch; when the
+// next problem would not fit (problem or segment capacity), the batch collected so far is
+// launched and a new one started, so any number of problems is accepted.
 struct Batch {
   GemmBatch g{};
-  Batch(int splits, int accumulate, float* partial) {
+  cudaStream_t st;
+  float* auto_part;  // split-K scratch for automatic splitting (nullptr: never split automatically)
+  cudaError_t err = cudaSuccess;
+  Batch(cudaStream_t s, int splits, int accumulate, float* partial, float* auto_split_part = nullptr)
+      : st(s), auto_part(auto_split_part) {
     g.splits = splits;
     g.accumulate = accumulate;
     g.partial = partial;
   }
-  // Use split-K when the output tiles alone would leave SMs idle (needs `partial`).
-  cudaError_t launch(cudaStream_t st, float* part = nullptr) {
-    if (g.splits == 1 && part) {
-      const int tiles = gemm_tiles(g);
-      if (tiles > 0 && tiles < 2 * 148) {
-        g.splits = std::min(kSplits, (2 * 148 + tiles - 1) / tiles);
-        g.partial = part;
+  // Launch the collected problems.  With automatic splitting, split-K is used when the
+  // output tiles alone would leave SMs idle.
+  void flush() {
+    if (g.n_problems == 0) return;
+    if (err == cudaSuccess) {
+      GemmBatch h = g;
+      if (h.splits == 1 && auto_part) {
+        const int tiles = gemm_tiles(h);
+        if (tiles > 0 && tiles < 2 * 148) {
+          h.splits = std::min(kSplits, (2 * 148 + tiles - 1) / tiles);
+          h.partial = auto_part;
+        }
       }
+      err = launch_gemm(h, st);
     }
-    return launch_gemm(g, st);
+    g.n_problems = 0;
+    g.n_segs = 0;
   }
-  void problem(float* C, Idx2 Cm, Idx2 Cn, int M, int N) {
+  cudaError_t finish() {
+    flush();
+    return err;
+  }
+  void problem(float* C, Idx2 Cm, Idx2 Cn, int M, int N, int nseg) {
+    if (g.n_problems + 1 > MAX_GEMM_PROBLEMS || g.n_segs + nseg > MAX_GEMM_SEGS) flush();
     GemmProblem& p = g.pr[g.n_problems++];
     p.C = C; p.Cm = Cm; p.Cn = Cn; p.M = M; p.N = N;
     p.seg0 = g.n_segs; p.nseg = 0; p.Ktot = 0;
@@ -544,18 +563,24 @@ struct Batch {
   }
 };
 
+int paths_into(const tpconv_plan* P, int block, bool out_side) {
+  int n = 0;
+  for (const PathH& p : P->paths) n += (out_side ? p.b_out : p.b_in) == block;
+  return n;
+}
+
 // m_g[(i,mo), w] = sum_{pi in g} sum_{q,u} S_pi[(i,mo),(q,u)] A_pi[(q,u), w]   (eqs. 34-35),
 // optionally + sum_pi S2_pi A2_pi (eq. 37: dm = dS A + S dA)
 cudaError_t gemm_state_times_A(const tpconv_plan* P, const float* S, const float* W, const float* S2,
                                const float* W2, float* out, int n0, int cn, float* part, cudaStream_t st) {
-  Batch b(1, 0, nullptr);
+  Batch b(st, 1, 0, nullptr, part);
   for (int bo = 0; bo < (int)P->out.size(); ++bo) {
     const Block& B = P->out[bo];
     const int RO = 2 * B.l + 1;
-    bool any = false;
-    for (const PathH& p : P->paths) any = any || p.b_out == bo;
-    if (!any) continue;
-    b.problem(out + (long long)n0 * P->dim_out + B.offset, idx2(RO, P->dim_out, B.mul), idx1(1), cn * RO, B.mul);
+    const int np = paths_into(P, bo, true);
+    if (np == 0) continue;
+    b.problem(out + (long long)n0 * P->dim_out + B.offset, idx2(RO, P->dim_out, B.mul), idx1(1), cn * RO, B.mul,
+              np * ((S ? 1 : 0) + (S2 ? 1 : 0)));
     for (const PathH& p : P->paths) {
       if (p.b_out != bo) continue;
       const Idx2 Am = idx2(RO, P->dev.state_per_node, (long long)P->K * p.c_in);
@@ -564,35 +589,35 @@ cudaError_t gemm_state_times_A(const tpconv_plan* P, const float* S, const float
       if (S2) b.seg(S2 + p.st_off, Am, idx1(1), W2 + p.w_off, Bk, idx1(1), P->K * p.c_in);
     }
   }
-  return b.launch(st, part);
+  return b.finish();
 }
 
 // S_bar_pi[(i,mo),(q,u)] = sum_w m_bar[(i,mo), w] A_pi[(q,u), w]        (eq. 36)
 cudaError_t gemm_sbar(const tpconv_plan* P, const float* gout, const float* W, float* Sbar, int n0,
                       int cn, cudaStream_t st) {
-  Batch b(1, 0, nullptr);
+  Batch b(st, 1, 0, nullptr);
   for (const PathH& p : P->paths) {
     const int RO = 2 * p.l_out + 1;
     b.problem(Sbar + p.st_off, idx2(RO, P->dev.state_per_node, (long long)P->K * p.c_in), idx1(1), cn * RO,
-              P->K * p.c_in);
+              P->K * p.c_in, 1);
     b.seg(gout + (long long)n0 * P->dim_out + p.out_off, idx2(RO, P->dim_out, p.c_out), idx1(1), W + p.w_off,
           idx1(1), idx2(p.c_in, P->n_w, p.c_out), p.c_out);
   }
-  return launch_gemm(b.g, st);
+  return b.finish();
 }
 
 // x_bar[(j,mi), u] = sum_{pi from block} sum_{q,w} X_pi[(j,mi),(q,w)] A_pi[(q,u), w]
 // (mirrored eq. 21), optionally + X2 A2^T (eq. 30 with A_dot)
 cudaError_t gemm_xbar(const tpconv_plan* P, const float* X, const float* W, const float* X2, const float* W2,
                       float* gx, int n0, int cn, float* part, cudaStream_t st) {
-  Batch b(1, 0, nullptr);
+  Batch b(st, 1, 0, nullptr, part);
   for (int bi = 0; bi < (int)P->in.size(); ++bi) {
     const Block& B = P->in[bi];
     const int RI = 2 * B.l + 1;
-    bool any = false;
-    for (const PathH& p : P->paths) any = any || p.b_in == bi;
-    if (!any) continue;
-    b.problem(gx + (long long)n0 * P->dim_in + B.offset, idx2(RI, P->dim_in, B.mul), idx1(1), cn * RI, B.mul);
+    const int np = paths_into(P, bi, false);
+    if (np == 0) continue;
+    b.problem(gx + (long long)n0 * P->dim_in + B.offset, idx2(RI, P->dim_in, B.mul), idx1(1), cn * RI, B.mul,
+              np * ((X ? 1 : 0) + (X2 ? 1 : 0)));
     for (const PathH& p : P->paths) {
       if (p.b_in != bi) continue;
       const Idx2 Am = idx2(RI, P->dev.xstate_per_node, (long long)P->K * p.c_out);
@@ -601,34 +626,39 @@ cudaError_t gemm_xbar(const tpconv_plan* P, const float* X, const float* W, cons
       if (X2) b.seg(X2 + p.xst_off, Am, idx1(1), W2 + p.w_off, Bk, idx1(p.c_out), P->K * p.c_out);
     }
   }
-  return b.launch(st, part);
+  return b.finish();
 }
 
 // A_bar_pi[(q,u), w] (+)= sum_{(j,mi)} x[(j,mi), u] X_pi[(j,mi),(q,w)]     (mirrored eq. 19)
-// computed as its transpose, rows (q,w) and columns u, so the wide side fills the MMA rows
+// computed as its transpose, rows (q,w) and columns u, so the wide side fills the MMA rows.
+// The sum over (j, mi) is one segment per mi, so that every k map is a single stride
+// (the node) and operand tiles never cross a node boundary.
 cudaError_t gemm_abar_src(const tpconv_plan* P, const float* x, const float* X, float* gW, int n0, int cn,
                           int accumulate, float* part, cudaStream_t st) {
-  Batch b(kSplits, accumulate, part);
+  Batch b(st, kSplits, accumulate, part);
   for (const PathH& p : P->paths) {
     const int RI = 2 * p.l_in + 1;
-    b.problem(gW + p.w_off, idx2(p.c_out, P->n_w, 1), idx1(p.c_out), P->K * p.c_out, p.c_in);
-    b.seg(X + p.xst_off, idx1(1), idx2(RI, P->dev.xstate_per_node, (long long)P->K * p.c_out),
-          x + (long long)n0 * P->dim_in + p.in_off, idx2(RI, P->dim_in, p.c_in), idx1(1), cn * RI);
+    b.problem(gW + p.w_off, idx2(p.c_out, P->n_w, 1), idx1(p.c_out), P->K * p.c_out, p.c_in, RI);
+    for (int mi = 0; mi < RI; ++mi)
+      b.seg(X + p.xst_off + (long long)mi * P->K * p.c_out, idx1(1), idx1(P->dev.xstate_per_node),
+            x + (long long)n0 * P->dim_in + p.in_off + (long long)mi * p.c_in, idx1(P->dim_in), idx1(1), cn);
   }
-  return launch_gemm(b.g, st);
+  return b.finish();
 }
 
-// A_bar_pi[(q,u), w] (+)= sum_{(i,mo)} dS_pi[(i,mo),(q,u)] m_bar[(i,mo), w]   (eq. 39)
+// A_bar_pi[(q,u), w] (+)= sum_{(i,mo)} dS_pi[(i,mo),(q,u)] m_bar[(i,mo), w]   (eq. 39),
+// one segment per mo (single-stride k maps, as above)
 cudaError_t gemm_abar_recv(const tpconv_plan* P, const float* S, const float* gout, float* gW, int n0, int cn,
                            int accumulate, float* part, cudaStream_t st) {
-  Batch b(kSplits, accumulate, part);
+  Batch b(st, kSplits, accumulate, part);
   for (const PathH& p : P->paths) {
     const int RO = 2 * p.l_out + 1;
-    b.problem(gW + p.w_off, idx2(p.c_in, P->n_w, p.c_out), idx1(1), P->K * p.c_in, p.c_out);
-    b.seg(S + p.st_off, idx1(1), idx2(RO, P->dev.state_per_node, (long long)P->K * p.c_in),
-          gout + (long long)n0 * P->dim_out + p.out_off, idx2(RO, P->dim_out, p.c_out), idx1(1), cn * RO);
+    b.problem(gW + p.w_off, idx2(p.c_in, P->n_w, p.c_out), idx1(1), P->K * p.c_in, p.c_out, RO);
+    for (int mo = 0; mo < RO; ++mo)
+      b.seg(S + p.st_off + (long long)mo * P->K * p.c_in, idx1(1), idx1(P->dev.state_per_node),
+            gout + (long long)n0 * P->dim_out + p.out_off + (long long)mo * p.c_out, idx1(P->dim_out), idx1(1), cn);
   }
-  return launch_gemm(b.g, st);
+  return b.finish();
 }
 
 bool every_block_reached(const tpconv_plan* P, bool out_side) {

@@ -195,6 +195,27 @@ def test_general_parities_forward_backward(torch):
         assert rel_l2(a.cpu().numpy(), b) <= TOL
 
 
+def test_many_paths_overflow_one_gemm_batch(torch):
+    """34 paths whose weight-gradient contractions need more segments (one per m
+    component, 134 in all) than one grouped launch holds: the library splits them over
+    several launches."""
+    from equivariant_gnn_tensor_dst_b200 import binding
+    irr = "8x0e+8x1o+8x2e+8x3o+8x0o+8x1e"
+    c = workloads.Config(9, "many paths", 60, 10, irr, 3, irr, "uvw", "bessel", 8, 4.0)
+    p = Problem(None, config=c)
+    lp = lib_plan(c)
+    assert len(lp.paths()) == 34
+    assert sum(2 * q["l_out"] + 1 for q in lp.paths()) > 128
+    d = _dev(p)
+    out = binding.tpconv_forward(lp, d["x"], d["pos"], d["row_ptr"], d["src"], d["W"])
+    assert rel_l2(out.cpu().numpy(), conv.forward(p.plan, p.x, p.pos, p.row_ptr, p.src, p.W)) <= TOL
+    v = _graph_views(d, p.N)
+    gx, gp, gw = binding.tpconv_backward(lp, d["x"], d["pos"], d["row_ptr"], d["src"], *v, d["W"], d["gout"])
+    rx, rp, rw = conv.backward(p.plan, p.x, p.pos, p.row_ptr, p.src, p.W, p.gout)
+    for a, b in ((gx, rx), (gp, rp), (gw, rw)):
+        assert rel_l2(a.cpu().numpy(), b) <= TOL
+
+
 # ---------------------------------------------------------------------------
 # edge cases
 # ---------------------------------------------------------------------------
