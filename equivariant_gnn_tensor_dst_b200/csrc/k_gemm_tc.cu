@@ -12,19 +12,20 @@
 // decomposition of Ootomo and Yokota, 2022), which keeps the relative error near
 // 2^-21 instead of TF32's 2^-11.
 //
-// Structure: one CTA of 256 threads per 128 x NT output tile (NT = 64 or 128) and
-// split-K slice, two CTAs per SM, warp-specialised around a ring of shared-memory stages
-// of 32 k values:
+// Structure: one CTA of 288 threads per 128 x NT output tile (NT = 64 or 128) and
+// split-K slice, two CTAs per SM, warp-specialised around two rings: raw stages of 32 k
+// values, and operand slots (TMEM columns for A, shared memory for B):
 //   - warps 0-3 (producers) copy the raw fp32 A and B tiles of a stage from global memory
 //     with cp.async, through the same two-level affine index maps as the rest of the
 //     library (ir_mul node rows, weight columns and workspace states are read in place);
 //     the copies arrive on the stage's "full" mbarrier when they land;
-//   - warps 4-7 (converters) split the stage: thread (quadrant w, lane) owns output row
-//     32 w + lane and writes hi(A) and lo(A) of its row into its TMEM lane (tcgen05.st);
-//     B is split in place in shared memory (raw -> hi, plus a lo copy); one converter
-//     thread then issues hi*hi + hi*lo + lo*hi (A from TMEM, B from shared memory) into
-//     the fp32 TMEM accumulator and commits them to the stage's "empty" mbarrier, which
-//     the producers wait on before refilling the stage.
+//   - warps 4-7 (converters) split a stage into an operand slot: thread (quadrant w,
+//     lane) owns output row 32 w + lane and writes hi(A) and lo(A) of its row into its
+//     TMEM lane (tcgen05.st); B hi and B lo are written to shared memory.  The raw stage
+//     is released at once ("empty"), the slot handed to the MMA warp ("conv");
+//   - warp 8 (one thread) issues hi*hi + hi*lo + lo*hi (A from TMEM, B from shared
+//     memory) into the fp32 TMEM accumulator and commits them to the slot's "mdone"
+//     mbarrier, which frees the slot for the converters.
 // The epilogue reads the accumulator with tcgen05.ld (one TMEM lane = one output row) and
 // writes C (or the split-K partial) through the output map.  Every mbarrier wait is
 // bounded; a wait that gives up sets *err and the kernel still releases its TMEM.
@@ -38,7 +39,7 @@ namespace {
 
 constexpr int TC_M = 128;
 constexpr int TC_K = 32;           // k elements per stage (8 core-matrix columns)
-constexpr int TC_THREADS = 256;
+constexpr int TC_THREADS = 288;   // 4 producer warps, 4 converter warps, 1 MMA warp
 constexpr unsigned kWaitLimit = 1u << 20;
 
 __device__ __forceinline__ long long ixd(const Idx2& f, int i) {
@@ -78,6 +79,11 @@ __host__ __device__ constexpr uint32_t instr_desc() {
   return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(NT >> 3) << 17) | ((uint32_t)(TC_M >> 4) << 24);
 }
 
+// Bounded wait for the completion of an mbarrier phase.  SLEEP_NS > 0 backs off between
+// polls, for waits off the critical path (a producer ahead of its consumers, threads done
+// with their part of the tile), so that spinning threads do not take issue slots from
+// the warps doing the work.
+template <int SLEEP_NS = 0>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   for (unsigned it = 0; it < kWaitLimit; ++it) {
     uint32_t done;
@@ -89,6 +95,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
         : "r"(bar), "r"(parity)
         : "memory");
     if (done) return true;
+    if (SLEEP_NS > 0) __nanosleep(SLEEP_NS);
   }
   return false;
 }
@@ -160,26 +167,32 @@ __device__ __forceinline__ void issue_operand(const OpCursor& c, const float* sa
   }
 }
 
-// Shared-memory plan: RING stages, each [A raw | B raw | B lo], 1 KB aligned, then the
-// mbarriers and the TMEM address.
-//   A raw (128 x 32 fp32) is read back only by the converter warps, one output row per
+// Shared-memory plan (1 KB aligned): a ring of RR raw stages [A raw | B raw], a ring of
+// NS operand slots [B hi | B lo], then the mbarriers and the TMEM address.
+//   A raw (128 x 32 fp32) is read only by the converter warps, one output row per
 //   thread, so its layout is chosen for conflict-free reads: k-contiguous operands are
 //   stored row-major with the 16-byte chunks of row r XOR-swizzled by r % 8 ("KM"),
 //   m-contiguous operands k-major, [k][128 m] ("MM").
-//   B raw / B lo (NT x 32) are in the tensor core's K-major no-swizzle core-matrix
-//   layout (tile_off); B raw doubles as the "hi" operand.
-// TMEM: columns [0, NT) the fp32 accumulator; stage s holds A hi in columns
+//   B raw, B hi and B lo (NT x 32) are in the tensor core's K-major no-swizzle
+//   core-matrix layout (tile_off).
+// A raw stage is released as soon as the converters have read it; an operand slot (and
+// its TMEM columns) when the MMAs that read it have completed.  The copies therefore run
+// ahead of the tensor core by up to RR stages regardless of the MMA latency.
+// TMEM: columns [0, NT) the fp32 accumulator; operand slot s holds A hi in columns
 // NT + 64 s + [0, 32) and A lo in NT + 64 s + [32, 64).
 template <int NT>
 struct TcSmem {
   static constexpr int A_BYTES = TC_M * TC_K * 4;
   static constexpr int B_BYTES = NT * TC_K * 4;
-  static constexpr int STAGE = A_BYTES + 2 * B_BYTES;
-  static constexpr int RING = NT == 64 ? 3 : 2;       // stages (two CTAs share an SM)
-  static constexpr int BAR_OFF = RING * STAGE;
+  static constexpr int RAW = A_BYTES + B_BYTES;
+  static constexpr int RR = NT == 64 ? 3 : 2;         // raw stages (two CTAs share an SM)
+  static constexpr int NS = NT == 64 ? 2 : 1;         // operand slots
+  static constexpr int OPS_OFF = RR * RAW;
+  static constexpr int BAR_OFF = OPS_OFF + NS * 2 * B_BYTES;
   static constexpr int TOTAL = BAR_OFF + 128 + 1024;  // barriers, TMEM address; alignment slack
   static constexpr int TMEM_COLS = 256;
-  static_assert(NT + 64 * RING <= TMEM_COLS, "TMEM columns");
+  static_assert(NT + 64 * NS <= TMEM_COLS, "TMEM columns");
+  static_assert(2 * (RR + NS) * 8 + 4 <= 128, "barrier area");
 };
 
 constexpr int TC_PRODUCERS = 128;  // warps 0-3 copy operand tiles
@@ -210,9 +223,12 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
   char* smem = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   using SM = TcSmem<NT>;
   char* ring = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::BAR_OFF);  // stage copied (TC_PRODUCERS arrivals)
-  uint64_t* empty = full + SM::RING;                  // stage consumed by the MMAs (tcgen05.commit)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(empty + SM::RING);
+  char* ops = smem + SM::OPS_OFF;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::BAR_OFF);  // raw stage copied (TC_PRODUCERS arrivals)
+  uint64_t* empty = full + SM::RR;                    // raw stage read (TC_CONVERTERS arrivals)
+  uint64_t* conv = empty + SM::RR;                    // operand slot filled (TC_CONVERTERS arrivals)
+  uint64_t* mdone = conv + SM::NS;                    // operand slot consumed by the MMAs (tcgen05.commit)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdone + SM::NS);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // locate (problem, m tile, n tile)
@@ -228,9 +244,13 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
   const int kb = split * kper, ke = min(P.Ktot, kb + kper);
 
   if (tid == 0) {
-    for (int i = 0; i < SM::RING; ++i) {
+    for (int i = 0; i < SM::RR; ++i) {
       mbar_init(smem_u32(&full[i]), TC_PRODUCERS);
-      mbar_init(smem_u32(&empty[i]), 1);
+      mbar_init(smem_u32(&empty[i]), TC_CONVERTERS);
+    }
+    for (int i = 0; i < SM::NS; ++i) {
+      mbar_init(smem_u32(&conv[i]), TC_CONVERTERS);
+      mbar_init(smem_u32(&mdone[i]), 1);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -271,8 +291,8 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
   }
 
   if (warp < TC_PRODUCERS / 32) {
-    // ---- producers: copy stage `it` once the MMAs of stage it - RING have released it;
-    // up to RING stages are in flight
+    // ---- producers: copy stage `it` once the converters have read stage it - RR;
+    // up to RR stages are in flight
     const int p = tid;
     const int rowB = p % NT, kbegB = (p / NT) * KWB;
     Cursor ld{0, 0, 0, 0, false};
@@ -286,8 +306,8 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
     advance_to_valid(ld);
 #pragma unroll 1
     for (int it = 0; it < ntiles; ++it) {
-      const int slot = it % SM::RING;
-      if (it >= SM::RING) ok = mbar_wait(smem_u32(&empty[slot]), ((it / SM::RING) - 1) & 1) && ok;
+      const int slot = it % SM::RR;
+      if (it >= SM::RR) ok = mbar_wait<64>(smem_u32(&empty[slot]), ((it / SM::RR) - 1) & 1) && ok;
       const GemmSeg& S = g.sg[P.seg0 + ld.seg];
       if (ld.seg != cur_seg) {  // entering a segment: layout, row offsets, k map
         cur_seg = ld.seg;
@@ -307,7 +327,7 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
         }
         op_enter(cb, S.B, S.Bn, S.Bk, n0 + rowB, P.N, ld.kt);
       }
-      char* st = ring + slot * SM::STAGE;
+      char* st = ring + slot * SM::RAW;
       const uint32_t dA = smem_u32(st), dB = dA + SM::A_BYTES;
       const int kt = ld.kt, khi = ld.khi;
       int kq = kt / a_d, kr = kt % a_d;   // k map position of the tile start
@@ -365,12 +385,11 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
       if (ld.have && ld.seg == seg_before) op_step(cb, TC_K);
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
-  } else {
+  } else if (warp < (TC_PRODUCERS + TC_CONVERTERS) / 32) {
     // ---- converters: thread (quadrant w, lane) owns output row m = 32 w + lane; it splits
     // its 32 A values of the stage into hi / lo and stores them to its TMEM lane; the B
-    // residuals are split cooperatively in shared memory.  One thread then issues
-    // hi*hi + hi*lo + lo*hi for the stage's four K=8 steps (A from TMEM, B from shared
-    // memory) and commits them to the stage's empty barrier.
+    // residuals are split cooperatively in shared memory; then the stage is handed to the
+    // MMA warp through its conv barrier.
     const int c = tid - TC_PRODUCERS;
     const int quad = warp - TC_PRODUCERS / 32;
     const int m = 32 * quad + lane;
@@ -382,10 +401,13 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
       const bool mm = a_is_mm(g.sg[P.seg0 + cv.seg]);
       cv.kt += TC_K;
       advance_to_valid(cv);
-      const int slot = it % SM::RING;
-      char* st = ring + slot * SM::STAGE;
-      ok = mbar_wait(smem_u32(&full[slot]), (it / SM::RING) & 1) && ok;
-      const uint32_t acol = (uint32_t)(NT + 64 * slot);
+      const int slot = it % SM::RR, os = it % SM::NS;
+      char* st = ring + slot * SM::RAW;
+      ok = mbar_wait(smem_u32(&full[slot]), (it / SM::RR) & 1) && ok;
+      // the operand slot (and its TMEM columns) is free once the MMAs of stage it - NS
+      // have completed
+      if (it >= SM::NS) ok = mbar_wait(smem_u32(&mdone[os]), ((it / SM::NS) - 1) & 1) && ok;
+      const uint32_t acol = (uint32_t)(NT + 64 * os);
       // two halves of 16 k values: split, then store hi and lo to this thread's TMEM lane
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -425,27 +447,38 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
             "r"(lo[8]), "r"(lo[9]), "r"(lo[10]), "r"(lo[11]), "r"(lo[12]), "r"(lo[13]), "r"(lo[14]), "r"(lo[15])
             : "memory");
       }
-      // B split in place (layout-agnostic, elementwise): raw -> hi, plus the residual lo.
-      // Every value the tensor core reads from shared memory is thus written by a
-      // converter thread, which orders it before the MMAs with its own proxy fence.
-      char* braw = st + SM::A_BYTES;
-      char* blo = st + SM::A_BYTES + SM::B_BYTES;
+      // B split (layout-agnostic, elementwise) from the raw stage into the operand slot
+      const char* braw = st + SM::A_BYTES;
+      char* bhi = ops + os * 2 * SM::B_BYTES;
+      char* blo = bhi + SM::B_BYTES;
 #pragma unroll
       for (int q = c; q < SM::B_BYTES / 16; q += TC_CONVERTERS) {
         const float4 v = *reinterpret_cast<const float4*>(braw + q * 16);
         float4 h, l;
         h.x = tf32_hi(v.x); h.y = tf32_hi(v.y); h.z = tf32_hi(v.z); h.w = tf32_hi(v.w);
         l.x = v.x - h.x; l.y = v.y - h.y; l.z = v.z - h.z; l.w = v.w - h.w;
-        *reinterpret_cast<float4*>(braw + q * 16) = h;
+        *reinterpret_cast<float4*>(bhi + q * 16) = h;
         *reinterpret_cast<float4*>(blo + q * 16) = l;
       }
+      // every value read from the raw stage has been used: the producers may refill it
+      mbar_arrive(smem_u32(&empty[slot]));
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-      asm volatile("bar.sync 1, %0;" ::"n"(TC_CONVERTERS) : "memory");
-      if (c == 0) {
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const uint32_t b_hi = smem_u32(braw), b_lo = smem_u32(blo);
+      mbar_arrive(smem_u32(&conv[os]));
+    }
+  } else {
+    // ---- MMA warp: hi*hi + hi*lo + lo*hi for the stage's four K=8 steps (A from TMEM,
+    // B from shared memory), committed to the slot's mdone barrier.  The whole warp runs
+    // the loop (no lane spins apart from the others); lane 0 issues.
+#pragma unroll 1
+    for (int it = 0; it < ntiles; ++it) {
+      const int os = it % SM::NS;
+      ok = mbar_wait(smem_u32(&conv[os]), (it / SM::NS) & 1) && ok;
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      if (lane == 0) {
+        const uint32_t b_hi = smem_u32(ops + os * 2 * SM::B_BYTES), b_lo = b_hi + SM::B_BYTES;
+        const uint32_t acol = (uint32_t)(NT + 64 * os);
 #pragma unroll
         for (int ks = 0; ks < TC_K / 8; ++ks) {
           // one K=8 step: 8 TMEM columns of A, two 4-wide k columns of B
@@ -467,16 +500,17 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
               "r"(alo), "l"(dbh), "r"(IDESC), "r"(1u));
         }
         asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                         smem_u32(&empty[slot]))
+                         smem_u32(&mdone[os]))
                      : "memory");
       }
+      __syncwarp();
     }
   }
   // the last commit completes after every MMA of the tile (tcgen05 operations complete
   // in issue order)
   if (ntiles > 0) {
     const int j = ntiles - 1;
-    ok = mbar_wait(smem_u32(&empty[j % SM::RING]), (j / SM::RING) & 1) && ok;
+    ok = mbar_wait<128>(smem_u32(&mdone[j % SM::NS]), (j / SM::NS) & 1) && ok;
   }
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const int it = ntiles;
@@ -500,11 +534,12 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
   }
   float* const outbase = g.splits > 1 ? g.partial + P.part_off : P.C;
   const int quad = warp & 3, half = warp >> 2;
+  const bool epi = warp < 8;                             // the MMA warp takes no part
 #pragma unroll 1
   for (int c0 = 0; c0 < NT; c0 += 64) {
     uint32_t r[32];
     const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(c0 + half * 32);
-    asm volatile(
+    if (epi) asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
         "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
@@ -513,15 +548,17 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
           "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
           "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+    if (epi) asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
     __syncthreads();  // previous slice read out of `ep`; offset tables written
     const int row = quad * 32 + lane;
+    if (epi) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) ep[row * 65 + half * 32 + j] = (it > 0) ? __uint_as_float(r[j]) : 0.f;
+      for (int j = 0; j < 32; ++j) ep[row * 65 + half * 32 + j] = (it > 0) ? __uint_as_float(r[j]) : 0.f;
+    }
     __syncthreads();
     const int ncols = min(64, NT - c0);
 #pragma unroll 4
-    for (int q = 0; q < TC_M / 8; ++q) {
+    for (int q = 0; q < (epi ? TC_M / 8 : 0); ++q) {
       const int rr = q * 8 + warp;                       // 8 warps store 8 rows per step
       const int m = m0 + rr;
       if (m >= P.M) continue;
