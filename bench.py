@@ -108,13 +108,13 @@ def flop_model(plan):
         f["state"] += 2 * ci * (nnz + K * ro)              # eq. 32 coupling + eq. 33 outer product
         f["recv"] += 2 * ci * (2 * nnz + 2 * K * ro)       # coupling, phi_bar, T_bar, Y_bar
         f["src"] += 2 * co * (nnz + K * ri)                # adjoint coupling + source state
-        # S A, m_bar A^T, S^T m_bar (receiver side); X A^T, x^T X (source side)
-        f["gemm_node"] += 2 * K * ci * co * (3 * ro + 2 * ri)
-        # fp32 operand bytes of the five channel contractions of a forward+backward step:
+        # S A, m_bar A^T (receiver side); X A^T, x^T X (source side, which also gives A_bar)
+        f["gemm_node"] += 2 * K * ci * co * (2 * ro + 2 * ri)
+        # fp32 operand bytes of the four channel contractions of a forward+backward step:
         # m = S A (read S, write m), S_bar = m_bar A^T (read m_bar, write S_bar),
-        # A_bar += S^T m_bar (read S, m_bar), x_bar = X A^T (read X, write x_bar),
-        # A_bar += x^T X (read x, X); the weights stay in L2.
-        f["gemm_node_bytes"] += 4 * (3 * ro * K * ci + 3 * ro * co + 2 * ri * K * co + 2 * ri * ci)
+        # x_bar = X A^T (read X, write x_bar), A_bar = x^T X (read x, X); the weights stay
+        # in L2.
+        f["gemm_node_bytes"] += 4 * (2 * ro * K * ci + 2 * ro * co + 2 * ri * K * co + 2 * ri * ci)
     return f
 
 
@@ -256,8 +256,7 @@ def run_native(args):
 
     # live roofline of every kernel category (CUDA events over the timed region)
     fm = flop_model(plan)
-    # the receiver state runs in the forward pass and again in the backward pass
-    algo = {"uvw_receiver_state": 2 * fm["state"] * E, "uvw_receiver_backward": fm["recv"] * E,
+    algo = {"uvw_receiver_state": fm["state"] * E, "uvw_receiver_backward": fm["recv"] * E,
             "uvw_source_state": fm["src"] * E, "channel_gemm": fm["gemm_node"] * N}
     peaks = measured_peaks()
     tc_peak = peaks["bf16"] * TF32_PER_BF16 / SPLIT_MMAS

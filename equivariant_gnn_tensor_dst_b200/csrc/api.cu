@@ -197,12 +197,15 @@ struct Layout {
   bool has_gbuf = false, has_part = false;
 };
 
+// Nodes per chunk: the most that fit the budget, then evened out over the chunks that
+// number needs (so that no chunk is left with a small remainder).
 int chunk_for(size_t budget_floats, long long fixed, long long per_node, long long N) {
   if (per_node <= 0 || N <= 0) return (int)std::max<long long>(N, 0);
   long long avail = (long long)budget_floats - fixed;
   long long c = avail > 0 ? avail / per_node : 1;
   c = std::max<long long>(1, std::min<long long>(c, N));
-  return (int)c;
+  const long long chunks = (N + c - 1) / c;
+  return (int)((N + chunks - 1) / chunks);
 }
 
 // Workspace of one pass.  The scratch budget covers the node states of a receiver (or
