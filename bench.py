@@ -37,10 +37,16 @@ FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # SM count x FP32 lanes x FM
 L2_FLUSH_BYTES = 256 << 20                          # > 126 MB L2
 TF32_PER_BF16 = 1.1 / 2.25                          # nominal dense TF32 / BF16 tensor rates
 SPLIT_MMAS = 3                                      # 3xTF32: three TF32 products per fp32 product
-# DRAM bytes per launch of each kernel category, averaged over one step of this workload
-# from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum); None when not
-# measured for the current kernels.
-TRAFFIC_BYTES_PER_LAUNCH = {}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per step of the N=4096 uvw
+# workload for each kernel category, from one ncu capture of the 2048-node case whose
+# launches have the same 1024-node chunk shape (per step: twice its launches).  Valid for
+# the kernels as captured; only reported for that workload.
+TRAFFIC_BYTES_PER_STEP = {
+    "channel_gemm": 2 * (6 * 92.80e6 + 2 * 32.93e6 + 6 * 12.70e6),
+    "uvw_receiver_backward": 4 * 96.65e6,
+    "uvw_source_state": 4 * 35.09e6,
+    "uvw_receiver_state": 4 * 34.54e6,
+}
 
 
 def measured_peaks():
@@ -287,8 +293,11 @@ def run_native(args):
                   "peak_note": "derived: 148 SMs x 128 FP32 lanes x 2 flop x 1965 MHz"}
             rl["algorithmic_per_step"] = {"flop": algo[k]}
         rl["frac"] = round(rl["achieved"] / rl["peak"], 4)
-        tb = TRAFFIC_BYTES_PER_LAUNCH.get(k)
-        rl["traffic"] = tb
+        headline = args.cfg == CFG and args.nodes is None
+        tb = TRAFFIC_BYTES_PER_STEP.get(k) if headline else None
+        rl["traffic"] = round(tb) if tb else None
+        if tb:
+            rl["traffic_note"] = "DRAM bytes per step (all launches of the category), ncu capture"
         rooflines[k] = rl
     dom = max(rooflines, key=lambda k: kern[k][0])
     roofline = dict(rooflines[dom], kernel=dom)
