@@ -107,10 +107,17 @@ def reduce_over_ranks(total_ms, edges, device=None):
 
 def flop_model(plan):
     K = plan.num_basis
-    f = dict(state=0, recv=0, src=0, gemm_node=0, gemm_node_bytes=0)
+    f = dict(state=0, recv=0, src=0, gemm_node=0, gemm_node_bytes=0, uvu_fwd=0, uvu_recv=0, uvu_gradw=0, uvu_src=0)
     for p in plan.paths():
         ri, ro = 2 * p["l_in"] + 1, 2 * p["l_out"] + 1
         nnz, ci, co = p["nnz"], p["c_in"], p["c_out"]
+        # uvu (channelwise, no state): w = phi A per channel, coupling, w * C into m (eqs. 7, 17);
+        # receiver adjoint h = m_bar . C, phi_bar, Y_bar; weight gradient phi (m_bar . C);
+        # source adjoint w * adj(C)
+        f["uvu_fwd"] += 2 * ci * (K + nnz + ro)
+        f["uvu_recv"] += 2 * ci * (2 * nnz + 2 * ro + 2 * K)
+        f["uvu_gradw"] += 2 * ci * (nnz + ro + K)
+        f["uvu_src"] += 2 * ci * (K + nnz + ro)
         f["state"] += 2 * ci * (nnz + K * ro)              # eq. 32 coupling + eq. 33 outer product
         f["recv"] += 2 * ci * (2 * nnz + 2 * K * ro)       # coupling, phi_bar, T_bar, Y_bar
         f["src"] += 2 * co * (nnz + K * ri)                # adjoint coupling + source state
@@ -263,7 +270,9 @@ def run_native(args):
     # live roofline of every kernel category (CUDA events over the timed region)
     fm = flop_model(plan)
     algo = {"uvw_receiver_state": fm["state"] * E, "uvw_receiver_backward": fm["recv"] * E,
-            "uvw_source_state": fm["src"] * E, "channel_gemm": fm["gemm_node"] * N}
+            "uvw_source_state": fm["src"] * E, "channel_gemm": fm["gemm_node"] * N,
+            "uvu_forward": fm["uvu_fwd"] * E, "uvu_receiver_backward": fm["uvu_recv"] * E,
+            "uvu_weight_gradient": fm["uvu_gradw"] * E, "uvu_source_backward": fm["uvu_src"] * E}
     peaks = measured_peaks()
     tc_peak = peaks["bf16"] * TF32_PER_BF16 / SPLIT_MMAS
     kern = {k: v for k, v in prof.items() if v[1] > 0}
@@ -299,11 +308,11 @@ def run_native(args):
         if tb:
             rl["traffic_note"] = "DRAM bytes per step (all launches of the category), ncu capture"
         rooflines[k] = rl
-    dom = max(rooflines, key=lambda k: kern[k][0])
-    roofline = dict(rooflines[dom], kernel=dom)
+    dom = max(rooflines, key=lambda k: kern[k][0]) if rooflines else None
+    roofline = dict(rooflines[dom], kernel=dom) if dom else None
     breakdown = {k: {"ms_per_step": round(v[0] / args.steps, 4), "launches_per_step": v[1] / args.steps,
                      "share": round(v[0] / timed_ms, 4) if timed_ms else None} for k, v in kern.items()}
-    total_algo = sum(algo.values())
+    total_algo = sum(v for k, v in algo.items() if k in kern)
 
     # end-to-end through the public API: pinned host inputs in, results out, every step
     e2e = None

@@ -199,11 +199,22 @@ __device__ __forceinline__ void uvu_recv_body(const DevPlan& P, const DevPath& p
   const float* xb = x + p.in_off + (act ? u : 0);
   const int yw = reduce_multi_index<8>(lane), pw_ = reduce_multi_index<KP>(lane);
   const bool ywr = reduce_multi_writer<8>(lane), pwr = reduce_multi_writer<KP>(lane);
+  // x rows of the chunk's sources, one edge ahead of the arithmetic
+  float xn[RI];
+  {
+    const long long row = (long long)sm.j[0] * P.dim_in;
+#pragma unroll
+    for (int k = 0; k < RI; ++k) xn[k] = act ? __ldg(xb + row + k * p.c_in) : 0.f;
+  }
   for (int t = 0; t < ne; ++t) {
-    const long long row = (long long)sm.j[t] * P.dim_in;
     float xv[RI], Y[RS], C[RO];
 #pragma unroll
-    for (int k = 0; k < RI; ++k) xv[k] = act ? __ldg(xb + row + k * p.c_in) : 0.f;
+    for (int k = 0; k < RI; ++k) xv[k] = xn[k];
+    if (t + 1 < ne) {
+      const long long row = (long long)sm.j[t + 1] * P.dim_in;
+#pragma unroll
+      for (int k = 0; k < RI; ++k) xn[k] = act ? __ldg(xb + row + k * p.c_in) : 0.f;
+    }
 #pragma unroll
     for (int k = 0; k < RS; ++k) Y[k] = sm.Y[t][LS * LS + k];
     cg_couple<LI, LS, LO>(xv, Y, C);

@@ -249,11 +249,22 @@ __device__ __forceinline__ void uvw_recv_body(const DevPlan& P, const DevPath& p
   }
   const int yw = reduce_multi_index<8>(lane), pw_ = reduce_multi_index<KP>(lane);
   const bool ywr = reduce_multi_writer<8>(lane), pwr = reduce_multi_writer<KP>(lane);
+  // x rows of the chunk's sources, one edge ahead of the arithmetic
+  float xn[RI];
+  {
+    const long long row = (long long)sm.j[0] * P.dim_in;
+#pragma unroll
+    for (int m = 0; m < RI; ++m) xn[m] = act ? __ldg(xb + row + m * p.c_in) : 0.f;
+  }
   for (int t = 0; t < ne; ++t) {
-    const long long row = (long long)sm.j[t] * P.dim_in;
     float xv[RI];
 #pragma unroll
-    for (int m = 0; m < RI; ++m) xv[m] = act ? __ldg(xb + row + m * p.c_in) : 0.f;
+    for (int m = 0; m < RI; ++m) xv[m] = xn[m];
+    if (t + 1 < ne) {
+      const long long row = (long long)sm.j[t + 1] * P.dim_in;
+#pragma unroll
+      for (int m = 0; m < RI; ++m) xn[m] = act ? __ldg(xb + row + m * p.c_in) : 0.f;
+    }
     float Y[RS], phi[KP];
 #pragma unroll
     for (int k = 0; k < RS; ++k) Y[k] = sm.Y[t][LS * LS + k];
