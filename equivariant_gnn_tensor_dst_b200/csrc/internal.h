@@ -9,6 +9,9 @@ constexpr int MAX_PATHS = 64;
 constexpr int MAX_TASKS = 256;
 constexpr int MAX_BLOCKS = 16;
 constexpr int WARPS_PER_CTA = 4;
+// Resident CTAs per SM requested by the streaming kernels (second launch-bounds argument,
+// a register cap of 65536 / (128 x blocks)): 4 or 5 where that measured faster, else left
+// to the compiler.
 
 // One path of the plan as the kernels see it.
 struct DevPath {

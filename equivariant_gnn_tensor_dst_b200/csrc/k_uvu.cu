@@ -245,7 +245,7 @@ __device__ __forceinline__ void uvu_recv_body(const DevPlan& P, const DevPath& p
 // One CTA per (receiver, share of its 32-edge chunks); its warps split the (path,
 // channel chunk) tasks.
 template <int KP>
-__global__ void __launch_bounds__(WARPS_PER_CTA * 32)
+__global__ void __launch_bounds__(WARPS_PER_CTA * 32, 5)
     k_uvu_recv_bwd(DevPlan P, Tasks T, const float* __restrict__ x, const float* __restrict__ pos,
                    const int* __restrict__ row_ptr, const int* __restrict__ src,
                    const float* __restrict__ W, const float* __restrict__ gout, int N,

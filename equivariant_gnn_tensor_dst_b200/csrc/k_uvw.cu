@@ -191,7 +191,7 @@ __device__ __forceinline__ void uvw_state_body(const DevPlan& P, const DevPath& 
 }
 
 template <int KP, int MODE>
-__global__ void __launch_bounds__(WARPS_PER_CTA * 32)
+__global__ void __launch_bounds__(WARPS_PER_CTA * 32, MODE == 0 ? 5 : 4)
     k_uvw_state(DevPlan P, Tasks T, const float* __restrict__ x, const float* __restrict__ xdot,
                 const float* __restrict__ pos, const float* __restrict__ posdot,
                 const int* __restrict__ row_ptr, const int* __restrict__ src, int node0,
@@ -304,7 +304,7 @@ __device__ __forceinline__ void uvw_recv_body(const DevPlan& P, const DevPath& p
 // channel chunk) tasks and keep per-warp partial sums of phi_bar and Y_bar per edge,
 // added in warp order.
 template <int KP>
-__global__ void __launch_bounds__(WARPS_PER_CTA * 32)
+__global__ void __launch_bounds__(WARPS_PER_CTA * 32, 4)
     k_uvw_recv_bwd(DevPlan P, Tasks T, const float* __restrict__ x, const float* __restrict__ pos,
                    const int* __restrict__ row_ptr, const int* __restrict__ src,
                    const float* __restrict__ Sbar, int node0, int n_nodes, float4* gbuf) {
@@ -476,7 +476,7 @@ __device__ __forceinline__ void uvw_src_body(const DevPlan& P, const DevPath& p,
 }
 
 template <int KP, int MODE>
-__global__ void __launch_bounds__(WARPS_PER_CTA * 32)
+__global__ void __launch_bounds__(WARPS_PER_CTA * 32, MODE == 0 ? 5 : 4)
     k_uvw_src_state(DevPlan P, Tasks T, const float* __restrict__ pos,
                     const float* __restrict__ posdot, const int* __restrict__ t_ptr,
                     const int* __restrict__ t_dst, const float* __restrict__ gout, int node0,
