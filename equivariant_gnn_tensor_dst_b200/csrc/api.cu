@@ -148,6 +148,13 @@ Prof& prof() {
   return p;
 }
 
+// Kernel launches counted where their number is known only at launch time.
+void prof_add_launches(int c, int n) {
+  Prof& P = prof();
+  std::lock_guard<std::mutex> g(P.mu);
+  if (P.on) P.launches[c] += n;
+}
+
 // Brackets one library call that launches `nk` kernels on stream s.
 struct ProfScope {
   int slot = -1;
@@ -521,19 +528,22 @@ struct Batch {
     g.partial = partial;
   }
   // Launch the collected problems.  With automatic splitting, split-K is used when the
-  // output tiles alone would leave SMs idle.
+  // output tiles alone would leave SMs idle: as many splits as keep the grid within one
+  // wave of resident CTAs (two per SM), so that no partial second wave runs.
   void flush() {
     if (g.n_problems == 0) return;
     if (err == cudaSuccess) {
       GemmBatch h = g;
       if (h.splits == 1 && auto_part) {
         const int tiles = gemm_tiles(h);
-        if (tiles > 0 && tiles < 2 * 148) {
-          h.splits = std::min(kSplits, (2 * 148 + tiles - 1) / tiles);
+        const int wave = 2 * 148;
+        if (tiles > 0 && 2 * tiles <= wave) {
+          h.splits = std::min(kSplits, wave / tiles);
           h.partial = auto_part;
         }
       }
       err = launch_gemm(h, st);
+      if (h.total_tiles > 0) prof_add_launches(PC_GEMM, h.splits > 1 ? 2 : 1);
     }
     g.n_problems = 0;
     g.n_segs = 0;
@@ -638,7 +648,7 @@ cudaError_t gemm_xbar(const tpconv_plan* P, const float* X, const float* W, cons
 // (the node) and operand tiles never cross a node boundary.
 cudaError_t gemm_abar_src(const tpconv_plan* P, const float* x, const float* X, float* gW, int n0, int cn,
                           int accumulate, float* part, cudaStream_t st) {
-  Batch b(st, kSplits, accumulate, part);
+  Batch b(st, 1, accumulate, nullptr, part);
   for (const PathH& p : P->paths) {
     const int RI = 2 * p.l_in + 1;
     b.problem(gW + p.w_off, idx2(p.c_out, P->n_w, 1), idx1(p.c_out), P->K * p.c_out, p.c_in, RI);
@@ -653,7 +663,7 @@ cudaError_t gemm_abar_src(const tpconv_plan* P, const float* x, const float* X, 
 // one segment per mo (single-stride k maps, as above)
 cudaError_t gemm_abar_recv(const tpconv_plan* P, const float* S, const float* gout, float* gW, int n0, int cn,
                            int accumulate, float* part, cudaStream_t st) {
-  Batch b(st, kSplits, accumulate, part);
+  Batch b(st, 1, accumulate, nullptr, part);
   for (const PathH& p : P->paths) {
     const int RO = 2 * p.l_out + 1;
     b.problem(gW + p.w_off, idx2(p.c_in, P->n_w, p.c_out), idx1(1), P->K * p.c_in, p.c_out, RO);
@@ -706,7 +716,7 @@ tpconv_status tpconv_forward(tpconv_plan_t P, int64_t N, int64_t E, const float*
     const int cn = std::min(L.recv_chunk, n - n0);
     TPC_RUN(PC_UVW_STATE, 1, launch_uvw_state(P->dev, P->t_in, 0, x, nullptr, pos, nullptr, row_ptr, src, n0, cn, S,
                              nullptr, s));
-    TPC_RUN(PC_GEMM, 2, gemm_state_times_A(P, S, W, nullptr, nullptr, out, n0, cn, fptr(ws, L.part), s));
+    TPC_RUN(PC_GEMM, 0, gemm_state_times_A(P, S, W, nullptr, nullptr, out, n0, cn, fptr(ws, L.part), s));
   }
   return TPCONV_OK;
 }
@@ -760,7 +770,7 @@ tpconv_status tpconv_backward(tpconv_plan_t P, int64_t N, int64_t E, const float
   if (grad_pos) {
     for (int n0 = 0; n0 < n; n0 += L.recv_chunk) {
       const int cn = std::min(L.recv_chunk, n - n0);
-      TPC_RUN(PC_GEMM, 1, gemm_sbar(P, grad_out, W, state, n0, cn, s));
+      TPC_RUN(PC_GEMM, 0, gemm_sbar(P, grad_out, W, state, n0, cn, s));
       TPC_RUN(PC_UVW_RECV_BWD, 1, launch_uvw_recv_bwd(P->dev, P->t_in, x, pos, row_ptr, src, state, n0, cn, gbuf, edge_split, s));
     }
     TPC_RUN(PC_POS, 1, launch_pos_finish(n, row_ptr, t_ptr, t_eid, gbuf, grad_pos, s));
@@ -772,8 +782,8 @@ tpconv_status tpconv_backward(tpconv_plan_t P, int64_t N, int64_t E, const float
       const int cn = std::min(L.src_chunk, n - n0);
       TPC_RUN(PC_UVW_SRC, 1, launch_uvw_src_state(P->dev, P->t_out, 0, pos, nullptr, t_ptr, t_eid, t_dst, grad_out, n0,
                                    cn, state, nullptr, s));
-      if (grad_x) TPC_RUN(PC_GEMM, 1, gemm_xbar(P, state, W, nullptr, nullptr, grad_x, n0, cn, part, s));
-      if (grad_W) TPC_RUN(PC_GEMM, 2, gemm_abar_src(P, x, state, grad_W, n0, cn, n0 > 0, part, s));
+      if (grad_x) TPC_RUN(PC_GEMM, 0, gemm_xbar(P, state, W, nullptr, nullptr, grad_x, n0, cn, part, s));
+      if (grad_W) TPC_RUN(PC_GEMM, 0, gemm_abar_src(P, x, state, grad_W, n0, cn, n0 > 0, part, s));
     }
   }
   return TPCONV_OK;
@@ -837,9 +847,9 @@ tpconv_status tpconv_double_backward(tpconv_plan_t P, int64_t N, int64_t E, cons
       TPC_RUN(PC_UVW_STATE_TAN, 1, launch_uvw_state(P->dev, P->t_in, 1, x, gg_x, pos, gg_pos, row_ptr, src, n0, cn,
                                need_S ? sb : nullptr, sa, s));
       if (grad_grad_out)
-        TPC_RUN(PC_GEMM, 1, gemm_state_times_A(P, tan_xp ? sa : nullptr, W, need_S ? sb : nullptr, gg_W, grad_grad_out, n0,
+        TPC_RUN(PC_GEMM, 0, gemm_state_times_A(P, tan_xp ? sa : nullptr, W, need_S ? sb : nullptr, gg_W, grad_grad_out, n0,
                                    cn, part, s));
-      if (grad_W && tan_xp) TPC_RUN(PC_GEMM, 2, gemm_abar_recv(P, sa, grad_out, grad_W, n0, cn, n0 > 0, part, s));
+      if (grad_W && tan_xp) TPC_RUN(PC_GEMM, 0, gemm_abar_recv(P, sa, grad_out, grad_W, n0, cn, n0 > 0, part, s));
     }
   }
   if (grad_x) {
@@ -851,7 +861,7 @@ tpconv_status tpconv_double_backward(tpconv_plan_t P, int64_t N, int64_t E, cons
         // sa = X' (tangent of the source state), sb = X
         TPC_RUN(PC_UVW_SRC_TAN, 1, launch_uvw_src_state(P->dev, P->t_out, 1, pos, gg_pos, t_ptr, t_eid, t_dst, grad_out, n0,
                                      cn, gg_W ? sb : nullptr, sa, s));
-        TPC_RUN(PC_GEMM, 1, gemm_xbar(P, gg_pos ? sa : nullptr, W, gg_W ? sb : nullptr, gg_W, grad_x, n0, cn, part, s));
+        TPC_RUN(PC_GEMM, 0, gemm_xbar(P, gg_pos ? sa : nullptr, W, gg_W ? sb : nullptr, gg_W, grad_x, n0, cn, part, s));
       }
     }
   }
@@ -987,7 +997,7 @@ extern "C" tpconv_status tpconv_forward_no_alloc(tpconv_plan_t P, int64_t N, int
     const int cn = std::min(L.recv_chunk, n - n0);
     TPC_RUN(PC_UVW_STATE, 1, launch_uvw_state(P->dev, P->t_in, 0, x, nullptr, pos, nullptr, row_ptr, src, n0, cn, S,
                                               nullptr, s));
-    TPC_RUN(PC_GEMM, 2, gemm_state_times_A(P, S, W, nullptr, nullptr, out, n0, cn, fptr(ws, L.part), s));
+    TPC_RUN(PC_GEMM, 0, gemm_state_times_A(P, S, W, nullptr, nullptr, out, n0, cn, fptr(ws, L.part), s));
   }
   return TPCONV_OK;
 }
