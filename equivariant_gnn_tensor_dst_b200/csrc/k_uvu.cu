@@ -197,8 +197,10 @@ __device__ __forceinline__ void uvu_recv_body(const DevPlan& P, const DevPath& p
   for (int o = 0; o < RO; ++o)
     mb[o] = act ? __ldg(gout + (long long)i * P.dim_out + p.out_off + o * p.c_out + u) : 0.f;
   const float* xb = x + p.in_off + (act ? u : 0);
-  const int yw = reduce_multi_index<8>(lane), pw_ = reduce_multi_index<KP>(lane);
-  const bool ywr = reduce_multi_writer<8>(lane), pwr = reduce_multi_writer<KP>(lane);
+  // Y_bar has RS components: reduce the next power of two of them
+  constexpr int NY = RS <= 1 ? 1 : RS <= 2 ? 2 : RS <= 4 ? 4 : 8;
+  const int yw = reduce_multi_index<NY>(lane), pw_ = reduce_multi_index<KP>(lane);
+  const bool ywr = reduce_multi_writer<NY>(lane), pwr = reduce_multi_writer<KP>(lane);
   // x rows of the chunk's sources, one edge ahead of the arithmetic
   float xn[RI];
   {
@@ -228,14 +230,14 @@ __device__ __forceinline__ void uvu_recv_body(const DevPlan& P, const DevPath& p
       we = fmaf(sm.phi[t][q], a[q], we);
       pp[q] = a[q] * h;                                        // eq. 20 (per channel)
     }
-    float G[RO], py[8];
+    float G[RO], py[NY];
 #pragma unroll
     for (int o = 0; o < RO; ++o) G[o] = mb[o] * we;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) py[k] = 0.f;
+    for (int k = 0; k < NY; ++k) py[k] = 0.f;
     cg_adj_y<LI, LS, LO>(xv, G, py);                            // eq. 22 (per channel)
     const float rphi = warp_reduce_multi<KP>(pp);
-    const float ry = warp_reduce_multi<8>(py);
+    const float ry = warp_reduce_multi<NY>(py);
     if (pwr) sm.accphi[w][t][pw_] += rphi;
     if (ywr && yw < RS) sm.accY[w][t][LS * LS + yw] += ry;
     __syncwarp();

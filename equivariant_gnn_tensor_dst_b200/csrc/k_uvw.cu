@@ -247,8 +247,10 @@ __device__ __forceinline__ void uvw_recv_body(const DevPlan& P, const DevPath& p
       for (int q = 0; q < KP; ++q)
         sb[q][o] = (act && q < P.K) ? Sbar[base + (long long)o * rs + q * p.c_in] : 0.f;
   }
-  const int yw = reduce_multi_index<8>(lane), pw_ = reduce_multi_index<KP>(lane);
-  const bool ywr = reduce_multi_writer<8>(lane), pwr = reduce_multi_writer<KP>(lane);
+  // Y_bar has RS components: reduce the next power of two of them
+  constexpr int NY = RS <= 1 ? 1 : RS <= 2 ? 2 : RS <= 4 ? 4 : 8;
+  const int yw = reduce_multi_index<NY>(lane), pw_ = reduce_multi_index<KP>(lane);
+  const bool ywr = reduce_multi_writer<NY>(lane), pwr = reduce_multi_writer<KP>(lane);
   // x rows of the chunk's sources, one edge ahead of the arithmetic
   float xn[RI];
   {
@@ -288,12 +290,12 @@ __device__ __forceinline__ void uvw_recv_body(const DevPlan& P, const DevPath& p
       for (int q = 0; q < KP; ++q) s = fmaf(phi[q], sb[q][o], s);
       Tb[o] = s;
     }
-    float py[8];
+    float py[NY];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) py[k] = 0.f;
+    for (int k = 0; k < NY; ++k) py[k] = 0.f;
     cg_adj_y<LI, LS, LO>(xv, Tb, py);
     const float rphi = warp_reduce_multi<KP>(pp);
-    const float ry = warp_reduce_multi<8>(py);
+    const float ry = warp_reduce_multi<NY>(py);
     if (pwr) sm.accphi[w][t][pw_] += rphi;
     if (ywr && yw < RS) sm.accY[w][t][LS * LS + yw] += ry;
     __syncwarp();
