@@ -470,6 +470,57 @@ def run_extras(args, dev, flush):
     return out
 
 
+def run_profiles(args):
+    """Forward, backward and full double backward (all three tangents) of every feature
+    profile (workloads.profile_configs) on one fixed graph; one JSON line."""
+    import torch
+
+    from equivariant_gnn_tensor_dst_b200 import binding
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    steps, warm = max(5, min(args.steps, 20)), 3
+    profs = workloads.profile_configs()
+    g, _ = workloads.make_graph(profs[0], seed=1100)
+    N, E = g.n_nodes, g.n_edges
+    tt = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)  # noqa: E731
+    pos, rp, src = tt(g.pos), tt(g.row_ptr), tt(g.src)
+    views = binding.tpconv_csr_transpose(rp, src, N)
+    rows = []
+    for c in profs:
+        plan = binding.Plan(c.irreps_in, c.sh_lmax, c.irreps_out, c.mode, c.radial, c.num_basis, c.r_cut,
+                            c.r_min, c.r_max)
+        rng = np.random.default_rng(2000 + c.cfg)
+        x = tt(workloads.normal(rng, (N, plan.dim_in)))
+        W = tt(workloads.weights(rng, c.num_basis, plan.fan_in_per_column()))
+        go = tt(workloads.normal(rng, (N, plan.dim_out)))
+        ggx, ggp = tt(workloads.normal(rng, (N, plan.dim_in))), tt(workloads.normal(rng, (N, 3)))
+        ggw = tt(workloads.normal(rng, (plan.num_basis, plan.weight_cols)))
+        wsb = plan.workspace_bytes(N, E)
+        ws = binding.workspace(wsb, dev)
+        o = torch.empty(N, plan.dim_out, device=dev)
+        gx, gp = torch.empty(N, plan.dim_in, device=dev), torch.empty(N, 3, device=dev)
+        gw = torch.empty(plan.num_basis, plan.weight_cols, device=dev)
+        dx, dg = torch.empty(N, plan.dim_in, device=dev), torch.empty(N, plan.dim_out, device=dev)
+        dw = torch.empty(plan.num_basis, plan.weight_cols, device=dev)
+        fwd = lambda: binding.tpconv_forward(plan, x, pos, rp, src, W, out=o, ws=ws)  # noqa: E731
+        bwd = lambda: binding.tpconv_backward(plan, x, pos, rp, src, *views, W, go, ws=ws,  # noqa: E731
+                                              outputs=(gx, gp, gw))
+        dbl = lambda: binding.tpconv_double_backward(plan, x, pos, rp, src, *views, W, go, gg_x=ggx,  # noqa: E731
+                                                     gg_pos=ggp, gg_W=ggw, ws=ws, outputs=(dx, dw, dg))
+        rec = {"profile": c.name, "mode": c.mode, "paths": len(plan.paths()), "workspace_bytes": wsb}
+        for name, fn in (("forward", fwd), ("backward", bwd), ("double_backward", dbl)):
+            ms = _timed(fn, flush, steps, warm)
+            rec[name + "_ms"] = round(ms, 4)
+            rec[name + "_edges_per_s"] = round(E / ms * 1e3, 1)
+        rows.append(rec)
+        del ws
+        torch.cuda.empty_cache()
+    print(json.dumps({"metric": "edges/s per pass on the feature-profile grid", "unit": "edges/s",
+                      "graph": {"nodes": N, "edges": E, "knn": profs[0].k, "density": profs[0].density},
+                      "l2": "flushed between timed calls", "steps": steps, "profiles": rows}), flush=True)
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle (baseline and reference arm)
 # ---------------------------------------------------------------------------
@@ -555,11 +606,15 @@ def main():
                     help="workload of the timed step (default: the uvw forward+backward workload)")
     ap.add_argument("--nodes", type=int, default=None,
                     help="resize the workload (same density and degree); for profiling small cases")
+    ap.add_argument("--profiles", action="store_true",
+                    help="instead of the timed step: every pass of the 25 feature profiles on one graph")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "native":
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.profiles:
+        run_profiles(args)
     else:
         run_native(args)
 

@@ -83,6 +83,12 @@ __device__ __forceinline__ void prep_edge(const DevPlan& P, const float* __restr
 // receiver state (eq. 33) and its tangent
 // ---------------------------------------------------------------------------
 
+// Resident CTAs per SM requested by the streaming kernels (register cap 65536 / (128 x
+// blocks)), chosen per radial width KP and pass: the fewest registers that do not spill
+// the KP x R accumulators (and their tangents in MODE 1), or that measured faster.
+#define TPC_MINB_STATE (KP == 8 ? (MODE == 0 ? 5 : 3) : (MODE == 0 ? 3 : 2))
+#define TPC_MINB_RECV (KP == 8 ? 4 : 3)
+
 template <int LI, int LS, int LO, int KP, int MODE>
 __device__ __forceinline__ void uvw_state_body(const DevPlan& P, const DevPath& p, int chunk, int i,
                                                int node_local, const float* __restrict__ x,
@@ -191,7 +197,7 @@ __device__ __forceinline__ void uvw_state_body(const DevPlan& P, const DevPath& 
 }
 
 template <int KP, int MODE>
-__global__ void __launch_bounds__(WARPS_PER_CTA * 32, MODE == 0 ? 5 : 4)
+__global__ void __launch_bounds__(WARPS_PER_CTA * 32, TPC_MINB_STATE)
     k_uvw_state(DevPlan P, Tasks T, const float* __restrict__ x, const float* __restrict__ xdot,
                 const float* __restrict__ pos, const float* __restrict__ posdot,
                 const int* __restrict__ row_ptr, const int* __restrict__ src, int node0,
@@ -306,7 +312,7 @@ __device__ __forceinline__ void uvw_recv_body(const DevPlan& P, const DevPath& p
 // channel chunk) tasks and keep per-warp partial sums of phi_bar and Y_bar per edge,
 // added in warp order.
 template <int KP>
-__global__ void __launch_bounds__(WARPS_PER_CTA * 32, 4)
+__global__ void __launch_bounds__(WARPS_PER_CTA * 32, TPC_MINB_RECV)
     k_uvw_recv_bwd(DevPlan P, Tasks T, const float* __restrict__ x, const float* __restrict__ pos,
                    const int* __restrict__ row_ptr, const int* __restrict__ src,
                    const float* __restrict__ Sbar, int node0, int n_nodes, float4* gbuf) {
@@ -478,7 +484,7 @@ __device__ __forceinline__ void uvw_src_body(const DevPlan& P, const DevPath& p,
 }
 
 template <int KP, int MODE>
-__global__ void __launch_bounds__(WARPS_PER_CTA * 32, MODE == 0 ? 5 : 4)
+__global__ void __launch_bounds__(WARPS_PER_CTA * 32, TPC_MINB_STATE)
     k_uvw_src_state(DevPlan P, Tasks T, const float* __restrict__ pos,
                     const float* __restrict__ posdot, const int* __restrict__ t_ptr,
                     const int* __restrict__ t_dst, const float* __restrict__ gout, int node0,

@@ -77,6 +77,46 @@ CONFIGS = {
 }
 
 
+# Feature-profile grids.  The pages time sixteen fully connected uvw profiles on a fixed
+# graph, varying angular order, channel width, scalar fraction and radial-operator size,
+# and channelwise uvu at three equal-multiplicity widths for each angular order; they do
+# not list the profiles.  Reading used here: uvw = lmax {2, 3} x width C {32, 64} x
+# {evenly spread: C per l; scalar-heavy: 4C x 0e, C/2 x 1o, C/4 x 2e, C/8 x 3o} x Bessel
+# K {8, 16}; uvu = lmax {1, 2, 3} x C {32, 64, 128} with C per l, Gaussian K=16 on
+# [0, 6].  Irreps in = out, SH lmax = feature lmax, natural parity (0e, 1o, 2e, 3o).  The
+# fixed graph is the uvw forward+backward workload's (N=4096, kNN k=32, density 0.1).
+
+_PARITY = "eoeo"
+
+
+def _irreps(mults):
+    return "+".join(f"{m}x{l}{_PARITY[l]}" for l, m in enumerate(mults) if m > 0)
+
+
+def profile_configs(n_nodes=4096, k=32):
+    out = []
+    idx = 100
+    for lmax in (2, 3):
+        for c in (32, 64):
+            for kind in ("even", "scalar-heavy"):
+                if kind == "even":
+                    mults = [c] * (lmax + 1)
+                else:
+                    mults = [4 * c, c // 2, c // 4, c // 8][:lmax + 1]
+                irr = _irreps(mults)
+                for kb in (8, 16):
+                    out.append(Config(idx, f"uvw lmax {lmax} C{c} {kind} K{kb}: {irr}", n_nodes, k, irr, lmax,
+                                      irr, "uvw", "bessel", kb, 5.0, passes=("fwd", "bwd", "dbl")))
+                    idx += 1
+    for lmax in (1, 2, 3):
+        for c in (32, 64, 128):
+            irr = _irreps([c] * (lmax + 1))
+            out.append(Config(idx, f"uvu lmax {lmax} C{c}: {irr}", n_nodes, k, irr, lmax, irr, "uvu",
+                              "gaussian", 16, 6.0, r_min=0.0, r_max=6.0, passes=("fwd", "bwd", "dbl")))
+            idx += 1
+    return out
+
+
 def _f32(a):
     return np.ascontiguousarray(np.asarray(a, dtype=np.float64).astype(np.float32))
 
