@@ -15,6 +15,7 @@ LIB_PATH = os.path.join(_HERE, "libtpconv.so")
 UVW, UVU = 0, 1
 BESSEL, GAUSSIAN = 0, 1
 PASS_FORWARD, PASS_BACKWARD, PASS_DOUBLE_BACKWARD = 1, 2, 4
+MATH_FP32, MATH_TF32 = 0, 1
 
 _c_i64 = ctypes.c_int64
 _c_p = ctypes.c_void_p
@@ -36,6 +37,7 @@ SIGNATURES = {
     "tpconv_plan_path_coupling": (ctypes.c_int, [_c_p, _c_i64, ctypes.POINTER(ctypes.c_int32),
                                                  ctypes.POINTER(ctypes.c_double), _c_i64]),
     "tpconv_set_workspace_budget": (ctypes.c_int, [_c_p, ctypes.c_size_t]),
+    "tpconv_plan_set_math": (ctypes.c_int, [_c_p, ctypes.c_int32]),
     "tpconv_workspace_bytes": (ctypes.c_int, [_c_p, _c_i64, _c_i64, ctypes.c_uint32,
                                               ctypes.POINTER(ctypes.c_size_t)]),
     "tpconv_csr_transpose_workspace_bytes": (ctypes.c_int, [_c_i64, _c_i64, ctypes.POINTER(ctypes.c_size_t)]),
@@ -138,6 +140,10 @@ class Plan:
 
     def set_workspace_budget(self, nbytes):
         check(lib().tpconv_set_workspace_budget(self._h, int(nbytes)), "tpconv_set_workspace_budget")
+
+    def set_math(self, math):
+        """MATH_FP32 (default, 3xTF32 contractions) or MATH_TF32 (one TF32 product)."""
+        check(lib().tpconv_plan_set_math(self._h, int(math)), "tpconv_plan_set_math")
 
     def workspace_bytes(self, n_nodes, n_edges, passes=PASS_FORWARD | PASS_BACKWARD | PASS_DOUBLE_BACKWARD):
         out = ctypes.c_size_t()

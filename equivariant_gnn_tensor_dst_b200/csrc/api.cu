@@ -192,6 +192,7 @@ struct tpconv_plan {
   Tasks t_bi{};   // (input block, chunk)   uvu source pass
   BlockPaths bp_out{}, bp_in{};
   size_t budget = kDefaultBudget;
+  int math = TPCONV_MATH_FP32;
 };
 
 namespace {
@@ -427,6 +428,13 @@ tpconv_status tpconv_set_workspace_budget(tpconv_plan_t P, size_t bytes) {
   return TPCONV_OK;
 }
 
+tpconv_status tpconv_plan_set_math(tpconv_plan_t P, int32_t math) {
+  if (!P) return TPCONV_ERR_INVALID_ARG;
+  if (math != TPCONV_MATH_FP32 && math != TPCONV_MATH_TF32) return TPCONV_ERR_UNSUPPORTED;
+  P->math = math;
+  return TPCONV_OK;
+}
+
 tpconv_status tpconv_workspace_bytes(tpconv_plan_t P, int64_t N, int64_t E, uint32_t pass_mask,
                                      size_t* bytes) {
   if (!P || !bytes || N < 0 || E < 0) return TPCONV_ERR_INVALID_ARG;
@@ -521,8 +529,10 @@ struct Batch {
   cudaStream_t st;
   float* auto_part;  // split-K scratch for automatic splitting (nullptr: never split automatically)
   cudaError_t err = cudaSuccess;
-  Batch(cudaStream_t s, int splits, int accumulate, float* partial, float* auto_split_part = nullptr)
+  Batch(const tpconv_plan* P, cudaStream_t s, int splits, int accumulate, float* partial,
+        float* auto_split_part = nullptr)
       : st(s), auto_part(auto_split_part) {
+    g.math = P->math;
     g.splits = splits;
     g.accumulate = accumulate;
     g.partial = partial;
@@ -586,7 +596,7 @@ int paths_into(const tpconv_plan* P, int block, bool out_side) {
 // optionally + sum_pi S2_pi A2_pi (eq. 37: dm = dS A + S dA)
 cudaError_t gemm_state_times_A(const tpconv_plan* P, const float* S, const float* W, const float* S2,
                                const float* W2, float* out, int n0, int cn, float* part, cudaStream_t st) {
-  Batch b(st, 1, 0, nullptr, part);
+  Batch b(P, st, 1, 0, nullptr, part);
   for (int bo = 0; bo < (int)P->out.size(); ++bo) {
     const Block& B = P->out[bo];
     const int RO = 2 * B.l + 1;
@@ -608,7 +618,7 @@ cudaError_t gemm_state_times_A(const tpconv_plan* P, const float* S, const float
 // S_bar_pi[(i,mo),(q,u)] = sum_w m_bar[(i,mo), w] A_pi[(q,u), w]        (eq. 36)
 cudaError_t gemm_sbar(const tpconv_plan* P, const float* gout, const float* W, float* Sbar, int n0,
                       int cn, cudaStream_t st) {
-  Batch b(st, 1, 0, nullptr);
+  Batch b(P, st, 1, 0, nullptr);
   for (const PathH& p : P->paths) {
     const int RO = 2 * p.l_out + 1;
     b.problem(Sbar + p.st_off, idx2(RO, P->dev.state_per_node, (long long)P->K * p.c_in), idx1(1), cn * RO,
@@ -623,7 +633,7 @@ cudaError_t gemm_sbar(const tpconv_plan* P, const float* gout, const float* W, f
 // (mirrored eq. 21), optionally + X2 A2^T (eq. 30 with A_dot)
 cudaError_t gemm_xbar(const tpconv_plan* P, const float* X, const float* W, const float* X2, const float* W2,
                       float* gx, int n0, int cn, float* part, cudaStream_t st) {
-  Batch b(st, 1, 0, nullptr, part);
+  Batch b(P, st, 1, 0, nullptr, part);
   for (int bi = 0; bi < (int)P->in.size(); ++bi) {
     const Block& B = P->in[bi];
     const int RI = 2 * B.l + 1;
@@ -648,7 +658,7 @@ cudaError_t gemm_xbar(const tpconv_plan* P, const float* X, const float* W, cons
 // (the node) and operand tiles never cross a node boundary.
 cudaError_t gemm_abar_src(const tpconv_plan* P, const float* x, const float* X, float* gW, int n0, int cn,
                           int accumulate, float* part, cudaStream_t st) {
-  Batch b(st, 1, accumulate, nullptr, part);
+  Batch b(P, st, 1, accumulate, nullptr, part);
   for (const PathH& p : P->paths) {
     const int RI = 2 * p.l_in + 1;
     b.problem(gW + p.w_off, idx2(p.c_out, P->n_w, 1), idx1(p.c_out), P->K * p.c_out, p.c_in, RI);
@@ -663,7 +673,7 @@ cudaError_t gemm_abar_src(const tpconv_plan* P, const float* x, const float* X, 
 // one segment per mo (single-stride k maps, as above)
 cudaError_t gemm_abar_recv(const tpconv_plan* P, const float* S, const float* gout, float* gW, int n0, int cn,
                            int accumulate, float* part, cudaStream_t st) {
-  Batch b(st, 1, accumulate, nullptr, part);
+  Batch b(P, st, 1, accumulate, nullptr, part);
   for (const PathH& p : P->paths) {
     const int RO = 2 * p.l_out + 1;
     b.problem(gW + p.w_off, idx2(p.c_in, P->n_w, p.c_out), idx1(1), P->K * p.c_in, p.c_out, RO);

@@ -10,7 +10,7 @@
 // a = hi + lo with hi = a truncated to TF32 and lo = a - hi; each k-step
 // issues hi*hi + hi*lo + lo*hi into the same fp32 accumulator ("3xTF32", the
 // decomposition of Ootomo and Yokota, 2022), which keeps the relative error near
-// 2^-21 instead of TF32's 2^-11.
+// 2^-21 instead of TF32's 2^-11.  The optional TF32 mode issues hi*hi only.
 //
 // Structure: one CTA of 288 threads per 128 x NT output tile (NT = 64 or 128) and
 // split-K slice, two CTAs per SM, warp-specialised around two rings: raw stages of 32 k
@@ -32,6 +32,7 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 #include "internal.h"
+#include "tpconv.h"
 
 namespace tpc {
 
@@ -265,6 +266,7 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
   const uint32_t tmem = *tmem_slot;
 
   constexpr uint32_t IDESC = instr_desc<NT>();
+  const bool tf32 = g.math == TPCONV_MATH_TF32;  // one TF32 product per term, no residuals
   constexpr int KWB = TC_K / (TC_PRODUCERS / NT);    // k values per producer for the B operand
   bool ok = true;
 
@@ -440,7 +442,7 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
             "r"(hi[0]), "r"(hi[1]), "r"(hi[2]), "r"(hi[3]), "r"(hi[4]), "r"(hi[5]), "r"(hi[6]), "r"(hi[7]),
             "r"(hi[8]), "r"(hi[9]), "r"(hi[10]), "r"(hi[11]), "r"(hi[12]), "r"(hi[13]), "r"(hi[14]), "r"(hi[15])
             : "memory");
-        asm volatile(
+        if (!tf32) asm volatile(
             "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
                 tlane + acol + 32u + 16u * h),
             "r"(lo[0]), "r"(lo[1]), "r"(lo[2]), "r"(lo[3]), "r"(lo[4]), "r"(lo[5]), "r"(lo[6]), "r"(lo[7]),
@@ -451,14 +453,20 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
       const char* braw = st + SM::A_BYTES;
       char* bhi = ops + os * 2 * SM::B_BYTES;
       char* blo = bhi + SM::B_BYTES;
+      if (tf32) {
 #pragma unroll
-      for (int q = c; q < SM::B_BYTES / 16; q += TC_CONVERTERS) {
-        const float4 v = *reinterpret_cast<const float4*>(braw + q * 16);
-        float4 h, l;
-        h.x = tf32_hi(v.x); h.y = tf32_hi(v.y); h.z = tf32_hi(v.z); h.w = tf32_hi(v.w);
-        l.x = v.x - h.x; l.y = v.y - h.y; l.z = v.z - h.z; l.w = v.w - h.w;
-        *reinterpret_cast<float4*>(bhi + q * 16) = h;
-        *reinterpret_cast<float4*>(blo + q * 16) = l;
+        for (int q = c; q < SM::B_BYTES / 16; q += TC_CONVERTERS)
+          *reinterpret_cast<float4*>(bhi + q * 16) = *reinterpret_cast<const float4*>(braw + q * 16);
+      } else {
+#pragma unroll
+        for (int q = c; q < SM::B_BYTES / 16; q += TC_CONVERTERS) {
+          const float4 v = *reinterpret_cast<const float4*>(braw + q * 16);
+          float4 h, l;
+          h.x = tf32_hi(v.x); h.y = tf32_hi(v.y); h.z = tf32_hi(v.z); h.w = tf32_hi(v.w);
+          l.x = v.x - h.x; l.y = v.y - h.y; l.z = v.z - h.z; l.w = v.w - h.w;
+          *reinterpret_cast<float4*>(bhi + q * 16) = h;
+          *reinterpret_cast<float4*>(blo + q * 16) = l;
+        }
       }
       // every value read from the raw stage has been used: the producers may refill it
       mbar_arrive(smem_u32(&empty[slot]));
@@ -490,14 +498,16 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
               "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
               "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem),
               "r"(ahi), "l"(dbh), "r"(IDESC), "r"(acc0));
-          asm volatile(
-              "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-              "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem),
-              "r"(ahi), "l"(dbl), "r"(IDESC), "r"(1u));
-          asm volatile(
-              "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-              "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem),
-              "r"(alo), "l"(dbh), "r"(IDESC), "r"(1u));
+          if (!tf32) {
+            asm volatile(
+                "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem),
+                "r"(ahi), "l"(dbl), "r"(IDESC), "r"(1u));
+            asm volatile(
+                "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem),
+                "r"(alo), "l"(dbh), "r"(IDESC), "r"(1u));
+          }
         }
         asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                          smem_u32(&mdone[os]))

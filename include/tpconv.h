@@ -129,6 +129,18 @@ tpconv_status tpconv_plan_path_coupling(tpconv_plan_t plan, int64_t index, int32
  * ranges; results do not depend on it.                                              */
 tpconv_status tpconv_set_workspace_budget(tpconv_plan_t plan, size_t bytes);
 
+/* Arithmetic of the channel contractions (the per-node products with the radial
+ * parameters A, Sobek section 4, eqs. 34-36 and their mirrored source-side forms).
+ *   TPCONV_MATH_FP32 (default): fp32 products from three TF32 tensor-core products
+ *     per term (hi*hi + hi*lo + lo*hi); results match fp32 to about 1e-6 relative.
+ *   TPCONV_MATH_TF32: one TF32 product per term (operands truncated to 10 mantissa
+ *     bits); about 1e-3 relative error, faster contractions.
+ * The streaming (edge) arithmetic is fp32 in both modes.  Any other value returns
+ * TPCONV_ERR_UNSUPPORTED and leaves the plan unchanged.                             */
+#define TPCONV_MATH_FP32 0
+#define TPCONV_MATH_TF32 1
+tpconv_status tpconv_plan_set_math(tpconv_plan_t plan, int32_t math);
+
 /* Workspace bytes needed by the passes in pass_mask for a graph of N nodes and E
  * edges.  The node-state part is bounded by the budget and does not grow with E;
  * backward adds 16 bytes per edge of position-gradient staging (only when a

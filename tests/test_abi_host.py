@@ -157,3 +157,12 @@ def test_binding_arity_matches_header():
     for name, params in re.findall(r"\b(tpconv_\w+)\s*\(([^;{]*?)\)\s*;", txt, flags=re.S):
         n = 0 if params.strip() in ("", "void") else params.count(",") + 1
         assert len(binding.SIGNATURES[name][1]) == n, name
+
+
+def test_plan_set_math_arguments():
+    L = binding.lib()
+    p = binding.Plan("8x0e+8x1o", 2, "8x0e+8x1o", "uvw", "bessel", 8, 3.0)
+    assert L.tpconv_plan_set_math(p.handle, binding.MATH_TF32) == 0
+    assert L.tpconv_plan_set_math(p.handle, binding.MATH_FP32) == 0
+    assert L.tpconv_plan_set_math(p.handle, 7) == 3          # TPCONV_ERR_UNSUPPORTED
+    assert L.tpconv_plan_set_math(None, binding.MATH_FP32) == 1   # TPCONV_ERR_INVALID_ARG

@@ -155,6 +155,35 @@ def test_double_backward_parity(torch, cfg):
         assert rel_l2(gg.cpu().numpy(), rg) <= TOL
 
 
+@pytest.mark.parametrize("cfg", [2, 5])
+def test_tf32_math_mode(torch, cfg):
+    """TF32 contractions (one tensor-core product per term): every pass within the
+    1e-2 relative bar for TF32 modes; the default mode stays within 1e-4."""
+    from equivariant_gnn_tensor_dst_b200 import binding
+    p = Problem(cfg, n_nodes=REDUCED[cfg])
+    lp = lib_plan(p.cfg)
+    lp.set_math(binding.MATH_TF32)
+    d = _dev(p)
+    v = _graph_views(d, p.N)
+    out = binding.tpconv_forward(lp, d["x"], d["pos"], d["row_ptr"], d["src"], d["W"])
+    assert rel_l2(out.cpu().numpy(), conv.forward(p.plan, p.x, p.pos, p.row_ptr, p.src, p.W)) <= 1e-2
+    gx, gp, gw = binding.tpconv_backward(lp, d["x"], d["pos"], d["row_ptr"], d["src"], *v, d["W"], d["gout"])
+    rx, rp, rw = conv.backward(p.plan, p.x, p.pos, p.row_ptr, p.src, p.W, p.gout)
+    for a, b in ((gx, rx), (gp, rp), (gw, rw)):
+        assert rel_l2(a.cpu().numpy(), b) <= 1e-2
+    ggx = workloads.normal(p.rng, p.x.shape)
+    ggp = workloads.normal(p.rng, p.pos.shape)
+    ggw = workloads.normal(p.rng, p.W.shape)
+    dx, dw, dg = binding.tpconv_double_backward(lp, d["x"], d["pos"], d["row_ptr"], d["src"], *v, d["W"],
+                                                d["gout"], gg_x=cuda(ggx), gg_pos=cuda(ggp), gg_W=cuda(ggw))
+    ex, ew, eg = conv.double_backward(p.plan, p.x, p.pos, p.row_ptr, p.src, p.W, p.gout, ggx, ggp, ggw)
+    for a, b in ((dx, ex), (dw, ew), (dg, eg)):
+        assert rel_l2(a.cpu().numpy(), b) <= 1e-2
+    lp.set_math(binding.MATH_FP32)
+    out = binding.tpconv_forward(lp, d["x"], d["pos"], d["row_ptr"], d["src"], d["W"])
+    assert rel_l2(out.cpu().numpy(), conv.forward(p.plan, p.x, p.pos, p.row_ptr, p.src, p.W)) <= TOL
+
+
 def test_force_training_step(torch):
     """Energy = sum of scalar outputs, forces F = -dE/dpos, loss |F - F_ref|^2, then the
     gradient of the loss w.r.t. W and x through the double backward."""
