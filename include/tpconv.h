@@ -45,6 +45,10 @@
  *    launched; a failed launch returns TPCONV_ERR_CUDA.
  *  - Results are deterministic: no floating-point atomics; every reduction has a
  *    fixed order (Sobek, section 4: receiver and source CSR ownership).
+ *  - tpconv_forward, tpconv_backward and tpconv_double_backward may be captured into
+ *    a CUDA graph once the same plan has run each captured pass eagerly on the device
+ *    (the first launch of a kernel sets its shared-memory attribute, which is not a
+ *    stream operation).  Replays read the buffers' current contents.
  */
 #ifndef TPCONV_H
 #define TPCONV_H
