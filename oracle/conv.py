@@ -15,6 +15,9 @@ Sobek: Streaming Equivariant Tensor Product Convolutions (arXiv 2607.18074):
   it returns dLambda/dx (eq. 30), dLambda/dA (eq. 27) and dLambda/dm_bar (eq. 25).
 * forward_streaming: the receiver-factorised order of eqs. 16 and 32-35 (state S,
   then m = S A).  Used only by the self-test that both orders agree (eq. 15 = eq. 16).
+* forward_embedded / backward_embedded: the same with the edge embedding phi_e and the
+  harmonics Y_e given per edge instead of computed from positions (the pages' own
+  interface, which returns the edge-owned adjoints phi_bar and Y_bar).
 
 Notation: for path pi with coupling c^pi[m_in, m_sh, m_out] (so3.path_coupling),
     C_{pi,u,mo}(x_j, Y) = sum_{mi,my} c^pi x_{j,u,mi} Y_my             (eq. 32)
@@ -173,15 +176,31 @@ def _edge_h(plan, mb, C):
 # ---------------------------------------------------------------------------
 
 def forward(plan, x, pos, row_ptr, src, A, edges=None):
-    x, pos, A = _f64(x), _f64(pos), _f64(A)
+    pos = _f64(pos)
     src = np.asarray(src, dtype=np.int64)
     dst = receivers_of(row_ptr)
-    N = pos.shape[0]
+    geo = lambda eb, need: _geometry(plan, pos, src, dst, eb, need)  # noqa: E731
+    return _forward(plan, x, src, dst, A, geo, pos.shape[0], edges)
+
+
+def forward_embedded(plan, x, Y, phi, row_ptr, n_nodes, src, A, edges=None):
+    """Forward with the edge embedding given per edge (Sobek's interface, section 3:
+    any invariant phi_e, e.g. a learned function of |r_e|, and the harmonics Y_e):
+    Y [E, (lmax+1)^2] and phi [E, K] in receiver-CSR edge order."""
+    src = np.asarray(src, dtype=np.int64)
+    Y, phi = _f64(Y), _f64(phi)
+    dst = receivers_of(row_ptr)
+    geo = lambda eb, need: (Y[eb], None, phi[eb], None)  # noqa: E731
+    return _forward(plan, x, src, dst, A, geo, n_nodes, edges)
+
+
+def _forward(plan, x, src, dst, A, geo, N, edges):
+    x, A = _f64(x), _f64(A)
     out = np.zeros((N, plan.dim_out))
     for eb in _edge_batches(src.shape[0], plan.n_w, edges):
         if eb.size == 0:
             continue
-        Y, _, phi, _ = _geometry(plan, pos, src, dst, eb, False)
+        Y, _, phi, _ = geo(eb, False)
         w = _radial_project(phi, A)                     # eqs. 12-13: W = phi A
         xs = x[src[eb]]
         z = np.zeros((eb.size, plan.dim_out))
@@ -200,17 +219,48 @@ def forward(plan, x, pos, row_ptr, src, A, edges=None):
 
 def backward(plan, x, pos, row_ptr, src, A, grad_out, edges=None):
     """Returns (grad_x [N, dim_in], grad_pos [N, 3], grad_A [K, N_w])."""
-    x, pos, A, mbar = _f64(x), _f64(pos), _f64(A), _f64(grad_out)
+    pos = _f64(pos)
     src = np.asarray(src, dtype=np.int64)
     dst = receivers_of(row_ptr)
     N = pos.shape[0]
-    gx = np.zeros((N, plan.dim_in))
     gpos = np.zeros((N, 3))
+
+    def edge_adjoints(eb, dY, dphi, ybar, phibar):
+        g = np.einsum("esk,es->ek", dY, ybar) + np.einsum("eqk,eq->ek", dphi, phibar)
+        np.add.at(gpos, src[eb], g)
+        np.add.at(gpos, dst[eb], -g)
+
+    geo = lambda eb, need: _geometry(plan, pos, src, dst, eb, need)  # noqa: E731
+    gx, gA = _backward(plan, x, src, dst, A, grad_out, geo, N, edges, edge_adjoints)
+    return gx, gpos, gA
+
+
+def backward_embedded(plan, x, Y, phi, row_ptr, n_nodes, src, A, grad_out, edges=None):
+    """Backward of forward_embedded.  Returns (grad_x [N, dim_in], grad_A [K, N_w],
+    grad_phi [E, K] (eq. 20), grad_Y [E, (lmax+1)^2] (eq. 22)), the last two edge-owned."""
+    src = np.asarray(src, dtype=np.int64)
+    Y, phi = _f64(Y), _f64(phi)
+    dst = receivers_of(row_ptr)
+    gphi = np.zeros_like(phi)
+    gY = np.zeros_like(Y)
+
+    def edge_adjoints(eb, dY, dphi, ybar, phibar):
+        gY[eb] = ybar
+        gphi[eb] = phibar
+
+    geo = lambda eb, need: (Y[eb], None, phi[eb], None)  # noqa: E731
+    gx, gA = _backward(plan, x, src, dst, A, grad_out, geo, n_nodes, edges, edge_adjoints)
+    return gx, gA, gphi, gY
+
+
+def _backward(plan, x, src, dst, A, grad_out, geo, N, edges, edge_adjoints):
+    x, A, mbar = _f64(x), _f64(A), _f64(grad_out)
+    gx = np.zeros((N, plan.dim_in))
     gA = np.zeros_like(A)
     for eb in _edge_batches(src.shape[0], plan.n_w, edges):
         if eb.size == 0:
             continue
-        Y, dY, phi, dphi = _geometry(plan, pos, src, dst, eb, True)
+        Y, dY, phi, dphi = geo(eb, True)
         w = _radial_project(phi, A)
         xs = x[src[eb]]
         mb_rows = mbar[dst[eb]]
@@ -229,11 +279,9 @@ def backward(plan, x, pos, row_ptr, src, A, grad_out, edges=None):
             ybar[:, sl] += _couple_adj_y(c, xj, G)                               # eq. 22
         gA += phi.T @ h                                                           # eq. 19
         phibar = h @ A.T                                                          # eq. 20
-        g = np.einsum("esk,es->ek", dY, ybar) + np.einsum("eqk,eq->ek", dphi, phibar)
-        np.add.at(gpos, src[eb], g)
-        np.add.at(gpos, dst[eb], -g)
+        edge_adjoints(eb, dY, dphi, ybar, phibar)
         np.add.at(gx, src[eb], xbar)
-    return gx, gpos, gA
+    return gx, gA
 
 
 # ---------------------------------------------------------------------------
