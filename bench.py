@@ -433,6 +433,17 @@ def run_extras(args, dev, flush):
         rec.update({"forward_ms": round(ms_f, 4), "forward_edges_per_s": round(E / ms_f * 1e3, 1),
                     "backward_ms": round(ms_b, 4), "backward_edges_per_s": round(E / ms_b * 1e3, 1)})
         if c.mode == "uvw":
+            # the embedded-input interface: phi_e and Y_e given per edge, phi_bar and Y_bar returned
+            Ye = tt(workloads.normal(rng, (E, (c.sh_lmax + 1) ** 2)))
+            pe = tt(workloads.normal(rng, (E, c.num_basis)))
+            gphi = torch.empty(E, c.num_basis, device=dev)
+            gY = torch.empty(E, (c.sh_lmax + 1) ** 2, device=dev)
+            fe = lambda: binding.tpconv_forward_embedded(plan, x, Ye, pe, rp, src, W, out=o, ws=ws)  # noqa: E731
+            be = lambda: binding.tpconv_backward_embedded(plan, x, Ye, pe, rp, src, *views, W, go, ws=ws,  # noqa: E731
+                                                          outputs=(gx, gw, gphi, gY))
+            ms_ef, ms_eb = _timed(fe, flush, steps, warm), _timed(be, flush, steps, warm)
+            rec["embedded_interface"] = {"forward_ms": round(ms_ef, 4), "backward_ms": round(ms_eb, 4),
+                                         "forward_backward_edges_per_s": round(E / (ms_ef + ms_eb) * 1e3, 1)}
             # the optional TF32 contraction mode (1e-2 accuracy class), reported separately
             plan.set_math(binding.MATH_TF32)
             ms_tf, ms_tb = _timed(fwd, flush, steps, warm), _timed(bwd, flush, steps, warm)

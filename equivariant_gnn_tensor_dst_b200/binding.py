@@ -46,6 +46,8 @@ SIGNATURES = {
     "tpconv_forward": (ctypes.c_int, [_c_p, _c_i64, _c_i64] + [_c_p] * 7 + [ctypes.c_size_t, _c_p]),
     "tpconv_backward": (ctypes.c_int, [_c_p, _c_i64, _c_i64] + [_c_p] * 13 + [ctypes.c_size_t, _c_p]),
     "tpconv_double_backward": (ctypes.c_int, [_c_p, _c_i64, _c_i64] + [_c_p] * 17 + [ctypes.c_size_t, _c_p]),
+    "tpconv_forward_embedded": (ctypes.c_int, [_c_p, _c_i64, _c_i64] + [_c_p] * 8 + [ctypes.c_size_t, _c_p]),
+    "tpconv_backward_embedded": (ctypes.c_int, [_c_p, _c_i64, _c_i64] + [_c_p] * 15 + [ctypes.c_size_t, _c_p]),
     "tpconv_profile_begin": (ctypes.c_int, [ctypes.c_int32]),
     "tpconv_profile_end": (ctypes.c_int, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_c_i64), ctypes.c_int32]),
     "tpconv_profile_category_name": (ctypes.c_char_p, [ctypes.c_int32]),
@@ -251,6 +253,47 @@ def tpconv_backward(plan, x, pos, row_ptr, src, t_ptr, t_eid, t_dst, W, grad_out
                                 _ptr(gx), _ptr(gp), _ptr(gw), _ptr(ws), ws.numel(), _stream(stream)),
           "tpconv_backward")
     return gx, gp, gw
+
+
+def tpconv_forward_embedded(plan, x, Y, phi, row_ptr, src, W, out=None, ws=None, stream=None):
+    """Forward with the edge embedding given per edge: Y [E, (lmax+1)^2], phi [E, K]."""
+    import torch
+    for t, n in ((x, "x"), (Y, "Y"), (phi, "phi"), (W, "W")):
+        _need(t, torch.float32, n)
+    _need(row_ptr, torch.int32, "row_ptr")
+    _need(src, torch.int32, "src")
+    N, E = row_ptr.numel() - 1, src.numel()
+    if out is None:
+        out = torch.empty(N, plan.dim_out, dtype=torch.float32, device=x.device)
+    if ws is None:
+        ws = workspace(plan.workspace_bytes(N, E, PASS_FORWARD), x.device)
+    check(lib().tpconv_forward_embedded(plan.handle, N, E, _ptr(x), _ptr(Y), _ptr(phi), _ptr(row_ptr), _ptr(src),
+                                        _ptr(W), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
+          "tpconv_forward_embedded")
+    return out
+
+
+def tpconv_backward_embedded(plan, x, Y, phi, row_ptr, src, t_ptr, t_eid, t_dst, W, grad_out, need_x=True,
+                             need_W=True, need_phi=True, need_Y=True, ws=None, outputs=None, stream=None):
+    """Returns (grad_x, grad_W, grad_phi [E, K], grad_Y [E, (lmax+1)^2])."""
+    import torch
+    N, E = row_ptr.numel() - 1, src.numel()
+    dev = x.device
+    if outputs is None:
+        gx = torch.empty(N, plan.dim_in, dtype=torch.float32, device=dev) if need_x else None
+        gw = torch.empty(plan.num_basis, plan.weight_cols, dtype=torch.float32, device=dev) if need_W else None
+        gphi = torch.empty(E, plan.num_basis, dtype=torch.float32, device=dev) if need_phi else None
+        gY = torch.empty(E, Y.shape[1], dtype=torch.float32, device=dev) if need_Y else None
+    else:
+        gx, gw, gphi, gY = outputs
+    if ws is None:
+        ws = workspace(plan.workspace_bytes(N, E, PASS_BACKWARD), dev)
+    check(lib().tpconv_backward_embedded(plan.handle, N, E, _ptr(x), _ptr(Y), _ptr(phi), _ptr(row_ptr), _ptr(src),
+                                         _ptr(t_ptr), _ptr(t_eid), _ptr(t_dst), _ptr(W), _ptr(grad_out),
+                                         _ptr(gx), _ptr(gw), _ptr(gphi), _ptr(gY), _ptr(ws), ws.numel(),
+                                         _stream(stream)),
+          "tpconv_backward_embedded")
+    return gx, gw, gphi, gY
 
 
 def tpconv_double_backward(plan, x, pos, row_ptr, src, t_ptr, t_eid, t_dst, W, grad_out, gg_x=None,

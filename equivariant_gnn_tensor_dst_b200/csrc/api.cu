@@ -351,6 +351,10 @@ tpconv_status tpconv_plan_create(tpconv_plan_t* out, const char* irreps_in, int3
   D.env_c = (float)(pp * (pp + 1) / 2.0);
   D.state_per_node = st_off;
   D.xstate_per_node = xst_off;
+  D.n_sh = (P->lmax + 1) * (P->lmax + 1);
+  D.emb_Y = D.emb_phi = nullptr;
+  D.emb_eid = nullptr;
+  D.emb_gY = D.emb_gphi = nullptr;
   for (int k = 0; k < D.n_paths; ++k) {
     const PathH& h = P->paths[k];
     DevPath& d = D.p[k];
@@ -791,6 +795,90 @@ tpconv_status tpconv_backward(tpconv_plan_t P, int64_t N, int64_t E, const float
     for (int n0 = 0; n0 < n; n0 += L.src_chunk) {
       const int cn = std::min(L.src_chunk, n - n0);
       TPC_RUN(PC_UVW_SRC, 1, launch_uvw_src_state(P->dev, P->t_out, 0, pos, nullptr, t_ptr, t_eid, t_dst, grad_out, n0,
+                                   cn, state, nullptr, s));
+      if (grad_x) TPC_RUN(PC_GEMM, 0, gemm_xbar(P, state, W, nullptr, nullptr, grad_x, n0, cn, part, s));
+      if (grad_W) TPC_RUN(PC_GEMM, 0, gemm_abar_src(P, x, state, grad_W, n0, cn, n0 > 0, part, s));
+    }
+  }
+  return TPCONV_OK;
+}
+
+tpconv_status tpconv_forward_embedded(tpconv_plan_t P, int64_t N, int64_t E, const float* x,
+                                      const float* Y, const float* phi, const int32_t* row_ptr,
+                                      const int32_t* src, const float* W, float* out, void* ws,
+                                      size_t ws_bytes, struct CUstream_st* stream) {
+  tpconv_status st = common_checks(P, N, E);
+  if (st != TPCONV_OK) return st;
+  if (P->mode != TPCONV_UVW) return TPCONV_ERR_UNSUPPORTED;
+  if (N == 0) return TPCONV_OK;
+  st = check_ptrs({x, row_ptr, W, out}, {src, Y, phi});
+  if (st != TPCONV_OK) return st;
+  if (E > 0 && (!src || !Y || !phi)) return TPCONV_ERR_INVALID_ARG;
+  const Layout L = make_layout(P, N, E, TPCONV_PASS_FORWARD);
+  st = check_ws(L, ws, ws_bytes);
+  if (st != TPCONV_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int n = (int)N;
+  DevPlan D = P->dev;
+  D.emb_Y = Y;
+  D.emb_phi = phi;
+  if (!every_block_reached(P, true)) TPC_TRY(cudaMemsetAsync(out, 0, sizeof(float) * (size_t)N * P->dim_out, s));
+  float* S = fptr(ws, L.state_a);
+  for (int n0 = 0; n0 < n; n0 += L.recv_chunk) {
+    const int cn = std::min(L.recv_chunk, n - n0);
+    TPC_RUN(PC_UVW_STATE, 1, launch_uvw_state(D, P->t_in, 0, x, nullptr, nullptr, nullptr, row_ptr, src, n0, cn, S,
+                             nullptr, s));
+    TPC_RUN(PC_GEMM, 0, gemm_state_times_A(P, S, W, nullptr, nullptr, out, n0, cn, fptr(ws, L.part), s));
+  }
+  return TPCONV_OK;
+}
+
+tpconv_status tpconv_backward_embedded(tpconv_plan_t P, int64_t N, int64_t E, const float* x,
+                                       const float* Y, const float* phi, const int32_t* row_ptr,
+                                       const int32_t* src, const int32_t* t_ptr, const int32_t* t_eid,
+                                       const int32_t* t_dst, const float* W, const float* grad_out,
+                                       float* grad_x, float* grad_W, float* grad_phi, float* grad_Y,
+                                       void* ws, size_t ws_bytes, struct CUstream_st* stream) {
+  tpconv_status st = common_checks(P, N, E);
+  if (st != TPCONV_OK) return st;
+  if (P->mode != TPCONV_UVW) return TPCONV_ERR_UNSUPPORTED;
+  st = check_ptrs({}, {x, Y, phi, row_ptr, src, t_ptr, t_eid, t_dst, W, grad_out, grad_x, grad_W, grad_phi, grad_Y});
+  if (st != TPCONV_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (N == 0) {
+    if (grad_W) TPC_TRY(cudaMemsetAsync(grad_W, 0, sizeof(float) * (size_t)P->K * P->n_w, s));
+    return TPCONV_OK;
+  }
+  if (!x || !row_ptr || !W || !grad_out || (E > 0 && (!src || !Y || !phi))) return TPCONV_ERR_INVALID_ARG;
+  if ((grad_x || grad_W) && (!t_ptr || (E > 0 && (!t_eid || !t_dst)))) return TPCONV_ERR_INVALID_ARG;
+  const Layout L = make_layout(P, N, E, TPCONV_PASS_BACKWARD);
+  st = check_ws(L, ws, ws_bytes);
+  if (st != TPCONV_OK) return st;
+  const int n = (int)N;
+  float4* gbuf = reinterpret_cast<float4*>(static_cast<char*>(ws) + L.gbuf);
+  float* part = fptr(ws, L.part);
+  DevPlan D = P->dev;
+  D.emb_Y = Y;
+  D.emb_phi = phi;
+  D.emb_eid = t_eid;
+  D.emb_gY = grad_Y;
+  D.emb_gphi = grad_phi;
+  const int edge_split = (int)std::max<long long>(1, std::min<long long>(16, (4 * E / std::max<int64_t>(N, 1) + 31) / 32));
+  float* state = fptr(ws, L.state_a);
+  if ((grad_phi || grad_Y) && E > 0) {
+    for (int n0 = 0; n0 < n; n0 += L.recv_chunk) {
+      const int cn = std::min(L.recv_chunk, n - n0);
+      TPC_RUN(PC_GEMM, 0, gemm_sbar(P, grad_out, W, state, n0, cn, s));
+      TPC_RUN(PC_UVW_RECV_BWD, 1, launch_uvw_recv_bwd(D, P->t_in, x, nullptr, row_ptr, src, state, n0, cn, gbuf,
+                                    edge_split, s));
+    }
+  }
+  if (grad_x && !every_block_reached(P, false))
+    TPC_TRY(cudaMemsetAsync(grad_x, 0, sizeof(float) * (size_t)N * P->dim_in, s));
+  if (grad_x || grad_W) {
+    for (int n0 = 0; n0 < n; n0 += L.src_chunk) {
+      const int cn = std::min(L.src_chunk, n - n0);
+      TPC_RUN(PC_UVW_SRC, 1, launch_uvw_src_state(D, P->t_out, 0, nullptr, nullptr, t_ptr, t_eid, t_dst, grad_out, n0,
                                    cn, state, nullptr, s));
       if (grad_x) TPC_RUN(PC_GEMM, 0, gemm_xbar(P, state, W, nullptr, nullptr, grad_x, n0, cn, part, s));
       if (grad_W) TPC_RUN(PC_GEMM, 0, gemm_abar_src(P, x, state, grad_W, n0, cn, n0 > 0, part, s));

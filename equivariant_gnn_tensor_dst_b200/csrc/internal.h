@@ -32,6 +32,14 @@ struct DevPlan {
   float env_a, env_b, env_c;
   int state_per_node;   // sum_pi R_out * K * C_in
   int xstate_per_node;  // sum_pi R_in * K * C_out
+  int n_sh;             // (lmax + 1)^2
+  // embedded-input calls only (all NULL otherwise): per-edge Y [E][n_sh] and phi [E][K]
+  // in receiver-CSR edge order, the source view's edge ids, and the edge-owned adjoints
+  const float* emb_Y;
+  const float* emb_phi;
+  const int* emb_eid;
+  float* emb_gY;
+  float* emb_gphi;
   DevPath p[MAX_PATHS];
 };
 

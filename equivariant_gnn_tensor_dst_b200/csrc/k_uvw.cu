@@ -37,9 +37,23 @@ struct GeoSmem {
 template <int LI, int LS, int LO, int KP, bool TAN>
 __device__ __forceinline__ void prep_edge(const DevPlan& P, const float* __restrict__ pos,
                                           const float* __restrict__ posdot, int i, int j,
-                                          int store, GeoSmem<KP, TAN>& sm, int w, int lane) {
+                                          int store, int e, GeoSmem<KP, TAN>& sm, int w, int lane) {
   constexpr int RS = 2 * LS + 1;
   constexpr int N4 = CgInfo<LI, LS, LO>::n4;
+  if (!TAN && P.emb_Y) {
+    // embedded input: Y_e and phi_e of edge e as given
+    float Y[RS], cy[4 * N4];
+#pragma unroll
+    for (int k = 0; k < RS; ++k) Y[k] = __ldg(P.emb_Y + (long long)e * P.n_sh + LS * LS + k);
+    sm.j[w][lane] = store;
+    cg_products<LI, LS, LO>(Y, cy);
+#pragma unroll
+    for (int b = 0; b < N4; ++b)
+      reinterpret_cast<float4*>(sm.cy[w][lane])[b] = make_float4(cy[4 * b], cy[4 * b + 1], cy[4 * b + 2], cy[4 * b + 3]);
+#pragma unroll
+    for (int q = 0; q < KP; ++q) sm.phi[w][lane][q] = q < P.K ? __ldg(P.emb_phi + (long long)e * P.K + q) : 0.f;
+    return;
+  }
   const EdgeGeo g = edge_geo(pos, i, j);
   const Pow3 pw(g.ux, g.uy, g.uz);
   float Y[RS];
@@ -116,7 +130,7 @@ __device__ __forceinline__ void uvw_state_body(const DevPlan& P, const DevPath& 
     const int ne = min(32, ee - e0);
     if (lane < ne) {
       const int j = __ldg(src + e0 + lane);
-      prep_edge<LI, LS, LO, KP, TAN>(P, pos, posdot, i, j, j, sm, w, lane);
+      prep_edge<LI, LS, LO, KP, TAN>(P, pos, posdot, i, j, j, e0 + lane, sm, w, lane);
     }
     __syncwarp();
     // x of the next edge is loaded while the current one is consumed
@@ -328,11 +342,19 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32, TPC_MINB_RECV)
     const int ne = min(32, ee - e0);
     if (w == 0 && lane < ne) {
       const int j = __ldg(src + e0 + lane);
-      const EdgeGeo g = edge_geo(pos, i, j);
-      const Pow3 pw(g.ux, g.uy, g.uz);
       float Y[16], phi[KP], dphi[KP];
-      sh_all(pw, Y);
-      radial<KP, false>(P, g.d, phi, dphi);
+      if (P.emb_Y) {   // embedded input: Y_e and phi_e as given
+        const long long e = e0 + lane;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) Y[k] = k < P.n_sh ? __ldg(P.emb_Y + e * P.n_sh + k) : 0.f;
+#pragma unroll
+        for (int q = 0; q < KP; ++q) phi[q] = q < P.K ? __ldg(P.emb_phi + e * P.K + q) : 0.f;
+      } else {
+        const EdgeGeo g = edge_geo(pos, i, j);
+        const Pow3 pw(g.ux, g.uy, g.uz);
+        sh_all(pw, Y);
+        radial<KP, false>(P, g.d, phi, dphi);
+      }
       sm.j[lane] = j;
 #pragma unroll
       for (int k = 0; k < 16; ++k) sm.Y[lane][k] = Y[k];
@@ -351,7 +373,24 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32, TPC_MINB_RECV)
       });
     }
     __syncthreads();
-    if (w == 0 && lane < ne) {
+    if (w == 0 && lane < ne && (P.emb_gY || P.emb_gphi)) {
+      // embedded input: the edge-owned adjoints Y_bar (eq. 22) and phi_bar (eq. 20)
+      const long long e = e0 + lane;
+      if (P.emb_gY)
+        for (int k = 0; k < P.n_sh; ++k) {
+          float s = 0.f;
+#pragma unroll
+          for (int ww = 0; ww < WARPS_PER_CTA; ++ww) s += sm.accY[ww][lane][k];
+          P.emb_gY[e * P.n_sh + k] = s;
+        }
+      if (P.emb_gphi)
+        for (int q = 0; q < P.K; ++q) {
+          float s = 0.f;
+#pragma unroll
+          for (int ww = 0; ww < WARPS_PER_CTA; ++ww) s += sm.accphi[ww][lane][q];
+          P.emb_gphi[e * P.K + q] = s;
+        }
+    } else if (w == 0 && lane < ne) {
       const int j = sm.j[lane];
       const EdgeGeo g = edge_geo(pos, i, j);
       const Pow3 pw(g.ux, g.uy, g.uz);
@@ -415,7 +454,8 @@ __device__ __forceinline__ void uvw_src_body(const DevPlan& P, const DevPath& p,
     // edge j -> i seen from its source: r = pos[j] - pos[i]; keep the receiver index
     if (lane < ne) {
       const int i = __ldg(t_dst + k0 + lane);
-      prep_edge<LI, LS, LO, KP, TAN>(P, pos, posdot, i, j, i, sm, w, lane);
+      const int e = P.emb_eid ? __ldg(P.emb_eid + k0 + lane) : 0;
+      prep_edge<LI, LS, LO, KP, TAN>(P, pos, posdot, i, j, i, e, sm, w, lane);
     }
     __syncwarp();
     float mn[RO];

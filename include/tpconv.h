@@ -202,6 +202,27 @@ tpconv_status tpconv_double_backward(tpconv_plan_t plan, int64_t N, int64_t E, c
                                      float* grad_W, float* grad_grad_out, float* grad_pos,
                                      void* ws, size_t ws_bytes, struct CUstream_st* stream);
 
+/* Sobek's own interface (section 3 and the wrapper it describes): the edge embedding is
+ * given per edge instead of computed from positions.  Y [E][(lmax+1)^2] holds the real
+ * harmonics (or any per-edge vector in their place, same component order as the plan's
+ * sh_lmax) and phi [E][K] any invariant edge embedding (e.g. a learned function of
+ * |r_e|), both fp32 in receiver-CSR edge order.  uvw plans only (uvu:
+ * TPCONV_ERR_UNSUPPORTED).  Workspace: as tpconv_forward / tpconv_backward.
+ *   forward: out as tpconv_forward (eqs. 11-13 with the given phi, Y).
+ *   backward: grad_x (eq. 21), grad_W (eq. 19) and the edge-owned adjoints
+ *     grad_phi [E][K] (eq. 20) and grad_Y [E][(lmax+1)^2] (eq. 22); each nullable;
+ *     t_ptr/t_eid/t_dst (tpconv_csr_transpose) are needed for grad_x and grad_W.      */
+tpconv_status tpconv_forward_embedded(tpconv_plan_t plan, int64_t N, int64_t E, const float* x,
+                                      const float* Y, const float* phi, const int32_t* row_ptr,
+                                      const int32_t* src, const float* W, float* out, void* ws,
+                                      size_t ws_bytes, struct CUstream_st* stream);
+tpconv_status tpconv_backward_embedded(tpconv_plan_t plan, int64_t N, int64_t E, const float* x,
+                                       const float* Y, const float* phi, const int32_t* row_ptr,
+                                       const int32_t* src, const int32_t* t_ptr, const int32_t* t_eid,
+                                       const int32_t* t_dst, const float* W, const float* grad_out,
+                                       float* grad_x, float* grad_W, float* grad_phi, float* grad_Y,
+                                       void* ws, size_t ws_bytes, struct CUstream_st* stream);
+
 /* Forward without any allocation by the caller or the library, for callers that
  * cannot obtain device memory themselves: for example a plug-in whose host application
  * owns every device allocation, or code that must not call cudaMalloc because that
