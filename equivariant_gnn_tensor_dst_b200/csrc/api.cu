@@ -201,6 +201,7 @@ struct Layout {
   int recv_chunk = 0, src_chunk = 0;
   size_t state_a = 0, state_b = 0;  // offsets of the (up to two) state arrays
   size_t gbuf = 0, part = 0;
+  size_t order = 0;                 // receiver order of the pass (uvw, N ints)
   size_t total = 0;
   bool has_gbuf = false, has_part = false;
 };
@@ -238,6 +239,8 @@ Layout make_layout(const tpconv_plan* P, long long N, long long E, uint32_t pass
     L.has_part = true;
     L.part = off;
     off += align256(size_t(4) * kSplits * pf);
+    L.order = off;
+    off += align256(size_t(4) * std::max<long long>(N, 1));
   } else {
     if (pass != TPCONV_PASS_FORWARD) {
       L.has_part = true;
@@ -355,6 +358,7 @@ tpconv_status tpconv_plan_create(tpconv_plan_t* out, const char* irreps_in, int3
   D.emb_Y = D.emb_phi = nullptr;
   D.emb_eid = nullptr;
   D.emb_gY = D.emb_gphi = nullptr;
+  D.order = nullptr;
   for (int k = 0; k < D.n_paths; ++k) {
     const PathH& h = P->paths[k];
     DevPath& d = D.p[k];
@@ -700,6 +704,14 @@ bool every_block_reached(const tpconv_plan* P, bool out_side) {
 
 float* fptr(void* ws, size_t off) { return reinterpret_cast<float*>(static_cast<char*>(ws) + off); }
 
+// The receiver order of a uvw pass (chunks of L.recv_chunk nodes, heaviest first), written
+// to the workspace and attached to a copy of the plan's device image.
+cudaError_t attach_order(DevPlan& D, const Layout& L, void* ws, int n, const int32_t* row_ptr, cudaStream_t s) {
+  int* order = reinterpret_cast<int*>(static_cast<char*>(ws) + L.order);
+  D.order = order;
+  return launch_degree_order(n, row_ptr, L.recv_chunk, order, s);
+}
+
 }  // namespace
 
 extern "C" {
@@ -726,9 +738,11 @@ tpconv_status tpconv_forward(tpconv_plan_t P, int64_t N, int64_t E, const float*
   }
   if (!every_block_reached(P, true)) TPC_TRY(cudaMemsetAsync(out, 0, sizeof(float) * (size_t)N * P->dim_out, s));
   float* S = fptr(ws, L.state_a);
+  DevPlan D = P->dev;
+  TPC_RUN(PC_UVW_STATE, 1, attach_order(D, L, ws, n, row_ptr, s));
   for (int n0 = 0; n0 < n; n0 += L.recv_chunk) {
     const int cn = std::min(L.recv_chunk, n - n0);
-    TPC_RUN(PC_UVW_STATE, 1, launch_uvw_state(P->dev, P->t_in, 0, x, nullptr, pos, nullptr, row_ptr, src, n0, cn, S,
+    TPC_RUN(PC_UVW_STATE, 1, launch_uvw_state(D, P->t_in, 0, x, nullptr, pos, nullptr, row_ptr, src, n0, cn, S,
                              nullptr, s));
     TPC_RUN(PC_GEMM, 0, gemm_state_times_A(P, S, W, nullptr, nullptr, out, n0, cn, fptr(ws, L.part), s));
   }
@@ -782,10 +796,12 @@ tpconv_status tpconv_backward(tpconv_plan_t P, int64_t N, int64_t E, const float
 
   float* state = fptr(ws, L.state_a);
   if (grad_pos) {
+    DevPlan D = P->dev;
+    TPC_RUN(PC_UVW_RECV_BWD, 1, attach_order(D, L, ws, n, row_ptr, s));
     for (int n0 = 0; n0 < n; n0 += L.recv_chunk) {
       const int cn = std::min(L.recv_chunk, n - n0);
       TPC_RUN(PC_GEMM, 0, gemm_sbar(P, grad_out, W, state, n0, cn, s));
-      TPC_RUN(PC_UVW_RECV_BWD, 1, launch_uvw_recv_bwd(P->dev, P->t_in, x, pos, row_ptr, src, state, n0, cn, gbuf, edge_split, s));
+      TPC_RUN(PC_UVW_RECV_BWD, 1, launch_uvw_recv_bwd(D, P->t_in, x, pos, row_ptr, src, state, n0, cn, gbuf, edge_split, s));
     }
     TPC_RUN(PC_POS, 1, launch_pos_finish(n, row_ptr, t_ptr, t_eid, gbuf, grad_pos, s));
   }
@@ -822,6 +838,7 @@ tpconv_status tpconv_forward_embedded(tpconv_plan_t P, int64_t N, int64_t E, con
   DevPlan D = P->dev;
   D.emb_Y = Y;
   D.emb_phi = phi;
+  TPC_RUN(PC_UVW_STATE, 1, attach_order(D, L, ws, n, row_ptr, s));
   if (!every_block_reached(P, true)) TPC_TRY(cudaMemsetAsync(out, 0, sizeof(float) * (size_t)N * P->dim_out, s));
   float* S = fptr(ws, L.state_a);
   for (int n0 = 0; n0 < n; n0 += L.recv_chunk) {
@@ -866,6 +883,7 @@ tpconv_status tpconv_backward_embedded(tpconv_plan_t P, int64_t N, int64_t E, co
   const int edge_split = (int)std::max<long long>(1, std::min<long long>(16, (4 * E / std::max<int64_t>(N, 1) + 31) / 32));
   float* state = fptr(ws, L.state_a);
   if ((grad_phi || grad_Y) && E > 0) {
+    TPC_RUN(PC_UVW_RECV_BWD, 1, attach_order(D, L, ws, n, row_ptr, s));
     for (int n0 = 0; n0 < n; n0 += L.recv_chunk) {
       const int cn = std::min(L.recv_chunk, n - n0);
       TPC_RUN(PC_GEMM, 0, gemm_sbar(P, grad_out, W, state, n0, cn, s));
@@ -939,10 +957,12 @@ tpconv_status tpconv_double_backward(tpconv_plan_t P, int64_t N, int64_t E, cons
     TPC_TRY(cudaMemsetAsync(grad_grad_out, 0, sizeof(float) * (size_t)N * P->dim_out, s));
   if (grad_W && !tan_xp) TPC_TRY(cudaMemsetAsync(grad_W, 0, sizeof(float) * (size_t)P->K * P->n_w, s));
   if ((grad_grad_out || grad_W) && (tan_xp || need_S)) {
+    DevPlan D = P->dev;
+    TPC_RUN(PC_UVW_STATE_TAN, 1, attach_order(D, L, ws, n, row_ptr, s));
     for (int n0 = 0; n0 < n; n0 += L.recv_chunk) {
       const int cn = std::min(L.recv_chunk, n - n0);
       // sa = dS (tangent of eq. 33), sb = S (needed for S dA in eq. 37)
-      TPC_RUN(PC_UVW_STATE_TAN, 1, launch_uvw_state(P->dev, P->t_in, 1, x, gg_x, pos, gg_pos, row_ptr, src, n0, cn,
+      TPC_RUN(PC_UVW_STATE_TAN, 1, launch_uvw_state(D, P->t_in, 1, x, gg_x, pos, gg_pos, row_ptr, src, n0, cn,
                                need_S ? sb : nullptr, sa, s));
       if (grad_grad_out)
         TPC_RUN(PC_GEMM, 0, gemm_state_times_A(P, tan_xp ? sa : nullptr, W, need_S ? sb : nullptr, gg_W, grad_grad_out, n0,

@@ -40,6 +40,9 @@ struct DevPlan {
   const int* emb_eid;
   float* emb_gY;
   float* emb_gphi;
+  // receiver processing order of a pass (NULL: node order): within every chunk of
+  // `order_chunk` nodes, the chunk's nodes by descending in-degree class
+  const int* order;
   DevPath p[MAX_PATHS];
 };
 
@@ -187,6 +190,7 @@ cudaError_t launch_pos_finish(int N, const int* row_ptr, const int* t_ptr, const
                               const float4* gbuf, float* grad_pos, cudaStream_t s);
 cudaError_t launch_csr_transpose(int N, int E, const int* row_ptr, const int* src, int* t_ptr,
                                  int* t_eid, int* t_dst, int* cursor, cudaStream_t s);
+cudaError_t launch_degree_order(int N, const int* row_ptr, int chunk, int* order, cudaStream_t s);
 cudaError_t launch_validate_graph(int N, int E, const int* row_ptr, const int* src, int* err,
                                   cudaStream_t s);
 

@@ -267,6 +267,38 @@ cudaError_t launch_csr_transpose(int N, int E, const int* row_ptr, const int* sr
   return cudaGetLastError();
 }
 
+// Receiver order for load balance: within each chunk of `chunk` nodes (one CTA per
+// chunk), the nodes grouped by in-degree class floor(log2(degree + 1)), heaviest class
+// first (longest work first).  The order inside a class is arbitrary; results do not
+// depend on it, since every receiver's output is computed independently.
+__global__ void k_degree_order(int N, const int* __restrict__ row_ptr, int chunk, int* __restrict__ order) {
+  constexpr int NB = 32;
+  __shared__ int count[NB], cursor[NB];
+  const int n0 = blockIdx.x * chunk, n1 = min(N, n0 + chunk);
+  if (threadIdx.x < NB) count[threadIdx.x] = 0;
+  __syncthreads();
+  for (int n = n0 + threadIdx.x; n < n1; n += blockDim.x) {
+    const int d = __ldg(row_ptr + n + 1) - __ldg(row_ptr + n);
+    atomicAdd(&count[31 - __clz(d + 1)], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int off = n0;
+    for (int b = NB - 1; b >= 0; --b) { cursor[b] = off; off += count[b]; }
+  }
+  __syncthreads();
+  for (int n = n0 + threadIdx.x; n < n1; n += blockDim.x) {
+    const int d = __ldg(row_ptr + n + 1) - __ldg(row_ptr + n);
+    order[atomicAdd(&cursor[31 - __clz(d + 1)], 1)] = n;
+  }
+}
+
+cudaError_t launch_degree_order(int N, const int* row_ptr, int chunk, int* order, cudaStream_t s) {
+  if (N <= 0 || chunk <= 0) return cudaSuccess;
+  k_degree_order<<<(unsigned)((N + chunk - 1) / chunk), 256, 0, s>>>(N, row_ptr, chunk, order);
+  return cudaGetLastError();
+}
+
 __global__ void k_validate(int N, int E, const int* __restrict__ row_ptr,
                            const int* __restrict__ src, int* err) {
   const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;

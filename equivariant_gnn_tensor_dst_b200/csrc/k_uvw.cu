@@ -222,8 +222,9 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32, TPC_MINB_STATE)
   // the instruction working set small
   const long long gw = (long long)blockIdx.x * WARPS_PER_CTA + (threadIdx.x >> 5);
   const int task = (int)(gw / n_nodes);
-  const int node_local = (int)(gw % n_nodes);
+  const int slot = (int)(gw % n_nodes);
   if (task >= T.n) return;
+  const int node_local = P.order ? __ldg(P.order + node0 + slot) - node0 : slot;
   const DevPath& p = P.p[T.a[task]];
   const int chunk = T.b[task];
   const int i = node0 + node_local;
@@ -332,8 +333,8 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32, TPC_MINB_RECV)
                    const float* __restrict__ Sbar, int node0, int n_nodes, float4* gbuf) {
   __shared__ RecvSmem<KP> sm;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int node_local = blockIdx.x;
-  if (node_local >= n_nodes) return;
+  if ((int)blockIdx.x >= n_nodes) return;
+  const int node_local = P.order ? __ldg(P.order + node0 + blockIdx.x) - node0 : (int)blockIdx.x;
   const int i = node0 + node_local;
   const int eb = __ldg(row_ptr + i), ee = __ldg(row_ptr + i + 1);
   // the 32-edge chunks of one receiver are shared by gridDim.y CTAs (their per-edge
