@@ -42,10 +42,10 @@ SPLIT_MMAS = 3                                      # 3xTF32: three TF32 product
 # launches have the same 1024-node chunk shape (per step: twice its launches).  Valid for
 # the kernels as captured; only reported for that workload.
 TRAFFIC_BYTES_PER_STEP = {
-    "channel_gemm": 2 * (6 * 92.80e6 + 2 * 32.93e6 + 6 * 12.70e6),
-    "uvw_receiver_backward": 4 * 96.65e6,
-    "uvw_source_state": 4 * 35.09e6,
-    "uvw_receiver_state": 4 * 34.54e6,
+    "channel_gemm": 2 * (6 * 92.48e6 + 2 * 32.95e6 + 6 * 9.43e6),
+    "uvw_receiver_backward": 4 * 95.48e6,
+    "uvw_source_state": 4 * 35.57e6,
+    "uvw_receiver_state": 4 * 35.11e6,
 }
 
 
