@@ -16,6 +16,7 @@ UVW, UVU = 0, 1
 BESSEL, GAUSSIAN = 0, 1
 PASS_FORWARD, PASS_BACKWARD, PASS_DOUBLE_BACKWARD = 1, 2, 4
 MATH_FP32, MATH_TF32 = 0, 1
+LAYOUT_IR_MUL, LAYOUT_MUL_IR = 0, 1
 
 _c_i64 = ctypes.c_int64
 _c_p = ctypes.c_void_p
@@ -38,6 +39,7 @@ SIGNATURES = {
                                                  ctypes.POINTER(ctypes.c_double), _c_i64]),
     "tpconv_set_workspace_budget": (ctypes.c_int, [_c_p, ctypes.c_size_t]),
     "tpconv_plan_set_math": (ctypes.c_int, [_c_p, ctypes.c_int32]),
+    "tpconv_plan_set_layout": (ctypes.c_int, [_c_p, ctypes.c_int32]),
     "tpconv_workspace_bytes": (ctypes.c_int, [_c_p, _c_i64, _c_i64, ctypes.c_uint32,
                                               ctypes.POINTER(ctypes.c_size_t)]),
     "tpconv_csr_transpose_workspace_bytes": (ctypes.c_int, [_c_i64, _c_i64, ctypes.POINTER(ctypes.c_size_t)]),
@@ -142,6 +144,10 @@ class Plan:
 
     def set_workspace_budget(self, nbytes):
         check(lib().tpconv_set_workspace_budget(self._h, int(nbytes)), "tpconv_set_workspace_budget")
+
+    def set_layout(self, layout):
+        """LAYOUT_IR_MUL (default, blocks [2l+1][C]) or LAYOUT_MUL_IR (blocks [C][2l+1])."""
+        check(lib().tpconv_plan_set_layout(self._h, int(layout)), "tpconv_plan_set_layout")
 
     def set_math(self, math):
         """MATH_FP32 (default, 3xTF32 contractions) or MATH_TF32 (one TF32 product)."""

@@ -193,6 +193,7 @@ struct tpconv_plan {
   BlockPaths bp_out{}, bp_in{};
   size_t budget = kDefaultBudget;
   int math = TPCONV_MATH_FP32;
+  int layout = TPCONV_LAYOUT_IR_MUL;
 };
 
 namespace {
@@ -258,6 +259,58 @@ Layout make_layout(const tpconv_plan* P, long long N, long long E, uint32_t pass
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// mul_ir boundary: node arrays are converted to and from ir_mul in workspace buffers
+// placed after the pass's own workspace (three input-width and two output-width arrays).
+size_t conversion_bytes(const tpconv_plan* P, long long N) {
+  if (P->layout != TPCONV_LAYOUT_MUL_IR) return 0;
+  return 3 * align256(size_t(4) * N * P->dim_in) + 2 * align256(size_t(4) * N * P->dim_out) + 256;
+}
+
+LayoutMap layout_map(const std::vector<Block>& blocks) {
+  LayoutMap M{};
+  M.n = (int)blocks.size();
+  for (int b = 0; b < M.n; ++b) {
+    M.off[b] = blocks[b].offset;
+    M.l[b] = blocks[b].l;
+    M.mul[b] = blocks[b].mul;
+  }
+  return M;
+}
+
+struct ConvBufs {
+  size_t inner = 0;                   // bytes left to the pass itself
+  float *xin[3] = {}, *xout[2] = {};  // input-width and output-width buffers
+};
+
+tpconv_status conversion_setup(const tpconv_plan* P, int64_t N, int64_t E, uint32_t pass, void* ws,
+                               size_t ws_bytes, ConvBufs& B) {
+  B.inner = align256(make_layout(P, N, E, pass).total);
+  const size_t need = B.inner + conversion_bytes(P, N);
+  if (ws_bytes < need) return TPCONV_ERR_WORKSPACE_TOO_SMALL;
+  if (!ws) return TPCONV_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ws) & 15u) != 0) return TPCONV_ERR_MISALIGNED;
+  char* p = static_cast<char*>(ws) + B.inner;
+  for (int i = 0; i < 3; ++i) { B.xin[i] = reinterpret_cast<float*>(p); p += align256(size_t(4) * N * P->dim_in); }
+  for (int i = 0; i < 2; ++i) { B.xout[i] = reinterpret_cast<float*>(p); p += align256(size_t(4) * N * P->dim_out); }
+  return TPCONV_OK;
+}
+
+// copy a node array into the ir_mul layout (NULL stays NULL)
+const float* to_ir_mul(const tpconv_plan* P, bool in_side, int64_t N, const float* a, float* buf,
+                       cudaStream_t s, cudaError_t& e) {
+  if (!a) return nullptr;
+  const LayoutMap M = layout_map(in_side ? P->in : P->out);
+  if (e == cudaSuccess) e = launch_layout_convert((int)N, in_side ? P->dim_in : P->dim_out, M, 1, a, buf, s);
+  return buf;
+}
+
+void from_ir_mul(const tpconv_plan* P, bool in_side, int64_t N, const float* buf, float* a, cudaStream_t s,
+                 cudaError_t& e) {
+  if (!a) return;
+  const LayoutMap M = layout_map(in_side ? P->in : P->out);
+  if (e == cudaSuccess) e = launch_layout_convert((int)N, in_side ? P->dim_in : P->dim_out, M, 0, buf, a, s);
+}
 
 }  // namespace
 
@@ -436,6 +489,13 @@ tpconv_status tpconv_set_workspace_budget(tpconv_plan_t P, size_t bytes) {
   return TPCONV_OK;
 }
 
+tpconv_status tpconv_plan_set_layout(tpconv_plan_t P, int32_t layout) {
+  if (!P) return TPCONV_ERR_INVALID_ARG;
+  if (layout != TPCONV_LAYOUT_IR_MUL && layout != TPCONV_LAYOUT_MUL_IR) return TPCONV_ERR_UNSUPPORTED;
+  P->layout = layout;
+  return TPCONV_OK;
+}
+
 tpconv_status tpconv_plan_set_math(tpconv_plan_t P, int32_t math) {
   if (!P) return TPCONV_ERR_INVALID_ARG;
   if (math != TPCONV_MATH_FP32 && math != TPCONV_MATH_TF32) return TPCONV_ERR_UNSUPPORTED;
@@ -448,7 +508,7 @@ tpconv_status tpconv_workspace_bytes(tpconv_plan_t P, int64_t N, int64_t E, uint
   if (!P || !bytes || N < 0 || E < 0) return TPCONV_ERR_INVALID_ARG;
   size_t best = 0;
   for (uint32_t b : {TPCONV_PASS_FORWARD, TPCONV_PASS_BACKWARD, TPCONV_PASS_DOUBLE_BACKWARD})
-    if (pass_mask & b) best = std::max(best, make_layout(P, N, E, b).total);
+    if (pass_mask & b) best = std::max(best, make_layout(P, N, E, b).total + conversion_bytes(P, N));
   *bytes = best;
   return TPCONV_OK;
 }
@@ -716,7 +776,7 @@ cudaError_t attach_order(DevPlan& D, const Layout& L, void* ws, int n, const int
 
 extern "C" {
 
-tpconv_status tpconv_forward(tpconv_plan_t P, int64_t N, int64_t E, const float* x,
+static tpconv_status forward_ir_mul(tpconv_plan_t P, int64_t N, int64_t E, const float* x,
                              const float* pos, const int32_t* row_ptr, const int32_t* src,
                              const float* W, float* out, void* ws, size_t ws_bytes,
                              struct CUstream_st* stream) {
@@ -749,7 +809,7 @@ tpconv_status tpconv_forward(tpconv_plan_t P, int64_t N, int64_t E, const float*
   return TPCONV_OK;
 }
 
-tpconv_status tpconv_backward(tpconv_plan_t P, int64_t N, int64_t E, const float* x,
+static tpconv_status backward_ir_mul(tpconv_plan_t P, int64_t N, int64_t E, const float* x,
                               const float* pos, const int32_t* row_ptr, const int32_t* src,
                               const int32_t* t_ptr, const int32_t* t_eid, const int32_t* t_dst,
                               const float* W, const float* grad_out, float* grad_x,
@@ -819,7 +879,7 @@ tpconv_status tpconv_backward(tpconv_plan_t P, int64_t N, int64_t E, const float
   return TPCONV_OK;
 }
 
-tpconv_status tpconv_forward_embedded(tpconv_plan_t P, int64_t N, int64_t E, const float* x,
+static tpconv_status forward_embedded_ir_mul(tpconv_plan_t P, int64_t N, int64_t E, const float* x,
                                       const float* Y, const float* phi, const int32_t* row_ptr,
                                       const int32_t* src, const float* W, float* out, void* ws,
                                       size_t ws_bytes, struct CUstream_st* stream) {
@@ -850,7 +910,7 @@ tpconv_status tpconv_forward_embedded(tpconv_plan_t P, int64_t N, int64_t E, con
   return TPCONV_OK;
 }
 
-tpconv_status tpconv_backward_embedded(tpconv_plan_t P, int64_t N, int64_t E, const float* x,
+static tpconv_status backward_embedded_ir_mul(tpconv_plan_t P, int64_t N, int64_t E, const float* x,
                                        const float* Y, const float* phi, const int32_t* row_ptr,
                                        const int32_t* src, const int32_t* t_ptr, const int32_t* t_eid,
                                        const int32_t* t_dst, const float* W, const float* grad_out,
@@ -905,7 +965,7 @@ tpconv_status tpconv_backward_embedded(tpconv_plan_t P, int64_t N, int64_t E, co
   return TPCONV_OK;
 }
 
-tpconv_status tpconv_double_backward(tpconv_plan_t P, int64_t N, int64_t E, const float* x,
+static tpconv_status double_backward_ir_mul(tpconv_plan_t P, int64_t N, int64_t E, const float* x,
                                      const float* pos, const int32_t* row_ptr, const int32_t* src,
                                      const int32_t* t_ptr, const int32_t* t_eid,
                                      const int32_t* t_dst, const float* W, const float* grad_out,
@@ -984,6 +1044,123 @@ tpconv_status tpconv_double_backward(tpconv_plan_t P, int64_t N, int64_t E, cons
     }
   }
   return TPCONV_OK;
+}
+
+// Public passes: the ir_mul implementations above, with the node arrays converted at the
+// boundary when the plan's layout is mul_ir.
+tpconv_status tpconv_forward(tpconv_plan_t P, int64_t N, int64_t E, const float* x, const float* pos,
+                             const int32_t* row_ptr, const int32_t* src, const float* W, float* out, void* ws,
+                             size_t ws_bytes, struct CUstream_st* stream) {
+  if (!P || P->layout == TPCONV_LAYOUT_IR_MUL || N <= 0)
+    return forward_ir_mul(P, N, E, x, pos, row_ptr, src, W, out, ws, ws_bytes, stream);
+  if (!x || !out || N > 0x7ffffffe) return TPCONV_ERR_INVALID_ARG;
+  ConvBufs B;
+  tpconv_status st = conversion_setup(P, N, E, TPCONV_PASS_FORWARD, ws, ws_bytes, B);
+  if (st != TPCONV_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaSuccess;
+  const float* xi = to_ir_mul(P, true, N, x, B.xin[0], s, e);
+  if (e != cudaSuccess) return TPCONV_ERR_CUDA;
+  st = forward_ir_mul(P, N, E, xi, pos, row_ptr, src, W, B.xout[0], ws, B.inner, stream);
+  if (st != TPCONV_OK) return st;
+  from_ir_mul(P, false, N, B.xout[0], out, s, e);
+  return e == cudaSuccess ? TPCONV_OK : TPCONV_ERR_CUDA;
+}
+
+tpconv_status tpconv_backward(tpconv_plan_t P, int64_t N, int64_t E, const float* x, const float* pos,
+                              const int32_t* row_ptr, const int32_t* src, const int32_t* t_ptr,
+                              const int32_t* t_eid, const int32_t* t_dst, const float* W, const float* grad_out,
+                              float* grad_x, float* grad_pos, float* grad_W, void* ws, size_t ws_bytes,
+                              struct CUstream_st* stream) {
+  if (!P || P->layout == TPCONV_LAYOUT_IR_MUL || N <= 0)
+    return backward_ir_mul(P, N, E, x, pos, row_ptr, src, t_ptr, t_eid, t_dst, W, grad_out, grad_x, grad_pos,
+                           grad_W, ws, ws_bytes, stream);
+  if (!x || !grad_out || N > 0x7ffffffe) return TPCONV_ERR_INVALID_ARG;
+  ConvBufs B;
+  tpconv_status st = conversion_setup(P, N, E, TPCONV_PASS_BACKWARD, ws, ws_bytes, B);
+  if (st != TPCONV_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaSuccess;
+  const float* xi = to_ir_mul(P, true, N, x, B.xin[0], s, e);
+  const float* gi = to_ir_mul(P, false, N, grad_out, B.xout[0], s, e);
+  if (e != cudaSuccess) return TPCONV_ERR_CUDA;
+  st = backward_ir_mul(P, N, E, xi, pos, row_ptr, src, t_ptr, t_eid, t_dst, W, gi, grad_x ? B.xin[1] : nullptr,
+                       grad_pos, grad_W, ws, B.inner, stream);
+  if (st != TPCONV_OK) return st;
+  from_ir_mul(P, true, N, B.xin[1], grad_x, s, e);
+  return e == cudaSuccess ? TPCONV_OK : TPCONV_ERR_CUDA;
+}
+
+tpconv_status tpconv_double_backward(tpconv_plan_t P, int64_t N, int64_t E, const float* x, const float* pos,
+                                     const int32_t* row_ptr, const int32_t* src, const int32_t* t_ptr,
+                                     const int32_t* t_eid, const int32_t* t_dst, const float* W,
+                                     const float* grad_out, const float* gg_x, const float* gg_pos,
+                                     const float* gg_W, float* grad_x, float* grad_W, float* grad_grad_out,
+                                     float* grad_pos, void* ws, size_t ws_bytes, struct CUstream_st* stream) {
+  if (!P || P->layout == TPCONV_LAYOUT_IR_MUL || N <= 0)
+    return double_backward_ir_mul(P, N, E, x, pos, row_ptr, src, t_ptr, t_eid, t_dst, W, grad_out, gg_x, gg_pos,
+                                  gg_W, grad_x, grad_W, grad_grad_out, grad_pos, ws, ws_bytes, stream);
+  if (!x || !grad_out || N > 0x7ffffffe) return TPCONV_ERR_INVALID_ARG;
+  ConvBufs B;
+  tpconv_status st = conversion_setup(P, N, E, TPCONV_PASS_DOUBLE_BACKWARD, ws, ws_bytes, B);
+  if (st != TPCONV_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaSuccess;
+  const float* xi = to_ir_mul(P, true, N, x, B.xin[0], s, e);
+  const float* gi = to_ir_mul(P, false, N, grad_out, B.xout[0], s, e);
+  const float* ggi = to_ir_mul(P, true, N, gg_x, B.xin[1], s, e);
+  if (e != cudaSuccess) return TPCONV_ERR_CUDA;
+  st = double_backward_ir_mul(P, N, E, xi, pos, row_ptr, src, t_ptr, t_eid, t_dst, W, gi, ggi, gg_pos, gg_W,
+                              grad_x ? B.xin[2] : nullptr, grad_W, grad_grad_out ? B.xout[1] : nullptr, grad_pos,
+                              ws, B.inner, stream);
+  if (st != TPCONV_OK) return st;
+  from_ir_mul(P, true, N, B.xin[2], grad_x, s, e);
+  from_ir_mul(P, false, N, B.xout[1], grad_grad_out, s, e);
+  return e == cudaSuccess ? TPCONV_OK : TPCONV_ERR_CUDA;
+}
+
+tpconv_status tpconv_forward_embedded(tpconv_plan_t P, int64_t N, int64_t E, const float* x, const float* Y,
+                                      const float* phi, const int32_t* row_ptr, const int32_t* src, const float* W,
+                                      float* out, void* ws, size_t ws_bytes, struct CUstream_st* stream) {
+  if (!P || P->layout == TPCONV_LAYOUT_IR_MUL || N <= 0 || P->mode != TPCONV_UVW)
+    return forward_embedded_ir_mul(P, N, E, x, Y, phi, row_ptr, src, W, out, ws, ws_bytes, stream);
+  if (!x || !out || N > 0x7ffffffe) return TPCONV_ERR_INVALID_ARG;
+  ConvBufs B;
+  tpconv_status st = conversion_setup(P, N, E, TPCONV_PASS_FORWARD, ws, ws_bytes, B);
+  if (st != TPCONV_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaSuccess;
+  const float* xi = to_ir_mul(P, true, N, x, B.xin[0], s, e);
+  if (e != cudaSuccess) return TPCONV_ERR_CUDA;
+  st = forward_embedded_ir_mul(P, N, E, xi, Y, phi, row_ptr, src, W, B.xout[0], ws, B.inner, stream);
+  if (st != TPCONV_OK) return st;
+  from_ir_mul(P, false, N, B.xout[0], out, s, e);
+  return e == cudaSuccess ? TPCONV_OK : TPCONV_ERR_CUDA;
+}
+
+tpconv_status tpconv_backward_embedded(tpconv_plan_t P, int64_t N, int64_t E, const float* x, const float* Y,
+                                       const float* phi, const int32_t* row_ptr, const int32_t* src,
+                                       const int32_t* t_ptr, const int32_t* t_eid, const int32_t* t_dst,
+                                       const float* W, const float* grad_out, float* grad_x, float* grad_W,
+                                       float* grad_phi, float* grad_Y, void* ws, size_t ws_bytes,
+                                       struct CUstream_st* stream) {
+  if (!P || P->layout == TPCONV_LAYOUT_IR_MUL || N <= 0 || P->mode != TPCONV_UVW)
+    return backward_embedded_ir_mul(P, N, E, x, Y, phi, row_ptr, src, t_ptr, t_eid, t_dst, W, grad_out, grad_x,
+                                    grad_W, grad_phi, grad_Y, ws, ws_bytes, stream);
+  if (!x || !grad_out || N > 0x7ffffffe) return TPCONV_ERR_INVALID_ARG;
+  ConvBufs B;
+  tpconv_status st = conversion_setup(P, N, E, TPCONV_PASS_BACKWARD, ws, ws_bytes, B);
+  if (st != TPCONV_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaSuccess;
+  const float* xi = to_ir_mul(P, true, N, x, B.xin[0], s, e);
+  const float* gi = to_ir_mul(P, false, N, grad_out, B.xout[0], s, e);
+  if (e != cudaSuccess) return TPCONV_ERR_CUDA;
+  st = backward_embedded_ir_mul(P, N, E, xi, Y, phi, row_ptr, src, t_ptr, t_eid, t_dst, W, gi,
+                                grad_x ? B.xin[1] : nullptr, grad_W, grad_phi, grad_Y, ws, B.inner, stream);
+  if (st != TPCONV_OK) return st;
+  from_ir_mul(P, true, N, B.xin[1], grad_x, s, e);
+  return e == cudaSuccess ? TPCONV_OK : TPCONV_ERR_CUDA;
 }
 
 tpconv_status tpconv_profile_begin(int32_t max_records) {
@@ -1090,6 +1267,7 @@ extern "C" tpconv_status tpconv_forward_no_alloc(tpconv_plan_t P, int64_t N, int
                                                  const float* pos, const int32_t* row_ptr,
                                                  const int32_t* src, const float* W, float* out,
                                                  struct CUstream_st* stream) {
+  if (P && P->layout != TPCONV_LAYOUT_IR_MUL) return TPCONV_ERR_UNSUPPORTED;  // ir_mul boundary only
   tpconv_status st = common_checks(P, N, E);
   if (st != TPCONV_OK) return st;
   if (N == 0) return TPCONV_OK;

@@ -191,6 +191,15 @@ cudaError_t launch_pos_finish(int N, const int* row_ptr, const int* t_ptr, const
 cudaError_t launch_csr_transpose(int N, int E, const int* row_ptr, const int* src, int* t_ptr,
                                  int* t_eid, int* t_dst, int* cursor, cudaStream_t s);
 cudaError_t launch_degree_order(int N, const int* row_ptr, int chunk, int* order, cudaStream_t s);
+
+// Irrep blocks of a node row, for converting between the ir_mul layout (block [2l+1][C])
+// and the mul_ir layout (block [C][2l+1]).
+struct LayoutMap {
+  int n;
+  int off[MAX_BLOCKS], l[MAX_BLOCKS], mul[MAX_BLOCKS];
+};
+cudaError_t launch_layout_convert(int N, int dim, const LayoutMap& M, int to_ir_mul, const float* src,
+                                  float* dst, cudaStream_t s);
 cudaError_t launch_validate_graph(int N, int E, const int* row_ptr, const int* src, int* err,
                                   cudaStream_t s);
 

@@ -299,6 +299,37 @@ cudaError_t launch_degree_order(int N, const int* row_ptr, int chunk, int* order
   return cudaGetLastError();
 }
 
+// Layout conversion of node rows: element (m, u) of block b is at off + m*C + u in
+// ir_mul and at off + u*(2l+1) + m in mul_ir.  One thread per source element (reads
+// coalesced).
+__global__ void k_layout_convert(long long total, int dim, const __grid_constant__ LayoutMap M, int to_ir_mul,
+                                 const float* __restrict__ src, float* __restrict__ dst) {
+  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= total) return;
+  const long long row = t / dim;
+  const int c = (int)(t - row * dim);
+  int b = 0;
+  while (b + 1 < M.n && M.off[b + 1] <= c) ++b;
+  const int local = c - M.off[b], R = 2 * M.l[b] + 1, C = M.mul[b];
+  int d;
+  if (to_ir_mul) {   // source mul_ir: local = u*R + m
+    const int u = local / R, m = local - u * R;
+    d = M.off[b] + m * C + u;
+  } else {           // source ir_mul: local = m*C + u
+    const int m = local / C, u = local - m * C;
+    d = M.off[b] + u * R + m;
+  }
+  dst[row * dim + d] = src[t];
+}
+
+cudaError_t launch_layout_convert(int N, int dim, const LayoutMap& M, int to_ir_mul, const float* src,
+                                  float* dst, cudaStream_t s) {
+  const long long total = (long long)N * dim;
+  if (total <= 0) return cudaSuccess;
+  k_layout_convert<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(total, dim, M, to_ir_mul, src, dst);
+  return cudaGetLastError();
+}
+
 __global__ void k_validate(int N, int E, const int* __restrict__ row_ptr,
                            const int* __restrict__ src, int* err) {
   const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;

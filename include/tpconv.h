@@ -145,6 +145,20 @@ tpconv_status tpconv_set_workspace_budget(tpconv_plan_t plan, size_t bytes);
 #define TPCONV_MATH_TF32 1
 tpconv_status tpconv_plan_set_math(tpconv_plan_t plan, int32_t math);
 
+/* Boundary layout of the node arrays x, out, grad_out, gg_x, grad_x and grad_grad_out
+ * (Sobek's wrapper accepts both):
+ *   TPCONV_LAYOUT_IR_MUL (default): each irrep block stored [2l+1][C], channels
+ *     contiguous, as described at the top of this header;
+ *   TPCONV_LAYOUT_MUL_IR: each block stored [C][2l+1] (components contiguous).
+ * With MUL_IR the passes convert their node inputs to ir_mul in workspace buffers and
+ * their node outputs back (one extra read and write of each node array); the workspace
+ * grows accordingly (tpconv_workspace_bytes accounts for it) and results equal the
+ * ir_mul results with the same permutation applied.  Edge arrays (Y, phi and their
+ * adjoints), W and positions are unaffected.  Any other value: TPCONV_ERR_UNSUPPORTED. */
+#define TPCONV_LAYOUT_IR_MUL 0
+#define TPCONV_LAYOUT_MUL_IR 1
+tpconv_status tpconv_plan_set_layout(tpconv_plan_t plan, int32_t layout);
+
 /* Workspace bytes needed by the passes in pass_mask for a graph of N nodes and E
  * edges.  The node-state part is bounded by the budget and does not grow with E;
  * backward adds 16 bytes per edge of position-gradient staging (only when a
