@@ -885,7 +885,6 @@ static tpconv_status forward_embedded_ir_mul(tpconv_plan_t P, int64_t N, int64_t
                                       size_t ws_bytes, struct CUstream_st* stream) {
   tpconv_status st = common_checks(P, N, E);
   if (st != TPCONV_OK) return st;
-  if (P->mode != TPCONV_UVW) return TPCONV_ERR_UNSUPPORTED;
   if (N == 0) return TPCONV_OK;
   st = check_ptrs({x, row_ptr, W, out}, {src, Y, phi});
   if (st != TPCONV_OK) return st;
@@ -898,6 +897,11 @@ static tpconv_status forward_embedded_ir_mul(tpconv_plan_t P, int64_t N, int64_t
   DevPlan D = P->dev;
   D.emb_Y = Y;
   D.emb_phi = phi;
+  if (P->mode == TPCONV_UVU) {
+    TPC_RUN(PC_UVU_FWD, 1, launch_uvu_fwd(D, P->bp_out, P->t_bo, 0, x, nullptr, nullptr, nullptr, row_ptr, src, W,
+                           nullptr, n, out, s));
+    return TPCONV_OK;
+  }
   TPC_RUN(PC_UVW_STATE, 1, attach_order(D, L, ws, n, row_ptr, s));
   if (!every_block_reached(P, true)) TPC_TRY(cudaMemsetAsync(out, 0, sizeof(float) * (size_t)N * P->dim_out, s));
   float* S = fptr(ws, L.state_a);
@@ -918,7 +922,6 @@ static tpconv_status backward_embedded_ir_mul(tpconv_plan_t P, int64_t N, int64_
                                        void* ws, size_t ws_bytes, struct CUstream_st* stream) {
   tpconv_status st = common_checks(P, N, E);
   if (st != TPCONV_OK) return st;
-  if (P->mode != TPCONV_UVW) return TPCONV_ERR_UNSUPPORTED;
   st = check_ptrs({}, {x, Y, phi, row_ptr, src, t_ptr, t_eid, t_dst, W, grad_out, grad_x, grad_W, grad_phi, grad_Y});
   if (st != TPCONV_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
@@ -941,6 +944,21 @@ static tpconv_status backward_embedded_ir_mul(tpconv_plan_t P, int64_t N, int64_
   D.emb_gY = grad_Y;
   D.emb_gphi = grad_phi;
   const int edge_split = (int)std::max<long long>(1, std::min<long long>(16, (4 * E / std::max<int64_t>(N, 1) + 31) / 32));
+  if (P->mode == TPCONV_UVU) {
+    if ((grad_phi || grad_Y) && E > 0)
+      TPC_RUN(PC_UVU_RECV_BWD, 1, launch_uvu_recv_bwd(D, P->t_in, x, nullptr, row_ptr, src, W, grad_out, n, gbuf,
+                                    edge_split, s));
+    if (grad_W) {
+      const int nr = std::min(kUvuRanges, n);
+      TPC_RUN(PC_UVU_GRADW, 1, launch_uvu_gradw(D, P->t_in, 0, x, nullptr, nullptr, nullptr, row_ptr, src, grad_out,
+                               n, nr, part, s));
+      TPC_RUN(PC_UVU_GRADW, 1, launch_reduce_partials(part, nr, (long long)P->K * P->n_w, grad_W, 0, s));
+    }
+    if (grad_x)
+      TPC_RUN(PC_UVU_SRC, 1, launch_uvu_src(D, P->bp_in, P->t_bi, 0, nullptr, nullptr, t_ptr, t_eid, t_dst, W,
+                             nullptr, grad_out, n, grad_x, s));
+    return TPCONV_OK;
+  }
   float* state = fptr(ws, L.state_a);
   if ((grad_phi || grad_Y) && E > 0) {
     TPC_RUN(PC_UVW_RECV_BWD, 1, attach_order(D, L, ws, n, row_ptr, s));
@@ -1122,7 +1140,7 @@ tpconv_status tpconv_double_backward(tpconv_plan_t P, int64_t N, int64_t E, cons
 tpconv_status tpconv_forward_embedded(tpconv_plan_t P, int64_t N, int64_t E, const float* x, const float* Y,
                                       const float* phi, const int32_t* row_ptr, const int32_t* src, const float* W,
                                       float* out, void* ws, size_t ws_bytes, struct CUstream_st* stream) {
-  if (!P || P->layout == TPCONV_LAYOUT_IR_MUL || N <= 0 || P->mode != TPCONV_UVW)
+  if (!P || P->layout == TPCONV_LAYOUT_IR_MUL || N <= 0)
     return forward_embedded_ir_mul(P, N, E, x, Y, phi, row_ptr, src, W, out, ws, ws_bytes, stream);
   if (!x || !out || N > 0x7ffffffe) return TPCONV_ERR_INVALID_ARG;
   ConvBufs B;
@@ -1144,7 +1162,7 @@ tpconv_status tpconv_backward_embedded(tpconv_plan_t P, int64_t N, int64_t E, co
                                        const float* W, const float* grad_out, float* grad_x, float* grad_W,
                                        float* grad_phi, float* grad_Y, void* ws, size_t ws_bytes,
                                        struct CUstream_st* stream) {
-  if (!P || P->layout == TPCONV_LAYOUT_IR_MUL || N <= 0 || P->mode != TPCONV_UVW)
+  if (!P || P->layout == TPCONV_LAYOUT_IR_MUL || N <= 0)
     return backward_embedded_ir_mul(P, N, E, x, Y, phi, row_ptr, src, t_ptr, t_eid, t_dst, W, grad_out, grad_x,
                                     grad_W, grad_phi, grad_Y, ws, ws_bytes, stream);
   if (!x || !grad_out || N > 0x7ffffffe) return TPCONV_ERR_INVALID_ARG;

@@ -27,9 +27,18 @@ struct USmem {
 
 template <int LS, int KP, bool TAN>
 __device__ __forceinline__ void uprep(const DevPlan& P, const float* __restrict__ pos,
-                                      const float* __restrict__ posdot, int i, int j, int store,
+                                      const float* __restrict__ posdot, int i, int j, int store, int e,
                                       USmem<KP>& sm, int w, int lane) {
   constexpr int RS = 2 * LS + 1;
+  if (!TAN && P.emb_Y) {
+    // embedded input: Y_e and phi_e of edge e as given
+    sm.j[w][lane] = store;
+#pragma unroll
+    for (int k = 0; k < RS; ++k) sm.Y[w][lane][k] = __ldg(P.emb_Y + (long long)e * P.n_sh + LS * LS + k);
+#pragma unroll
+    for (int q = 0; q < KP; ++q) sm.phi[w][lane][q] = q < P.K ? __ldg(P.emb_phi + (long long)e * P.K + q) : 0.f;
+    return;
+  }
   const EdgeGeo g = edge_geo(pos, i, j);
   const Pow3 pw(g.ux, g.uy, g.uz);
   float Y[RS], phi[KP], dphi[KP];
@@ -90,7 +99,7 @@ __device__ __forceinline__ void uvu_fwd_body(const DevPlan& P, const DevPath& p,
     const int ne = min(32, ee - e0);
     if (lane < ne) {
       const int j = __ldg(src + e0 + lane);
-      uprep<LS, KP, TAN>(P, pos, posdot, i, j, j, sm, w, lane);
+      uprep<LS, KP, TAN>(P, pos, posdot, i, j, j, e0 + lane, sm, w, lane);
     }
     __syncwarp();
     for (int t = 0; t < ne; ++t) {
@@ -261,11 +270,19 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32, 5)
     const int ne = min(32, ee - e0);
     if (w == 0 && lane < ne) {
       const int j = __ldg(src + e0 + lane);
-      const EdgeGeo g = edge_geo(pos, i, j);
-      const Pow3 pw(g.ux, g.uy, g.uz);
       float Y[16], phi[KP], dphi[KP];
-      sh_all(pw, Y);
-      radial<KP, false>(P, g.d, phi, dphi);
+      if (P.emb_Y) {   // embedded input: Y_e and phi_e as given
+        const long long e = e0 + lane;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) Y[k] = k < P.n_sh ? __ldg(P.emb_Y + e * P.n_sh + k) : 0.f;
+#pragma unroll
+        for (int q = 0; q < KP; ++q) phi[q] = q < P.K ? __ldg(P.emb_phi + e * P.K + q) : 0.f;
+      } else {
+        const EdgeGeo g = edge_geo(pos, i, j);
+        const Pow3 pw(g.ux, g.uy, g.uz);
+        sh_all(pw, Y);
+        radial<KP, false>(P, g.d, phi, dphi);
+      }
       sm.j[lane] = j;
 #pragma unroll
       for (int k = 0; k < 16; ++k) sm.Y[lane][k] = Y[k];
@@ -284,7 +301,24 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32, 5)
       });
     }
     __syncthreads();
-    if (w == 0 && lane < ne) {
+    if (w == 0 && lane < ne && (P.emb_gY || P.emb_gphi)) {
+      // embedded input: the edge-owned adjoints Y_bar (eq. 22) and phi_bar (eq. 20)
+      const long long e = e0 + lane;
+      if (P.emb_gY)
+        for (int k = 0; k < P.n_sh; ++k) {
+          float s = 0.f;
+#pragma unroll
+          for (int ww = 0; ww < WARPS_PER_CTA; ++ww) s += sm.accY[ww][lane][k];
+          P.emb_gY[e * P.n_sh + k] = s;
+        }
+      if (P.emb_gphi)
+        for (int q = 0; q < P.K; ++q) {
+          float s = 0.f;
+#pragma unroll
+          for (int ww = 0; ww < WARPS_PER_CTA; ++ww) s += sm.accphi[ww][lane][q];
+          P.emb_gphi[e * P.K + q] = s;
+        }
+    } else if (w == 0 && lane < ne) {
       const int j = sm.j[lane];
       const EdgeGeo g = edge_geo(pos, i, j);
       const Pow3 pw(g.ux, g.uy, g.uz);
@@ -353,7 +387,7 @@ __device__ __forceinline__ void uvu_gradw_body(const DevPlan& P, const DevPath& 
       const int ne = min(32, ee - e0);
       if (lane < ne) {
         const int j = __ldg(src + e0 + lane);
-        uprep<LS, KP, TAN>(P, pos, posdot, i, j, j, sm, w, lane);
+        uprep<LS, KP, TAN>(P, pos, posdot, i, j, j, e0 + lane, sm, w, lane);
       }
       __syncwarp();
       for (int t = 0; t < ne; ++t) {
@@ -451,7 +485,8 @@ __device__ __forceinline__ void uvu_src_body(const DevPlan& P, const DevPath& p,
     const int ne = min(32, ke - k0);
     if (lane < ne) {
       const int i = __ldg(t_dst + k0 + lane);
-      uprep<LS, KP, TAN>(P, pos, posdot, i, j, i, sm, w, lane);
+      const int e = P.emb_eid ? __ldg(P.emb_eid + k0 + lane) : 0;
+      uprep<LS, KP, TAN>(P, pos, posdot, i, j, i, e, sm, w, lane);
     }
     __syncwarp();
     for (int t = 0; t < ne; ++t) {

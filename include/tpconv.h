@@ -220,8 +220,8 @@ tpconv_status tpconv_double_backward(tpconv_plan_t plan, int64_t N, int64_t E, c
  * given per edge instead of computed from positions.  Y [E][(lmax+1)^2] holds the real
  * harmonics (or any per-edge vector in their place, same component order as the plan's
  * sh_lmax) and phi [E][K] any invariant edge embedding (e.g. a learned function of
- * |r_e|), both fp32 in receiver-CSR edge order.  uvw plans only (uvu:
- * TPCONV_ERR_UNSUPPORTED).  Workspace: as tpconv_forward / tpconv_backward.
+ * |r_e|), both fp32 in receiver-CSR edge order.  uvw and uvu plans.  Workspace: as
+ * tpconv_forward / tpconv_backward.
  *   forward: out as tpconv_forward (eqs. 11-13 with the given phi, Y).
  *   backward: grad_x (eq. 21), grad_W (eq. 19) and the edge-owned adjoints
  *     grad_phi [E][K] (eq. 20) and grad_Y [E][(lmax+1)^2] (eq. 22); each nullable;

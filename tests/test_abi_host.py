@@ -168,13 +168,6 @@ def test_plan_set_math_arguments():
     assert L.tpconv_plan_set_math(None, binding.MATH_FP32) == 1   # TPCONV_ERR_INVALID_ARG
 
 
-def test_embedded_interface_rejects_uvu():
-    L = binding.lib()
-    p = binding.Plan("4x0e+4x1o", 1, "4x0e+4x1o", "uvu", "gaussian", 8, 3.0, 0.0, 3.0)
-    assert L.tpconv_forward_embedded(p.handle, 4, 0, *([None] * 8), 0, None) == 3     # UNSUPPORTED
-    assert L.tpconv_backward_embedded(p.handle, 4, 0, *([None] * 15), 0, None) == 3
-
-
 def test_plan_set_layout_arguments():
     L = binding.lib()
     p = binding.Plan("8x0e+8x1o", 2, "8x0e+8x1o", "uvw", "bessel", 8, 3.0)

@@ -23,7 +23,7 @@ def torch():
     return torch
 
 
-@pytest.mark.parametrize("cfg,n", [(2, 160), (4, 200), (5, 160)])
+@pytest.mark.parametrize("cfg,n", [(2, 160), (4, 200), (5, 160), (3, 96)])
 def test_embedded_parity_arbitrary_inputs(torch, cfg, n):
     from equivariant_gnn_tensor_dst_b200 import binding
     p = Problem(cfg, n_nodes=n)
