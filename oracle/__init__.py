@@ -15,7 +15,8 @@ Convolutions" (arXiv 2607.18074), section 2:
   Clebsch-Gordan coupling tensors (eq. 5, eq. 32's ``c^pi``);
 * ``radial``  -- the radial embedding ``phi(|r|)`` (the pages leave its form open);
 * ``conv``    -- the materialised per-edge operator (eqs. 6-7, 11-13), its first-order
-  adjoints (eqs. 18-22) and second-order directional adjoints (eqs. 23-30), plus a
+  adjoints (eqs. 18-22), second-order directional adjoints (eqs. 23-30) and the double
+  backward's position gradient (through second derivatives of Y and phi), plus a
   second evaluation in the receiver-factorised streaming order (eqs. 16, 32-35) used
   only to check that both orders agree.
 
@@ -26,8 +27,9 @@ equivariance, spherical-harmonic identities (addition theorem, parity, explicit
 Cartesian forms, quadrature orthonormality), radial-basis orthonormality and cutoff
 smoothness, operator equivariance under random O(3) elements, translation and
 permutation invariance, the scalar-input special case, agreement of the two
-evaluation orders, and central finite differences for every gradient and for the
-double backward.  Parity unpinned: the absolute orientation of the real SH basis and
+evaluation orders, central finite differences for every gradient and for the
+double backward, and for the second derivatives of Y and phi a closed form, Euler's
+relation, the radial Hessian form and Hessian symmetry.  Parity unpinned: the absolute orientation of the real SH basis and
 the sign of each CG tensor are conventions the pages do not fix; every observable
 invariant checked above is independent of them.
 """

@@ -12,7 +12,9 @@ Sobek: Streaming Equivariant Tensor Product Convolutions (arXiv 2607.18074):
   the first-order adjoint direction set to zero, which is what an autograd engine
   asks for after a first backward taken with create_graph: for
       Lambda = <gg_x, x_bar> + <gg_pos, pos_bar> + <gg_A, A_bar>
-  it returns dLambda/dx (eq. 30), dLambda/dA (eq. 27) and dLambda/dm_bar (eq. 25).
+  it returns dLambda/dx (eq. 30), dLambda/dA (eq. 27) and dLambda/dm_bar (eq. 25);
+  double_backward_pos adds dLambda/dpos, the tangent of the first-order position
+  gradient, through the second derivatives of Y and phi.
 * forward_streaming: the receiver-factorised order of eqs. 16 and 32-35 (state S,
   then m = S A).  Used only by the self-test that both orders agree (eq. 15 = eq. 16).
 * forward_embedded / backward_embedded: the same with the edge embedding phi_e and the
@@ -337,6 +339,69 @@ def double_backward(plan, x, pos, row_ptr, src, A, grad_out, gg_x=None, gg_pos=N
         np.add.at(mdot, dst[eb], z)
         np.add.at(gx, src[eb], xbar2)
     return gx, gA, mdot
+
+
+def double_backward_pos(plan, x, pos, row_ptr, src, A, grad_out, gg_x=None, gg_pos=None,
+                        gg_A=None, edges=None):
+    """dLambda/dpos [N, 3] for the Lambda of double_backward.
+
+    The pages stop at the first-order terms of eqs. 23-31 (the position gradient of the
+    double backward needs second derivatives of Y and phi, which they do not write out).
+    Reading taken: pos_bar = sum_e (+g_e at src, -g_e at dst) with
+        g_e = (dphi/dr)^T phi_bar_e + (dY/dr)^T Y_bar_e            (eqs. 20, 22 + chain rule)
+    and, Lambda being the derivative of <m_bar, m> along (x_dot, pos_dot, A_dot),
+    dLambda/dpos = d/d eps pos_bar(x + eps x_dot, pos + eps pos_dot, A + eps A_dot):
+        g_dot_e = (dphi/dr)^T phi_bar_dot + (dY/dr)^T Y_bar_dot
+                  + (d2phi/dr2 . r_dot)^T phi_bar + (d2Y/dr2 . r_dot)^T Y_bar,
+    with phi_bar_dot = h_dot A^T + h A_dot^T (eqs. 20, 26) and Y_bar_dot the tangent of
+    eq. 22 (x -> x_dot, and w -> w_dot of eq. 23), scattered like g_e."""
+    x, pos, A, mbar = _f64(x), _f64(pos), _f64(A), _f64(grad_out)
+    src = np.asarray(src, dtype=np.int64)
+    dst = receivers_of(row_ptr)
+    N = pos.shape[0]
+    xd = np.zeros_like(x) if gg_x is None else _f64(gg_x)
+    pd = np.zeros_like(pos) if gg_pos is None else _f64(gg_pos)
+    Ad = np.zeros_like(A) if gg_A is None else _f64(gg_A)
+    gpos = np.zeros((N, 3))
+    for eb in _edge_batches(src.shape[0], plan.n_w, edges):
+        if eb.size == 0:
+            continue
+        r = pos[src[eb]] - pos[dst[eb]]                                          # eq. 8
+        Y, dY, HY = so3.sh_with_hessian(plan.lmax, r)
+        phi, dphi, Hphi = _radial.basis_with_hessian(plan.radial, r)
+        rdot = pd[src[eb]] - pd[dst[eb]]
+        Ydot = np.einsum("esk,ek->es", dY, rdot)
+        phidot = np.einsum("eqk,ek->eq", dphi, rdot)
+        w = _radial_project(phi, A)
+        wdot = _radial_project(phidot, A) + _radial_project(phi, Ad)            # eq. 23
+        xs, xds = x[src[eb]], xd[src[eb]]
+        mb_rows = mbar[dst[eb]]
+        h = np.zeros((eb.size, plan.n_w))
+        hdot = np.zeros((eb.size, plan.n_w))
+        ybar = np.zeros((eb.size, plan.n_sh))
+        ybardot = np.zeros((eb.size, plan.n_sh))
+        for p, c in zip(plan.paths, plan.coupling):
+            bi, bo = plan.blocks_in[p.block_in], plan.blocks_out[p.block_out]
+            sl = slice(p.l_sh ** 2, (p.l_sh + 1) ** 2)
+            xj, xdj = _block(xs, bi), _block(xds, bi)
+            mb = _block(mb_rows, bo)
+            C = _couple(c, xj, Y[:, sl])
+            Cdot = _couple(c, xdj, Y[:, sl]) + _couple(c, xj, Ydot[:, sl])       # eq. 24
+            sw = slice(p.w_offset, p.w_offset + p.w_count)
+            h[:, sw] = _edge_h(plan, mb, C)                                      # eq. 18
+            hdot[:, sw] = _edge_h(plan, mb, Cdot)                                # eq. 26
+            wp, wdp = _wslice(plan, p, w), _wslice(plan, p, wdot)
+            G, Gdot = _adjoint_weights(plan, mb, wp), _adjoint_weights(plan, mb, wdp)
+            ybar[:, sl] += _couple_adj_y(c, xj, G)                               # eq. 22
+            ybardot[:, sl] += _couple_adj_y(c, xdj, G) + _couple_adj_y(c, xj, Gdot)
+        phibar = h @ A.T                                                          # eq. 20
+        phibardot = hdot @ A.T + h @ Ad.T
+        gdot = (np.einsum("esk,es->ek", dY, ybardot) + np.einsum("eqk,eq->ek", dphi, phibardot)
+                + np.einsum("eskl,el,es->ek", HY, rdot, ybar)
+                + np.einsum("eqkl,el,eq->ek", Hphi, rdot, phibar))
+        np.add.at(gpos, src[eb], gdot)
+        np.add.at(gpos, dst[eb], -gdot)
+    return gpos
 
 
 # ---------------------------------------------------------------------------

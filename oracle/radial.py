@@ -15,7 +15,8 @@ section 2, after eq. 8) and fix neither its form nor its cutoff.  Readings taken
 * An edge with d >= r_c is kept and contributes exactly zero; a zero-length edge
   takes the d -> 0 limit of phi (sin(b pi d / r_c) / d -> b pi / r_c).
 
-All functions take Duals so that d phi / d r comes out exactly (see dual.py).
+All functions take Duals so that d phi / d r (and, for the double backward's position
+gradient, d^2 phi / dr^2) comes out exactly (see dual.py).
 """
 
 from dataclasses import dataclass
@@ -59,7 +60,8 @@ def basis_dual(spec, d, with_envelope=True):
     out = []
     if spec.kind == BESSEL:
         tiny = d.v < 1e-12
-        safe_d = Dual(np.where(tiny, 1.0, d.v), np.where(tiny[:, None], 0.0, d.g))
+        safe_d = Dual(np.where(tiny, 1.0, d.v), np.where(tiny[:, None], 0.0, d.g),
+                      None if d.h is None else np.where(tiny[:, None, None], 0.0, d.h))
         for b in range(1, spec.num_basis + 1):
             k = b * pi / spec.r_cut
             f = (safe_d * k).sin() / safe_d * sqrt(2.0 / spec.r_cut)
@@ -83,3 +85,14 @@ def basis_of_vectors(spec, r):
     _, d = unit_direction(np.atleast_2d(r))
     ds = basis_dual(spec, d)
     return np.stack([q.v for q in ds], axis=1), np.stack([q.g for q in ds], axis=1)
+
+
+def basis_with_hessian(spec, r):
+    """phi [E, K], d phi / d r [E, K, 3] and d^2 phi / dr^2 [E, K, 3, 3]."""
+    from .so3 import unit_direction
+    _, d = unit_direction(np.atleast_2d(r), second=True)
+    ds = basis_dual(spec, d)
+    n = d.v.shape[0]
+    hs = [q.h if q.h is not None else np.zeros((n, 3, 3)) for q in ds]
+    return (np.stack([q.v for q in ds], axis=1), np.stack([q.g for q in ds], axis=1),
+            np.stack(hs, axis=1))

@@ -62,26 +62,29 @@ def _horner(coeffs, z):
     return acc
 
 
-def unit_direction(r):
-    """r_hat = r / |r| as Duals (eq. 8).  A zero-length vector maps to r_hat = 0."""
+def unit_direction(r, second=False):
+    """r_hat = r / |r| as Duals (eq. 8).  A zero-length vector maps to r_hat = 0.
+    With ``second`` the Duals also carry Hessians in r."""
     from .dual import edge_vector
-    rx, ry, rz = edge_vector(r)
+    rx, ry, rz = edge_vector(r, second)
     d = (rx * rx + ry * ry + rz * rz).sqrt()
     n = d.v.shape[0]
     zero = d.v < 1e-12
-    safe = Dual(np.where(zero, 1.0, d.v), np.where(zero[:, None], 0.0, d.g))
+    safe = Dual(np.where(zero, 1.0, d.v), np.where(zero[:, None], 0.0, d.g),
+                None if d.h is None else np.where(zero[:, None, None], 0.0, d.h))
     z0 = Dual.const(0.0, n)
     hat = [(c / safe).where(~zero, z0) for c in (rx, ry, rz)]
     return hat, d
 
 
-def sh_dual(lmax, r):
+def sh_dual(lmax, r, second=False):
     """Real SH of the directions of r [E,3] for l = 0..lmax.
 
     Returns a list (length (lmax+1)^2, order l-major then m = -l..l) of Duals whose
-    gradient is d Y / d r (the raw edge vector, not r_hat).
+    gradient is d Y / d r (the raw edge vector, not r_hat); with ``second`` they also
+    carry d^2 Y / dr^2.
     """
-    (x, y, z), _ = unit_direction(r)
+    (x, y, z), _ = unit_direction(r, second)
     n = x.v.shape[0]
     # powers (x + i y)^m as (re, im) Duals
     re = [Dual.const(1.0, n)]
@@ -113,6 +116,15 @@ def sh_with_grad(lmax, r):
     """Values [E, n_sh] and d Y / d r as [E, n_sh, 3]."""
     ds = sh_dual(lmax, np.atleast_2d(r))
     return np.stack([d.v for d in ds], axis=1), np.stack([d.g for d in ds], axis=1)
+
+
+def sh_with_hessian(lmax, r):
+    """Values [E, n_sh], d Y / d r [E, n_sh, 3] and d^2 Y / dr^2 [E, n_sh, 3, 3]."""
+    ds = sh_dual(lmax, np.atleast_2d(r), second=True)
+    n = ds[0].v.shape[0]
+    hs = [d.h if d.h is not None else np.zeros((n, 3, 3)) for d in ds]
+    return (np.stack([d.v for d in ds], axis=1), np.stack([d.g for d in ds], axis=1),
+            np.stack(hs, axis=1))
 
 
 # ---------------------------------------------------------------------------
