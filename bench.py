@@ -478,10 +478,19 @@ def run_extras(args, dev, flush):
             def dbl_only():
                 binding.tpconv_double_backward(plan, x, pos, rp, src, *views, W, mbar, gg_pos=gg, ws=ws,
                                                outputs=(dx, dw, None))
+            dpos = torch.empty(N, 3, device=dev)
+
+            def dbl_with_pos():
+                # the same double backward also returning d loss / d pos (positions learned)
+                binding.tpconv_double_backward(plan, x, pos, rp, src, *views, W, mbar, gg_pos=gg, ws=ws,
+                                               need_pos=True, outputs=(dx, dw, None, dpos))
             ms_s = _timed(force_step, flush, steps, warm)
             ms_d = _timed(dbl_only, flush, steps, warm)
+            ms_dp = _timed(dbl_with_pos, flush, steps, warm)
             rec.update({"double_backward_ms": round(ms_d, 4),
                         "double_backward_edges_per_s": round(E / ms_d * 1e3, 1),
+                        "double_backward_with_pos_ms": round(ms_dp, 4),
+                        "double_backward_with_pos_edges_per_s": round(E / ms_dp * 1e3, 1),
                         "force_step_ms": round(ms_s, 4), "force_step_edges_per_s": round(E / ms_s * 1e3, 1)})
         out[str(cfg)] = rec
         del ws

@@ -56,7 +56,7 @@ SIGNATURES = {
     "tpconv_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int32)]),
     "tpconv_forward_no_alloc": (ctypes.c_int, [_c_p, _c_i64, _c_i64] + [_c_p] * 6 + [_c_p]),
 }
-PROF_CATEGORIES = 12
+PROF_CATEGORIES = 13
 
 _lib = None
 
@@ -304,7 +304,9 @@ def tpconv_backward_embedded(plan, x, Y, phi, row_ptr, src, t_ptr, t_eid, t_dst,
 
 def tpconv_double_backward(plan, x, pos, row_ptr, src, t_ptr, t_eid, t_dst, W, grad_out, gg_x=None,
                            gg_pos=None, gg_W=None, need_x=True, need_W=True, need_grad_out=True,
-                           ws=None, outputs=None, stream=None):
+                           need_pos=False, ws=None, outputs=None, stream=None):
+    """Returns (grad_x, grad_W, grad_grad_out), plus grad_pos [N, 3] when need_pos
+    (``outputs`` then has four entries)."""
     import torch
     N, E = pos.shape[0], src.numel()
     dev = x.device
@@ -312,16 +314,19 @@ def tpconv_double_backward(plan, x, pos, row_ptr, src, t_ptr, t_eid, t_dst, W, g
         gx = torch.empty(N, plan.dim_in, dtype=torch.float32, device=dev) if need_x else None
         gw = torch.empty(plan.num_basis, plan.weight_cols, dtype=torch.float32, device=dev) if need_W else None
         gg = torch.empty(N, plan.dim_out, dtype=torch.float32, device=dev) if need_grad_out else None
+        gp = torch.empty(N, 3, dtype=torch.float32, device=dev) if need_pos else None
+    elif need_pos:
+        gx, gw, gg, gp = outputs
     else:
-        gx, gw, gg = outputs
+        (gx, gw, gg), gp = outputs, None
     if ws is None:
         ws = workspace(plan.workspace_bytes(N, E, PASS_DOUBLE_BACKWARD), dev)
     check(lib().tpconv_double_backward(plan.handle, N, E, _ptr(x), _ptr(pos), _ptr(row_ptr), _ptr(src),
                                        _ptr(t_ptr), _ptr(t_eid), _ptr(t_dst), _ptr(W), _ptr(grad_out),
                                        _ptr(gg_x), _ptr(gg_pos), _ptr(gg_W), _ptr(gx), _ptr(gw), _ptr(gg),
-                                       None, _ptr(ws), ws.numel(), _stream(stream)),
+                                       _ptr(gp), _ptr(ws), ws.numel(), _stream(stream)),
           "tpconv_double_backward")
-    return gx, gw, gg
+    return (gx, gw, gg, gp) if need_pos else (gx, gw, gg)
 
 
 def tpconv_profile_begin(max_records=8192):

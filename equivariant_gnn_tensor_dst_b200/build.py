@@ -29,7 +29,8 @@ def _units():
                 for part in parts:
                     units.append((src, {"TPC_UNIT_KP": kp, "TPC_UNIT_MODE": mode,
                                         "TPC_UNIT_PART": _PARTS[part]}))
-            units.append((src, {"TPC_UNIT_KP": kp, "TPC_UNIT_MODE": 0, "TPC_UNIT_PART": _PARTS["RECV"]}))
+            for mode in (0, 1):
+                units.append((src, {"TPC_UNIT_KP": kp, "TPC_UNIT_MODE": mode, "TPC_UNIT_PART": _PARTS["RECV"]}))
     return units
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -127,13 +127,14 @@ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 enum ProfCat {
   PC_UVW_STATE = 0, PC_UVW_STATE_TAN, PC_UVW_RECV_BWD, PC_UVW_SRC, PC_UVW_SRC_TAN, PC_GEMM,
-  PC_UVU_FWD, PC_UVU_RECV_BWD, PC_UVU_GRADW, PC_UVU_SRC, PC_POS, PC_GRAPH, PC_COUNT
+  PC_UVU_FWD, PC_UVU_RECV_BWD, PC_UVU_GRADW, PC_UVU_SRC, PC_POS, PC_GRAPH, PC_RECV_TAN, PC_COUNT
 };
 static_assert(PC_COUNT == TPCONV_PROF_CATEGORIES, "category count");
 const char* const kProfNames[PC_COUNT] = {
     "uvw_receiver_state", "uvw_receiver_state_tangent", "uvw_receiver_backward", "uvw_source_state",
     "uvw_source_state_tangent", "channel_gemm", "uvu_forward", "uvu_receiver_backward",
-    "uvu_weight_gradient", "uvu_source_backward", "position_gradient", "graph"};
+    "uvu_weight_gradient", "uvu_source_backward", "position_gradient", "graph",
+    "receiver_backward_tangent"};
 
 struct Prof {
   std::mutex mu;
@@ -219,8 +220,8 @@ int chunk_for(size_t budget_floats, long long fixed, long long per_node, long lo
 }
 
 // Workspace of one pass.  The scratch budget covers the node states of a receiver (or
-// source) range and the split-K slices of the channel contractions; backward adds the
-// per-edge position-gradient staging (16 bytes per edge) on top.
+// source) range and the split-K slices of the channel contractions; backward and double
+// backward add the per-edge position-gradient staging (16 bytes per edge) on top.
 Layout make_layout(const tpconv_plan* P, long long N, long long E, uint32_t pass) {
   Layout L;
   size_t off = 0;
@@ -249,7 +250,7 @@ Layout make_layout(const tpconv_plan* P, long long N, long long E, uint32_t pass
       off += align256(size_t(4) * kUvuRanges * P->K * (long long)P->n_w);
     }
   }
-  if (pass == TPCONV_PASS_BACKWARD) {
+  if (pass == TPCONV_PASS_BACKWARD || pass == TPCONV_PASS_DOUBLE_BACKWARD) {
     L.has_gbuf = true;
     L.gbuf = off;
     off += align256(size_t(16) * std::max<long long>(E, 1));
@@ -993,9 +994,8 @@ static tpconv_status double_backward_ir_mul(tpconv_plan_t P, int64_t N, int64_t 
                                      struct CUstream_st* stream) {
   tpconv_status st = common_checks(P, N, E);
   if (st != TPCONV_OK) return st;
-  if (grad_pos) return TPCONV_ERR_UNSUPPORTED;
   st = check_ptrs({}, {x, pos, row_ptr, src, t_ptr, t_eid, t_dst, W, grad_out, gg_x, gg_pos, gg_W, grad_x,
-                       grad_W, grad_grad_out});
+                       grad_W, grad_grad_out, grad_pos});
   if (st != TPCONV_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
   if (N == 0) {
@@ -1004,12 +1004,17 @@ static tpconv_status double_backward_ir_mul(tpconv_plan_t P, int64_t N, int64_t 
   }
   if (!x || !pos || !row_ptr || !W || !grad_out || (E > 0 && !src)) return TPCONV_ERR_INVALID_ARG;
   if (grad_x && (!t_ptr || (E > 0 && !t_dst))) return TPCONV_ERR_INVALID_ARG;
+  if (grad_pos && (!t_ptr || (E > 0 && !t_eid))) return TPCONV_ERR_INVALID_ARG;
   const Layout L = make_layout(P, N, E, TPCONV_PASS_DOUBLE_BACKWARD);
   st = check_ws(L, ws, ws_bytes);
   if (st != TPCONV_OK) return st;
   const int n = (int)N;
   float* part = fptr(ws, L.part);
   const bool tan_xp = gg_x || gg_pos;
+  float4* gbuf = reinterpret_cast<float4*>(static_cast<char*>(ws) + L.gbuf);
+  const int edge_split = (int)std::max<long long>(1, std::min<long long>(16, (4 * E / std::max<int64_t>(N, 1) + 31) / 32));
+  const bool any_tan = gg_x || gg_pos || gg_W;
+  if (grad_pos && !any_tan) TPC_TRY(cudaMemsetAsync(grad_pos, 0, sizeof(float) * 3 * (size_t)N, s));
 
   if (P->mode == TPCONV_UVU) {
     if (grad_grad_out)
@@ -1024,6 +1029,12 @@ static tpconv_status double_backward_ir_mul(tpconv_plan_t P, int64_t N, int64_t 
     if (grad_x)
       TPC_RUN(PC_UVU_SRC, 1, launch_uvu_src(P->dev, P->bp_in, P->t_bi, 1, pos, gg_pos, t_ptr, t_eid, t_dst, W, gg_W,
                              grad_out, n, grad_x, s));
+    if (grad_pos && any_tan) {
+      // the tangent of the first-order position gradient (second derivatives of Y, phi)
+      TPC_RUN(PC_RECV_TAN, 1, launch_uvu_recv_dbl(P->dev, P->t_in, x, gg_x, pos, gg_pos, row_ptr, src, W, gg_W,
+                                                 grad_out, n, gbuf, edge_split, s));
+      TPC_RUN(PC_POS, 1, launch_pos_finish(n, row_ptr, t_ptr, t_eid, gbuf, grad_pos, s));
+    }
     return TPCONV_OK;
   }
 
@@ -1060,6 +1071,21 @@ static tpconv_status double_backward_ir_mul(tpconv_plan_t P, int64_t N, int64_t 
         TPC_RUN(PC_GEMM, 0, gemm_xbar(P, gg_pos ? sa : nullptr, W, gg_W ? sb : nullptr, gg_W, grad_x, n0, cn, part, s));
       }
     }
+  }
+  if (grad_pos && any_tan) {
+    // the tangent of the first-order position gradient: per receiver range S_bar = m_bar A^T
+    // (sa) and S_bar_dot = m_bar A_dot^T (sb), then per edge through second derivatives
+    // of Y and phi, then the fixed-order scatter of the backward
+    DevPlan D = P->dev;
+    TPC_RUN(PC_RECV_TAN, 1, attach_order(D, L, ws, n, row_ptr, s));
+    for (int n0 = 0; n0 < n; n0 += L.recv_chunk) {
+      const int cn = std::min(L.recv_chunk, n - n0);
+      TPC_RUN(PC_GEMM, 0, gemm_sbar(P, grad_out, W, sa, n0, cn, s));
+      if (gg_W) TPC_RUN(PC_GEMM, 0, gemm_sbar(P, grad_out, gg_W, sb, n0, cn, s));
+      TPC_RUN(PC_RECV_TAN, 1, launch_uvw_recv_dbl(D, P->t_in, x, gg_x, pos, gg_pos, row_ptr, src, sa,
+                                                 gg_W ? sb : nullptr, n0, cn, gbuf, edge_split, s));
+    }
+    TPC_RUN(PC_POS, 1, launch_pos_finish(n, row_ptr, t_ptr, t_eid, gbuf, grad_pos, s));
   }
   return TPCONV_OK;
 }

@@ -68,6 +68,30 @@ __device__ __forceinline__ void sh_block_vjp(const Pow3& p, const float* w, floa
   }
 }
 
+// v += sum_k w[k] (Hess P_k) t  for block L (the derivative of sh_block_vjp's sum along
+// a direction t of the unit vector)
+template <int L>
+__device__ __forceinline__ void sh_block_hvp(const Pow3& p, const float* w, float tx, float ty, float tz,
+                                             float& gx, float& gy, float& gz) {
+  using T = tpc_tab::SH<L>;
+#pragma unroll
+  for (int t = 0; t < T::nterm; ++t) {
+    const int ex = T::ex(t), ey = T::ey(t), ez = T::ez(t);
+    const float c = T::coef(t) * w[T::k(t)];
+    const int ex1 = ex > 0 ? ex - 1 : 0, ey1 = ey > 0 ? ey - 1 : 0, ez1 = ez > 0 ? ez - 1 : 0;
+    const int ex2 = ex > 1 ? ex - 2 : 0, ey2 = ey > 1 ? ey - 2 : 0, ez2 = ez > 1 ? ez - 2 : 0;
+    const float hxx = ex > 1 ? (float)(ex * (ex - 1)) * p.x[ex2] * p.y[ey] * p.z[ez] : 0.f;
+    const float hyy = ey > 1 ? (float)(ey * (ey - 1)) * p.x[ex] * p.y[ey2] * p.z[ez] : 0.f;
+    const float hzz = ez > 1 ? (float)(ez * (ez - 1)) * p.x[ex] * p.y[ey] * p.z[ez2] : 0.f;
+    const float hxy = (ex > 0 && ey > 0) ? (float)(ex * ey) * p.x[ex1] * p.y[ey1] * p.z[ez] : 0.f;
+    const float hxz = (ex > 0 && ez > 0) ? (float)(ex * ez) * p.x[ex1] * p.y[ey] * p.z[ez1] : 0.f;
+    const float hyz = (ey > 0 && ez > 0) ? (float)(ey * ez) * p.x[ex] * p.y[ey1] * p.z[ez1] : 0.f;
+    gx = fmaf(c, hxx * tx + hxy * ty + hxz * tz, gx);
+    gy = fmaf(c, hxy * tx + hyy * ty + hyz * tz, gy);
+    gz = fmaf(c, hxz * tx + hyz * ty + hzz * tz, gz);
+  }
+}
+
 // all blocks l = 0..3 into Y[16]
 __device__ __forceinline__ void sh_all(const Pow3& p, float* Y) {
   sh_block<0>(p, Y);
@@ -81,6 +105,21 @@ __device__ __forceinline__ void sh_vjp_all(const Pow3& p, const float* w, float&
   sh_block_vjp<1>(p, w + 1, gx, gy, gz);
   sh_block_vjp<2>(p, w + 4, gx, gy, gz);
   sh_block_vjp<3>(p, w + 9, gx, gy, gz);
+}
+
+__device__ __forceinline__ void sh_hvp_all(const Pow3& p, const float* w, float tx, float ty, float tz,
+                                           float& gx, float& gy, float& gz) {
+  sh_block_hvp<1>(p, w + 1, tx, ty, tz, gx, gy, gz);
+  sh_block_hvp<2>(p, w + 4, tx, ty, tz, gx, gy, gz);
+  sh_block_hvp<3>(p, w + 9, tx, ty, tz, gx, gy, gz);
+}
+
+// Yd[k] = grad P_k . t for all blocks l = 0..3
+__device__ __forceinline__ void sh_dir_all(const Pow3& p, float tx, float ty, float tz, float* Yd) {
+  Yd[0] = 0.f;
+  sh_block_dir<1>(p, tx, ty, tz, Yd + 1);
+  sh_block_dir<2>(p, tx, ty, tz, Yd + 4);
+  sh_block_dir<3>(p, tx, ty, tz, Yd + 9);
 }
 
 template <int L>
@@ -170,6 +209,207 @@ __device__ __forceinline__ void radial(const DevPlan& P, float d, float* phi, fl
       if (DERIV) dphi[q] = df;
     }
   }
+}
+
+// phi_q(d) with its first and second derivatives in d (the double backward's position
+// gradient).  The same basis as radial(); the envelope's second derivative is
+// u''(t) = -a p (p-1) t^(p-2) + b (p+1) p t^(p-1) - c (p+2)(p+1) t^p  for t < 1, else 0.
+template <int KP>
+__device__ __forceinline__ void radial2(const DevPlan& P, float d, float* phi, float* dphi, float* d2phi) {
+  const float t = d * P.inv_r_cut;
+  float u = 0.f, du = 0.f, ddu = 0.f;
+  if (t < 1.f) {
+    envelope(P, t, u, du);
+    const int pp = P.poly_p;
+    const float p = (float)pp;
+    float tpm1 = 1.f;
+    for (int k = 0; k < pp - 1; ++k) tpm1 *= t;
+    float tpm2 = 0.f;
+    if (pp >= 2) {
+      tpm2 = 1.f;
+      for (int k = 0; k < pp - 2; ++k) tpm2 *= t;
+    }
+    ddu = -P.env_a * p * (p - 1.f) * tpm2 + P.env_b * (p + 1.f) * p * tpm1 - P.env_c * (p + 2.f) * (p + 1.f) * tpm1 * t;
+  }
+  du *= P.inv_r_cut;
+  ddu *= P.inv_r_cut * P.inv_r_cut;
+  if (P.radial_kind == 0) {
+    const float inv_d = d > 0.f ? 1.f / d : 0.f;
+#pragma unroll
+    for (int q = 0; q < KP; ++q) {
+      float f = 0.f, df = 0.f, d2f = 0.f;
+      if (q < P.K && t < 1.f) {
+        const float b = (float)(q + 1);
+        const float k = b * 3.14159265358979f * P.inv_r_cut;
+        if (d > 0.f) {
+          float s, c;
+          sincospif(b * t, &s, &c);
+          const float base = P.bessel_pref * s * inv_d;
+          const float g1 = (k * c - s * inv_d) * inv_d;   // d/dd of sin(kd)/d
+          const float dbase = P.bessel_pref * g1;
+          const float d2base = P.bessel_pref * (-k * k * s - 2.f * g1) * inv_d;
+          f = base * u;
+          df = dbase * u + base * du;
+          d2f = d2base * u + 2.f * dbase * du + base * ddu;
+        } else {
+          f = P.bessel_pref * k * u;
+        }
+      }
+      phi[q] = f;
+      dphi[q] = df;
+      d2phi[q] = d2f;
+    }
+  } else {
+#pragma unroll
+    for (int q = 0; q < KP; ++q) {
+      float f = 0.f, df = 0.f, d2f = 0.f;
+      if (q < P.K && t < 1.f) {
+        const float dm = d - (P.g_mu0 + P.g_step * (float)q);
+        const float g2 = P.g_inv_sigma2;
+        const float e = expf(-0.5f * dm * dm * g2);
+        const float e1 = -e * dm * g2;
+        const float e2 = e * (dm * dm * g2 * g2 - g2);
+        f = e * u;
+        df = e1 * u + e * du;
+        d2f = e2 * u + 2.f * e1 * du + e * ddu;
+      }
+      phi[q] = f;
+      dphi[q] = df;
+      d2phi[q] = d2f;
+    }
+  }
+}
+
+// The tangent of the first-order position gradient of one edge (double backward):
+//   g = (dphi/dr)^T phi_bar + (dY/dr)^T Y_bar, with phi(|r|) and Y(r / |r|),
+// differentiated along r_dot (v) with phi_bar and Y_bar moving by phi_bar_dot, Y_bar_dot:
+//   radial part  (sum pbd phi' + d_dot sum pb phi'') r_hat + (sum pb phi') r_hat_dot
+//   harmonic part, with G = grad_u F . Y_bar and Gt = grad_u F . Y_bar_dot + Hess_u F (Y_bar) r_hat_dot:
+//     (1/d) [Gt - (r_hat.Gt) r_hat - (r_hat_dot.G) r_hat - (r_hat.G) r_hat_dot - (d_dot/d)(G - (r_hat.G) r_hat)]
+// where d_dot = r_hat . v and r_hat_dot = (v - d_dot r_hat) / d.  Zero for a zero-length edge.
+template <int KP>
+__device__ __forceinline__ float3 position_tangent(const DevPlan& P, const EdgeGeo& g, float vx, float vy, float vz,
+                                                   const float* Yb, const float* Ybd, const float* pb,
+                                                   const float* pbd) {
+  const Pow3 pw(g.ux, g.uy, g.uz);
+  float phi[KP], dphi[KP], d2phi[KP];
+  radial2<KP>(P, g.d, phi, dphi, d2phi);
+  const float dd = g.ux * vx + g.uy * vy + g.uz * vz;
+  const float tx = (vx - dd * g.ux) * g.inv_d, ty = (vy - dd * g.uy) * g.inv_d, tz = (vz - dd * g.uz) * g.inv_d;
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f;
+#pragma unroll
+  for (int q = 0; q < KP; ++q) {
+    s0 = fmaf(pb[q], dphi[q], s0);
+    s1 = fmaf(pbd[q], dphi[q], s1);
+    s2 = fmaf(pb[q], d2phi[q], s2);
+  }
+  s1 = fmaf(dd, s2, s1);
+  float Gx = 0.f, Gy = 0.f, Gz = 0.f, Hx = 0.f, Hy = 0.f, Hz = 0.f;
+  sh_vjp_all(pw, Yb, Gx, Gy, Gz);
+  sh_vjp_all(pw, Ybd, Hx, Hy, Hz);
+  sh_hvp_all(pw, Yb, tx, ty, tz, Hx, Hy, Hz);
+  const float uG = g.ux * Gx + g.uy * Gy + g.uz * Gz;
+  const float uH = g.ux * Hx + g.uy * Hy + g.uz * Hz;
+  const float tG = tx * Gx + ty * Gy + tz * Gz;
+  const float k = dd * g.inv_d;
+  float3 o;
+  o.x = s1 * g.ux + s0 * tx + g.inv_d * (Hx - uH * g.ux - tG * g.ux - uG * tx - k * (Gx - uG * g.ux));
+  o.y = s1 * g.uy + s0 * ty + g.inv_d * (Hy - uH * g.uy - tG * g.uy - uG * ty - k * (Gy - uG * g.uy));
+  o.z = s1 * g.uz + s0 * tz + g.inv_d * (Hz - uH * g.uz - tG * g.uz - uG * tz - k * (Gz - uG * g.uz));
+  return o;
+}
+
+// Per-CTA edge data of the double backward's position-gradient kernels (one 32-edge
+// chunk of a receiver): Y, phi and their tangents along r_dot, and per-warp partial sums
+// of phi_bar, Y_bar and their tangents, combined in warp order.
+template <int KP>
+struct RecvDblSmem {
+  int j[32];
+  float Y[32][16], Yd[32][16];
+  float phi[32][KP], phid[32][KP];
+  float accY[WARPS_PER_CTA][32][16], accYd[WARPS_PER_CTA][32][16];
+  float accphi[WARPS_PER_CTA][32][KP], accphid[WARPS_PER_CTA][32][KP];
+};
+
+__device__ __forceinline__ float3 edge_rdot(const float* __restrict__ posdot, int i, int j) {
+  if (!posdot) return make_float3(0.f, 0.f, 0.f);
+  return make_float3(__ldg(posdot + 3 * j) - __ldg(posdot + 3 * i), __ldg(posdot + 3 * j + 1) - __ldg(posdot + 3 * i + 1),
+                     __ldg(posdot + 3 * j + 2) - __ldg(posdot + 3 * i + 2));
+}
+
+// lane-per-edge staging of edges e0 .. e0+ne-1 of receiver i (warp 0), and zeroed sums
+template <int KP>
+__device__ __forceinline__ void recv_dbl_prep(const DevPlan& P, const float* __restrict__ pos,
+                                              const float* __restrict__ posdot, const int* __restrict__ src,
+                                              int i, int e0, int ne, RecvDblSmem<KP>& sm) {
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (w == 0 && lane < ne) {
+    const int j = __ldg(src + e0 + lane);
+    const EdgeGeo g = edge_geo(pos, i, j);
+    const Pow3 pw(g.ux, g.uy, g.uz);
+    float Y[16], Yd[16], phi[KP], dphi[KP];
+    sh_all(pw, Y);
+    radial<KP, true>(P, g.d, phi, dphi);
+    const float3 v = edge_rdot(posdot, i, j);
+    const float dd = g.ux * v.x + g.uy * v.y + g.uz * v.z;   // d|r| along r_dot
+    sh_dir_all(pw, (v.x - dd * g.ux) * g.inv_d, (v.y - dd * g.uy) * g.inv_d, (v.z - dd * g.uz) * g.inv_d, Yd);
+    sm.j[lane] = j;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      sm.Y[lane][k] = Y[k];
+      sm.Yd[lane][k] = Yd[k];
+    }
+#pragma unroll
+    for (int q = 0; q < KP; ++q) {
+      sm.phi[lane][q] = phi[q];
+      sm.phid[lane][q] = dphi[q] * dd;
+    }
+  }
+  for (int k = threadIdx.x; k < WARPS_PER_CTA * 32 * 16; k += blockDim.x) {
+    (&sm.accY[0][0][0])[k] = 0.f;
+    (&sm.accYd[0][0][0])[k] = 0.f;
+  }
+  for (int k = threadIdx.x; k < WARPS_PER_CTA * 32 * KP; k += blockDim.x) {
+    (&sm.accphi[0][0][0])[k] = 0.f;
+    (&sm.accphid[0][0][0])[k] = 0.f;
+  }
+}
+
+// per edge (warp 0): the warp-ordered sums, then the tangent of g_e into gbuf
+template <int KP>
+__device__ __forceinline__ void recv_dbl_finish(const DevPlan& P, const float* __restrict__ pos,
+                                                const float* __restrict__ posdot, int i, int e0, int ne,
+                                                const RecvDblSmem<KP>& sm, float4* gbuf) {
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (w != 0 || lane >= ne) return;
+  const int j = sm.j[lane];
+  const EdgeGeo g = edge_geo(pos, i, j);
+  const float3 v = edge_rdot(posdot, i, j);
+  float Yb[16], Ybd[16], pb[KP], pbd[KP];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    float a = 0.f, b = 0.f;
+#pragma unroll
+    for (int ww = 0; ww < WARPS_PER_CTA; ++ww) {
+      a += sm.accY[ww][lane][k];
+      b += sm.accYd[ww][lane][k];
+    }
+    Yb[k] = a;
+    Ybd[k] = b;
+  }
+#pragma unroll
+  for (int q = 0; q < KP; ++q) {
+    float a = 0.f, b = 0.f;
+#pragma unroll
+    for (int ww = 0; ww < WARPS_PER_CTA; ++ww) {
+      a += sm.accphi[ww][lane][q];
+      b += sm.accphid[ww][lane][q];
+    }
+    pb[q] = a;
+    pbd[q] = b;
+  }
+  const float3 o = position_tangent<KP>(P, g, v.x, v.y, v.z, Yb, Ybd, pb, pbd);
+  gbuf[e0 + lane] = make_float4(o.x, o.y, o.z, 0.f);
 }
 
 // ---------------------------------------------------------------------------

@@ -120,6 +120,16 @@ template <int KP>
 cudaError_t run_uvw_recv_bwd(const DevPlan& P, const Tasks& T, const float* x, const float* pos,
                              const int* row_ptr, const int* src, const float* Sbar, int node0,
                              int n_nodes, float4* gbuf, int edge_split, cudaStream_t s);
+template <int KP>
+cudaError_t run_uvw_recv_dbl(const DevPlan& P, const Tasks& T, const float* x, const float* xdot,
+                             const float* pos, const float* posdot, const int* row_ptr, const int* src,
+                             const float* Sbar, const float* Sbard, int node0, int n_nodes, float4* gbuf,
+                             int edge_split, cudaStream_t s);
+template <int KP>
+cudaError_t run_uvu_recv_dbl(const DevPlan& P, const Tasks& T, const float* x, const float* xdot,
+                             const float* pos, const float* posdot, const int* row_ptr, const int* src,
+                             const float* W, const float* Wdot, const float* grad_out, int N, float4* gbuf,
+                             int edge_split, cudaStream_t s);
 template <int KP, int MODE>
 cudaError_t run_uvw_src_state(const DevPlan& P, const Tasks& T, const float* pos,
                               const float* posdot, const int* t_ptr, const int* t_dst,
@@ -160,6 +170,15 @@ cudaError_t launch_uvw_state(const DevPlan& P, const Tasks& T, int mode, const f
 cudaError_t launch_uvw_recv_bwd(const DevPlan& P, const Tasks& T, const float* x,
                                 const float* pos, const int* row_ptr, const int* src,
                                 const float* Sbar, int node0, int n_nodes, float4* gbuf,
+                                int edge_split, cudaStream_t s);
+// double backward position gradient: per-edge tangent of g_e into gbuf (then pos_finish)
+cudaError_t launch_uvw_recv_dbl(const DevPlan& P, const Tasks& T, const float* x, const float* xdot,
+                                const float* pos, const float* posdot, const int* row_ptr, const int* src,
+                                const float* Sbar, const float* Sbard, int node0, int n_nodes, float4* gbuf,
+                                int edge_split, cudaStream_t s);
+cudaError_t launch_uvu_recv_dbl(const DevPlan& P, const Tasks& T, const float* x, const float* xdot,
+                                const float* pos, const float* posdot, const int* row_ptr, const int* src,
+                                const float* W, const float* Wdot, const float* grad_out, int N, float4* gbuf,
                                 int edge_split, cudaStream_t s);
 cudaError_t launch_uvw_src_state(const DevPlan& P, const Tasks& T, int mode,
                                  const float* pos, const float* posdot, const int* t_ptr,

@@ -26,6 +26,28 @@ cudaError_t launch_uvw_recv_bwd(const DevPlan& P, const Tasks& T, const float* x
   return run_uvw_recv_bwd<16>(P, T, x, pos, row_ptr, src, Sbar, node0, n_nodes, gbuf, edge_split, s);
 }
 
+cudaError_t launch_uvw_recv_dbl(const DevPlan& P, const Tasks& T, const float* x, const float* xdot,
+                                const float* pos, const float* posdot, const int* row_ptr, const int* src,
+                                const float* Sbar, const float* Sbard, int node0, int n_nodes, float4* gbuf,
+                                int edge_split, cudaStream_t s) {
+  if (n_nodes <= 0) return cudaSuccess;
+  if (edge_split < 1) edge_split = 1;
+  if (P.K <= 8)
+    return run_uvw_recv_dbl<8>(P, T, x, xdot, pos, posdot, row_ptr, src, Sbar, Sbard, node0, n_nodes, gbuf, edge_split, s);
+  return run_uvw_recv_dbl<16>(P, T, x, xdot, pos, posdot, row_ptr, src, Sbar, Sbard, node0, n_nodes, gbuf, edge_split, s);
+}
+
+cudaError_t launch_uvu_recv_dbl(const DevPlan& P, const Tasks& T, const float* x, const float* xdot,
+                                const float* pos, const float* posdot, const int* row_ptr, const int* src,
+                                const float* W, const float* Wdot, const float* grad_out, int N, float4* gbuf,
+                                int edge_split, cudaStream_t s) {
+  if (N <= 0) return cudaSuccess;
+  if (edge_split < 1) edge_split = 1;
+  if (P.K <= 8)
+    return run_uvu_recv_dbl<8>(P, T, x, xdot, pos, posdot, row_ptr, src, W, Wdot, grad_out, N, gbuf, edge_split, s);
+  return run_uvu_recv_dbl<16>(P, T, x, xdot, pos, posdot, row_ptr, src, W, Wdot, grad_out, N, gbuf, edge_split, s);
+}
+
 cudaError_t launch_uvw_src_state(const DevPlan& P, const Tasks& T, int mode,
                                  const float* pos, const float* posdot, const int* t_ptr,
                                  const int* t_eid, const int* t_dst, const float* grad_out,

@@ -161,8 +161,8 @@ tpconv_status tpconv_plan_set_layout(tpconv_plan_t plan, int32_t layout);
 
 /* Workspace bytes needed by the passes in pass_mask for a graph of N nodes and E
  * edges.  The node-state part is bounded by the budget and does not grow with E;
- * backward adds 16 bytes per edge of position-gradient staging (only when a
- * position gradient is requested it is used).                                       */
+ * backward and double backward add 16 bytes per edge of position-gradient staging
+ * (used only when a position gradient is requested).                                 */
 tpconv_status tpconv_workspace_bytes(tpconv_plan_t plan, int64_t N, int64_t E,
                                      uint32_t pass_mask, size_t* bytes);
 
@@ -203,10 +203,14 @@ tpconv_status tpconv_backward(tpconv_plan_t plan, int64_t N, int64_t E, const fl
 /* Double backward.  With (x_bar, pos_bar, W_bar) = backward(x, pos, W, grad_out) and
  *   Lambda = <gg_x, x_bar> + <gg_pos, pos_bar> + <gg_W, W_bar>,
  * returns grad_x = dLambda/dx (eq. 30), grad_W = dLambda/dW (eq. 27) and
- * grad_grad_out = dLambda/dgrad_out (eq. 25, the forward tangent).  This is what an
- * autograd engine requests after a first backward taken with create_graph.  Tangents
- * gg_* may be NULL (zero); outputs may be NULL (skipped).  grad_pos (dLambda/dpos)
- * must be NULL: it is not provided (TPCONV_ERR_UNSUPPORTED otherwise).              */
+ * grad_grad_out = dLambda/dgrad_out (eq. 25, the forward tangent) and
+ * grad_pos = dLambda/dpos [N][3].  This is what an autograd engine requests after a
+ * first backward taken with create_graph.  The pages stop at the first-order terms;
+ * grad_pos is the tangent of the backward's per-edge position gradient
+ * g_e = (dphi/dr)^T phi_bar + (dY/dr)^T Y_bar along (gg_x, gg_pos, gg_W), which needs
+ * the second derivatives of Y(r_hat) and phi(|r|), scattered like g_e.  Tangents gg_*
+ * may be NULL (zero); outputs may be NULL (skipped).  The source view is required for
+ * grad_x (t_ptr, t_dst) and grad_pos (t_ptr, t_eid).                                 */
 tpconv_status tpconv_double_backward(tpconv_plan_t plan, int64_t N, int64_t E, const float* x,
                                      const float* pos, const int32_t* row_ptr,
                                      const int32_t* src, const int32_t* t_ptr,
@@ -269,7 +273,7 @@ tpconv_status tpconv_forward_no_alloc(tpconv_plan_t plan, int64_t N, int64_t E, 
  * total device milliseconds and launch counts into ms[n] / launches[n] (either may be
  * NULL; n <= TPCONV_PROF_CATEGORIES) and disables recording.  Not for use during
  * stream capture.                                                                     */
-#define TPCONV_PROF_CATEGORIES 12
+#define TPCONV_PROF_CATEGORIES 13
 
 /* Reads and clears the library's device error word (0 = fine; nonzero = a bounded wait
  * inside a tensor-core kernel gave up, so results of that launch are invalid).

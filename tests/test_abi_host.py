@@ -136,12 +136,27 @@ def test_forward_rejects_bad_arguments_before_launch():
     assert L.tpconv_forward(lp.handle, 0, 0, None, None, None, None, None, None, None, 0, None) == 0
 
 
-def test_double_backward_position_output_unsupported():
+def test_double_backward_position_output_checks():
+    """dLambda/dpos needs the source view's t_ptr and t_eid, takes 16-byte aligned
+    output, and its per-edge staging is counted in the double backward's workspace
+    (16 bytes per edge).  Every case returns before any launch."""
     L = binding.lib()
     lp = _lib_plan(5)
     fake = ctypes.c_void_p(1 << 20)
-    st = L.tpconv_double_backward(lp.handle, 10, 20, *([fake] * 17), 1 << 30, None)
-    assert st == 3
+    mis = ctypes.c_void_p((1 << 20) + 4)
+    ptrs = [fake] * 17          # x, pos, row_ptr, src, t_ptr, t_eid, t_dst, W, grad_out,
+    #                             gg_x, gg_pos, gg_W, grad_x, grad_W, grad_grad_out, grad_pos, ws
+    ptrs[5] = None              # t_eid missing
+    assert L.tpconv_double_backward(lp.handle, 10, 20, *ptrs, 1 << 30, None) == 1
+    ptrs = [fake] * 17
+    ptrs[15] = mis              # misaligned grad_pos
+    assert L.tpconv_double_backward(lp.handle, 10, 20, *ptrs, 1 << 30, None) == 5
+    ptrs = [fake] * 17          # workspace one byte short
+    need = lp.workspace_bytes(10, 20, binding.PASS_DOUBLE_BACKWARD)
+    assert L.tpconv_double_backward(lp.handle, 10, 20, *ptrs, need - 1, None) == 4
+    a = lp.workspace_bytes(1000, 64000, binding.PASS_DOUBLE_BACKWARD)
+    b = lp.workspace_bytes(1000, 128000, binding.PASS_DOUBLE_BACKWARD)
+    assert b - a == 16 * 64000
 
 
 def test_status_strings():
