@@ -487,6 +487,21 @@ def run_extras(args, dev, flush):
             ms_s = _timed(force_step, flush, steps, warm)
             ms_d = _timed(dbl_only, flush, steps, warm)
             ms_dp = _timed(dbl_with_pos, flush, steps, warm)
+            # the tangent receiver kernel of d loss / d pos against the derived FP32 peak: with
+            # gg_pos alone it does the receiver backward's arithmetic twice (values and tangents)
+            binding.tpconv_profile_begin(8192)
+            for _ in range(5):
+                flush.zero_()
+                dbl_with_pos()
+            prof = binding.tpconv_profile_end()
+            tan_ms = prof["receiver_backward_tangent"][0] / 5
+            if c.mode == "uvw" and tan_ms > 0:
+                flop = 2 * flop_model(plan)["recv"] * E
+                ach = flop / (tan_ms / 1e3) / 1e12
+                rec["position_tangent_kernel"] = {
+                    "ms": round(tan_ms, 4), "flop": int(flop), "bound": "alu", "achieved": round(ach, 3),
+                    "peak": round(FP32_PEAK_TFLOPS, 1), "unit": "TFLOP/s", "frac": round(ach / FP32_PEAK_TFLOPS, 4),
+                    "breakdown_ms": {k: round(v[0] / 5, 4) for k, v in prof.items() if v[1] > 0}}
             rec.update({"double_backward_ms": round(ms_d, 4),
                         "double_backward_edges_per_s": round(E / ms_d * 1e3, 1),
                         "double_backward_with_pos_ms": round(ms_dp, 4),

@@ -29,7 +29,8 @@ def _units():
                 for part in parts:
                     units.append((src, {"TPC_UNIT_KP": kp, "TPC_UNIT_MODE": mode,
                                         "TPC_UNIT_PART": _PARTS[part]}))
-            for mode in (0, 1):
+            # receiver backward (0) and its tangent without (1) and with (2) an A_dot term
+            for mode in (0, 1, 2):
                 units.append((src, {"TPC_UNIT_KP": kp, "TPC_UNIT_MODE": mode, "TPC_UNIT_PART": _PARTS["RECV"]}))
     return units
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -76,6 +77,8 @@ def build(verbose=False, jobs=None, extra_flags=()):
         if _mtime(obj) < max(_mtime(src), newest_header):
             dflags = [f"-D{k}={v}" for k, v in defs.items()]
             todo.append([_nvcc(), "-c", src, "-o", obj] + flags + dflags)
+    # longest compiles (the tangent receiver units) first
+    todo.sort(key=lambda c: 0 if "-DTPC_UNIT_PART=3" in c and "-DTPC_UNIT_MODE=0" not in c else 1)
     if todo:
         with cf.ThreadPoolExecutor(max_workers=jobs or min(os.cpu_count() or 8, len(todo))) as ex:
             for out in ex.map(_run, todo):

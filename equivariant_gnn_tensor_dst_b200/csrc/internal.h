@@ -120,12 +120,12 @@ template <int KP>
 cudaError_t run_uvw_recv_bwd(const DevPlan& P, const Tasks& T, const float* x, const float* pos,
                              const int* row_ptr, const int* src, const float* Sbar, int node0,
                              int n_nodes, float4* gbuf, int edge_split, cudaStream_t s);
-template <int KP>
+template <int KP, bool AD>   // AD: the A_dot tangent is present (its own build unit)
 cudaError_t run_uvw_recv_dbl(const DevPlan& P, const Tasks& T, const float* x, const float* xdot,
                              const float* pos, const float* posdot, const int* row_ptr, const int* src,
                              const float* Sbar, const float* Sbard, int node0, int n_nodes, float4* gbuf,
                              int edge_split, cudaStream_t s);
-template <int KP>
+template <int KP, bool AD>
 cudaError_t run_uvu_recv_dbl(const DevPlan& P, const Tasks& T, const float* x, const float* xdot,
                              const float* pos, const float* posdot, const int* row_ptr, const int* src,
                              const float* W, const float* Wdot, const float* grad_out, int N, float4* gbuf,

@@ -364,7 +364,7 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32, 5)
 // g_e per edge (position_tangent).
 // ---------------------------------------------------------------------------
 
-template <int LI, int LS, int LO, int KP>
+template <int LI, int LS, int LO, int KP, bool AD>
 __device__ __forceinline__ void uvu_recv_dbl_body(const DevPlan& P, const DevPath& p, int chunk, int i,
                                                   int ne, const float* __restrict__ x,
                                                   const float* __restrict__ xdot,
@@ -375,18 +375,19 @@ __device__ __forceinline__ void uvu_recv_dbl_body(const DevPlan& P, const DevPat
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int u = chunk * 32 + lane;
   const bool act = u < p.c_in;
-  float a[KP], ad[KP], mb[RO];
+  float a[KP], ad[AD ? KP : 1], mb[RO];
 #pragma unroll
   for (int q = 0; q < KP; ++q) {
     const bool ok = act && q < P.K;
     a[q] = ok ? __ldg(W + (long long)q * P.n_w + p.w_off + u) : 0.f;
-    ad[q] = (ok && Wdot) ? __ldg(Wdot + (long long)q * P.n_w + p.w_off + u) : 0.f;
+    if constexpr (AD) ad[q] = ok ? __ldg(Wdot + (long long)q * P.n_w + p.w_off + u) : 0.f;
   }
 #pragma unroll
   for (int o = 0; o < RO; ++o)
     mb[o] = act ? __ldg(gout + (long long)i * P.dim_out + p.out_off + o * p.c_out + u) : 0.f;
   const float* xb = x + p.in_off + (act ? u : 0);
-  const float* xdb = xdot ? xdot + p.in_off + (act ? u : 0) : nullptr;
+  const bool XD = xdot != nullptr;   // warp-uniform: the x_dot terms are skipped when absent
+  const float* xdb = XD ? xdot + p.in_off + (act ? u : 0) : nullptr;
   constexpr int NY = RS <= 1 ? 1 : RS <= 2 ? 2 : RS <= 4 ? 4 : 8;
   const int yw = reduce_multi_index<NY>(lane), pw_ = reduce_multi_index<KP>(lane);
   const bool ywr = reduce_multi_writer<NY>(lane), pwr = reduce_multi_writer<KP>(lane);
@@ -394,24 +395,30 @@ __device__ __forceinline__ void uvu_recv_dbl_body(const DevPlan& P, const DevPat
     const long long row = (long long)sm.j[t] * P.dim_in;
     float xv[RI], xdv[RI], Y[RS], Yd[RS];
 #pragma unroll
-    for (int k = 0; k < RI; ++k) {
-      xv[k] = act ? __ldg(xb + row + k * p.c_in) : 0.f;
-      xdv[k] = (act && xdb) ? __ldg(xdb + row + k * p.c_in) : 0.f;
+    for (int k = 0; k < RI; ++k) xv[k] = act ? __ldg(xb + row + k * p.c_in) : 0.f;
+    if (XD) {
+#pragma unroll
+      for (int k = 0; k < RI; ++k) xdv[k] = act ? __ldg(xdb + row + k * p.c_in) : 0.f;
     }
 #pragma unroll
     for (int k = 0; k < RS; ++k) {
       Y[k] = sm.Y[t][LS * LS + k];
       Yd[k] = sm.Yd[t][LS * LS + k];
     }
-    float C[RO], Cd[RO], Ct[RO];
+    float C[RO], Cd[RO];
     cg_couple<LI, LS, LO>(xv, Y, C);
-    cg_couple<LI, LS, LO>(xdv, Y, Cd);
-    cg_couple<LI, LS, LO>(xv, Yd, Ct);
+    cg_couple<LI, LS, LO>(xv, Yd, Cd);
+    if (XD) {
+      float Ct[RO];
+      cg_couple<LI, LS, LO>(xdv, Y, Ct);
+#pragma unroll
+      for (int o = 0; o < RO; ++o) Cd[o] += Ct[o];
+    }
     float h = 0.f, hd = 0.f;
 #pragma unroll
     for (int o = 0; o < RO; ++o) {
       h = fmaf(mb[o], C[o], h);
-      hd = fmaf(mb[o], Cd[o] + Ct[o], hd);
+      hd = fmaf(mb[o], Cd[o], hd);
     }
     float we = 0.f, wed = 0.f;
     float pp[KP], ppd[KP];
@@ -420,9 +427,12 @@ __device__ __forceinline__ void uvu_recv_dbl_body(const DevPlan& P, const DevPat
       const float ph = sm.phi[t][q], phd = sm.phid[t][q];
       we = fmaf(ph, a[q], we);
       wed = fmaf(phd, a[q], wed);
-      wed = fmaf(ph, ad[q], wed);
       pp[q] = a[q] * h;
-      ppd[q] = fmaf(a[q], hd, ad[q] * h);
+      ppd[q] = a[q] * hd;
+      if constexpr (AD) {
+        wed = fmaf(ph, ad[q], wed);
+        ppd[q] = fmaf(ad[q], h, ppd[q]);
+      }
     }
     float G[RO], Gd[RO], py[NY], pyd[NY];
 #pragma unroll
@@ -436,8 +446,8 @@ __device__ __forceinline__ void uvu_recv_dbl_body(const DevPlan& P, const DevPat
       pyd[k] = 0.f;
     }
     cg_adj_y<LI, LS, LO>(xv, G, py);
-    cg_adj_y<LI, LS, LO>(xdv, G, pyd);
     cg_adj_y<LI, LS, LO>(xv, Gd, pyd);
+    if (XD) cg_adj_y<LI, LS, LO>(xdv, G, pyd);
     const float rphi = warp_reduce_multi<KP>(pp);
     const float rphid = warp_reduce_multi<KP>(ppd);
     const float ry = warp_reduce_multi<NY>(py);
@@ -455,7 +465,8 @@ __device__ __forceinline__ void uvu_recv_dbl_body(const DevPlan& P, const DevPat
 }
 
 // Same grid as k_uvu_recv_bwd: one CTA per (receiver, share of its 32-edge chunks).
-template <int KP>
+// AD: an A_dot tangent is present; without it those terms are zero.
+template <int KP, bool AD>
 __global__ void __launch_bounds__(WARPS_PER_CTA * 32, 2)
     k_uvu_recv_dbl(DevPlan P, Tasks T, const float* __restrict__ x, const float* __restrict__ xdot,
                    const float* __restrict__ pos, const float* __restrict__ posdot,
@@ -476,7 +487,7 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32, 2)
       const int chunk = T.b[task];
       dispatch_type(p.type, [&](auto tr) {
         using TR = decltype(tr);
-        uvu_recv_dbl_body<TR::li, TR::ls, TR::lo, KP>(P, p, chunk, i, ne, x, xdot, W, Wdot, gout, sm);
+        uvu_recv_dbl_body<TR::li, TR::ls, TR::lo, KP, AD>(P, p, chunk, i, ne, x, xdot, W, Wdot, gout, sm);
       });
     }
     __syncthreads();
@@ -714,13 +725,13 @@ cudaError_t run_uvu_recv_bwd(const DevPlan& P, const Tasks& T, const float* x, c
   return cudaGetLastError();
 }
 
-template <int KP>
+template <int KP, bool AD>
 cudaError_t run_uvu_recv_dbl(const DevPlan& P, const Tasks& T, const float* x, const float* xdot,
                              const float* pos, const float* posdot, const int* row_ptr, const int* src,
                              const float* W, const float* Wdot, const float* grad_out, int N, float4* gbuf,
                              int edge_split, cudaStream_t s) {
-  k_uvu_recv_dbl<KP><<<dim3((unsigned)N, (unsigned)edge_split), WARPS_PER_CTA * 32, 0, s>>>(
-      P, T, x, xdot, pos, posdot, row_ptr, src, W, Wdot, grad_out, N, gbuf);
+  k_uvu_recv_dbl<KP, AD><<<dim3((unsigned)N, (unsigned)edge_split), WARPS_PER_CTA * 32, 0, s>>>(
+      P, T, x, xdot, pos, posdot, row_ptr, src, W, AD ? Wdot : nullptr, grad_out, N, gbuf);
   return cudaGetLastError();
 }
 
@@ -771,8 +782,8 @@ template cudaError_t run_uvu_recv_bwd<TPC_UNIT_KP>(const DevPlan&, const Tasks&,
                                                    const float*, const float*, int, float4*, int,
                                                    cudaStream_t);
 #endif
-#if TPC_UNIT_PART == TPC_PART_RECV && TPC_UNIT_MODE == 1
-template cudaError_t run_uvu_recv_dbl<TPC_UNIT_KP>(const DevPlan&, const Tasks&, const float*, const float*,
+#if TPC_UNIT_PART == TPC_PART_RECV && (TPC_UNIT_MODE == 1 || TPC_UNIT_MODE == 2)
+template cudaError_t run_uvu_recv_dbl<TPC_UNIT_KP, TPC_UNIT_MODE == 2>(const DevPlan&, const Tasks&, const float*, const float*,
                                                    const float*, const float*, const int*, const int*,
                                                    const float*, const float*, const float*, int, float4*,
                                                    int, cudaStream_t);

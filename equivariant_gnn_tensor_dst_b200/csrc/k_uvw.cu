@@ -438,9 +438,9 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32, TPC_MINB_RECV)
 // then the tangent of g_e (position_tangent), staged per edge like the backward's g_e.
 // ---------------------------------------------------------------------------
 
-#define TPC_MINB_RECV_DBL (KP == 8 ? 2 : 1)
+#define TPC_MINB_RECV_DBL ((KP == 8 || !AD) ? 2 : 1)
 
-template <int LI, int LS, int LO, int KP>
+template <int LI, int LS, int LO, int KP, bool AD>
 __device__ __forceinline__ void uvw_recv_dbl_body(const DevPlan& P, const DevPath& p, int chunk,
                                                   int node_local, int ne,
                                                   const float* __restrict__ x,
@@ -453,8 +453,9 @@ __device__ __forceinline__ void uvw_recv_dbl_body(const DevPlan& P, const DevPat
   const int u = chunk * 32 + lane;
   const bool act = u < p.c_in;
   const float* xb = x + p.in_off + (act ? u : 0);
-  const float* xdb = xdot ? xdot + p.in_off + (act ? u : 0) : nullptr;
-  float sb[KP][RO], sbd[KP][RO];
+  const bool XD = xdot != nullptr;   // warp-uniform: the x_dot terms are skipped when absent
+  const float* xdb = XD ? xdot + p.in_off + (act ? u : 0) : nullptr;
+  float sb[KP][RO], sbd[AD ? KP : 1][RO];
   {
     const long long base = (long long)node_local * P.state_per_node + p.st_off + u;
     const int rs = P.K * p.c_in;
@@ -464,7 +465,7 @@ __device__ __forceinline__ void uvw_recv_dbl_body(const DevPlan& P, const DevPat
       for (int q = 0; q < KP; ++q) {
         const bool ok = act && q < P.K;
         sb[q][o] = ok ? Sbar[base + (long long)o * rs + q * p.c_in] : 0.f;
-        sbd[q][o] = (ok && Sbard) ? Sbard[base + (long long)o * rs + q * p.c_in] : 0.f;
+        if constexpr (AD) sbd[q][o] = ok ? Sbard[base + (long long)o * rs + q * p.c_in] : 0.f;
       }
   }
   constexpr int NY = RS <= 1 ? 1 : RS <= 2 ? 2 : RS <= 4 ? 4 : 8;
@@ -474,9 +475,10 @@ __device__ __forceinline__ void uvw_recv_dbl_body(const DevPlan& P, const DevPat
     const long long row = (long long)sm.j[t] * P.dim_in;
     float xv[RI], xdv[RI];
 #pragma unroll
-    for (int m = 0; m < RI; ++m) {
-      xv[m] = act ? __ldg(xb + row + m * p.c_in) : 0.f;
-      xdv[m] = (act && xdb) ? __ldg(xdb + row + m * p.c_in) : 0.f;
+    for (int m = 0; m < RI; ++m) xv[m] = act ? __ldg(xb + row + m * p.c_in) : 0.f;
+    if (XD) {
+#pragma unroll
+      for (int m = 0; m < RI; ++m) xdv[m] = act ? __ldg(xdb + row + m * p.c_in) : 0.f;
     }
     float Y[RS], Yd[RS], phi[KP], phid[KP];
 #pragma unroll
@@ -489,12 +491,15 @@ __device__ __forceinline__ void uvw_recv_dbl_body(const DevPlan& P, const DevPat
       phi[q] = sm.phi[t][q];
       phid[q] = sm.phid[t][q];
     }
-    float C[RO], Cd[RO], Ct[RO];
+    float C[RO], Cd[RO];
     cg_couple<LI, LS, LO>(xv, Y, C);
-    cg_couple<LI, LS, LO>(xdv, Y, Cd);
-    cg_couple<LI, LS, LO>(xv, Yd, Ct);
+    cg_couple<LI, LS, LO>(xv, Yd, Cd);
+    if (XD) {
+      float Ct[RO];
+      cg_couple<LI, LS, LO>(xdv, Y, Ct);
 #pragma unroll
-    for (int o = 0; o < RO; ++o) Cd[o] += Ct[o];
+      for (int o = 0; o < RO; ++o) Cd[o] += Ct[o];
+    }
     float pp[KP], ppd[KP];
 #pragma unroll
     for (int q = 0; q < KP; ++q) {
@@ -503,7 +508,7 @@ __device__ __forceinline__ void uvw_recv_dbl_body(const DevPlan& P, const DevPat
       for (int o = 0; o < RO; ++o) {
         a = fmaf(sb[q][o], C[o], a);
         b = fmaf(sb[q][o], Cd[o], b);
-        b = fmaf(sbd[q][o], C[o], b);
+        if constexpr (AD) b = fmaf(sbd[q][o], C[o], b);
       }
       pp[q] = a;
       ppd[q] = b;
@@ -516,7 +521,7 @@ __device__ __forceinline__ void uvw_recv_dbl_body(const DevPlan& P, const DevPat
       for (int q = 0; q < KP; ++q) {
         a = fmaf(phi[q], sb[q][o], a);
         b = fmaf(phid[q], sb[q][o], b);
-        b = fmaf(phi[q], sbd[q][o], b);
+        if constexpr (AD) b = fmaf(phi[q], sbd[q][o], b);
       }
       Tb[o] = a;
       Tbd[o] = b;
@@ -528,8 +533,8 @@ __device__ __forceinline__ void uvw_recv_dbl_body(const DevPlan& P, const DevPat
       pyd[k] = 0.f;
     }
     cg_adj_y<LI, LS, LO>(xv, Tb, py);
-    cg_adj_y<LI, LS, LO>(xdv, Tb, pyd);
     cg_adj_y<LI, LS, LO>(xv, Tbd, pyd);
+    if (XD) cg_adj_y<LI, LS, LO>(xdv, Tb, pyd);
     const float rphi = warp_reduce_multi<KP>(pp);
     const float rphid = warp_reduce_multi<KP>(ppd);
     const float ry = warp_reduce_multi<NY>(py);
@@ -547,7 +552,8 @@ __device__ __forceinline__ void uvw_recv_dbl_body(const DevPlan& P, const DevPat
 }
 
 // Same grid as k_uvw_recv_bwd: one CTA per (receiver, share of its 32-edge chunks).
-template <int KP>
+// AD: an A_dot tangent is present (S_bar_dot is read); without it those terms are zero.
+template <int KP, bool AD>
 __global__ void __launch_bounds__(WARPS_PER_CTA * 32, TPC_MINB_RECV_DBL)
     k_uvw_recv_dbl(DevPlan P, Tasks T, const float* __restrict__ x, const float* __restrict__ xdot,
                    const float* __restrict__ pos, const float* __restrict__ posdot,
@@ -569,7 +575,7 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32, TPC_MINB_RECV_DBL)
       const int chunk = T.b[task];
       dispatch_type(p.type, [&](auto tr) {
         using TR = decltype(tr);
-        uvw_recv_dbl_body<TR::li, TR::ls, TR::lo, KP>(P, p, chunk, node_local, ne, x, xdot, Sbar, Sbard, sm);
+        uvw_recv_dbl_body<TR::li, TR::ls, TR::lo, KP, AD>(P, p, chunk, node_local, ne, x, xdot, Sbar, Sbard, sm);
       });
     }
     __syncthreads();
@@ -734,13 +740,13 @@ cudaError_t run_uvw_recv_bwd(const DevPlan& P, const Tasks& T, const float* x, c
   return cudaGetLastError();
 }
 
-template <int KP>
+template <int KP, bool AD>
 cudaError_t run_uvw_recv_dbl(const DevPlan& P, const Tasks& T, const float* x, const float* xdot,
                              const float* pos, const float* posdot, const int* row_ptr, const int* src,
                              const float* Sbar, const float* Sbard, int node0, int n_nodes, float4* gbuf,
                              int edge_split, cudaStream_t s) {
-  k_uvw_recv_dbl<KP><<<dim3((unsigned)n_nodes, (unsigned)edge_split), WARPS_PER_CTA * 32, 0, s>>>(
-      P, T, x, xdot, pos, posdot, row_ptr, src, Sbar, Sbard, node0, n_nodes, gbuf);
+  k_uvw_recv_dbl<KP, AD><<<dim3((unsigned)n_nodes, (unsigned)edge_split), WARPS_PER_CTA * 32, 0, s>>>(
+      P, T, x, xdot, pos, posdot, row_ptr, src, Sbar, AD ? Sbard : nullptr, node0, n_nodes, gbuf);
   return cudaGetLastError();
 }
 
@@ -783,8 +789,8 @@ template cudaError_t run_uvw_recv_bwd<TPC_UNIT_KP>(const DevPlan&, const Tasks&,
                                                    const float*, int, int, float4*, int,
                                                    cudaStream_t);
 #endif
-#if TPC_UNIT_PART == TPC_PART_RECV && TPC_UNIT_MODE == 1
-template cudaError_t run_uvw_recv_dbl<TPC_UNIT_KP>(const DevPlan&, const Tasks&, const float*, const float*,
+#if TPC_UNIT_PART == TPC_PART_RECV && (TPC_UNIT_MODE == 1 || TPC_UNIT_MODE == 2)
+template cudaError_t run_uvw_recv_dbl<TPC_UNIT_KP, TPC_UNIT_MODE == 2>(const DevPlan&, const Tasks&, const float*, const float*,
                                                    const float*, const float*, const int*, const int*,
                                                    const float*, const float*, int, int, float4*, int,
                                                    cudaStream_t);

@@ -32,9 +32,15 @@ cudaError_t launch_uvw_recv_dbl(const DevPlan& P, const Tasks& T, const float* x
                                 int edge_split, cudaStream_t s) {
   if (n_nodes <= 0) return cudaSuccess;
   if (edge_split < 1) edge_split = 1;
-  if (P.K <= 8)
-    return run_uvw_recv_dbl<8>(P, T, x, xdot, pos, posdot, row_ptr, src, Sbar, Sbard, node0, n_nodes, gbuf, edge_split, s);
-  return run_uvw_recv_dbl<16>(P, T, x, xdot, pos, posdot, row_ptr, src, Sbar, Sbard, node0, n_nodes, gbuf, edge_split, s);
+#define TPC_RUN_DBL(KP, AD) \
+  return run_uvw_recv_dbl<KP, AD>(P, T, x, xdot, pos, posdot, row_ptr, src, Sbar, Sbard, node0, n_nodes, gbuf, edge_split, s)
+  if (P.K <= 8) {
+    if (Sbard) TPC_RUN_DBL(8, true);
+    TPC_RUN_DBL(8, false);
+  }
+  if (Sbard) TPC_RUN_DBL(16, true);
+  TPC_RUN_DBL(16, false);
+#undef TPC_RUN_DBL
 }
 
 cudaError_t launch_uvu_recv_dbl(const DevPlan& P, const Tasks& T, const float* x, const float* xdot,
@@ -43,9 +49,15 @@ cudaError_t launch_uvu_recv_dbl(const DevPlan& P, const Tasks& T, const float* x
                                 int edge_split, cudaStream_t s) {
   if (N <= 0) return cudaSuccess;
   if (edge_split < 1) edge_split = 1;
-  if (P.K <= 8)
-    return run_uvu_recv_dbl<8>(P, T, x, xdot, pos, posdot, row_ptr, src, W, Wdot, grad_out, N, gbuf, edge_split, s);
-  return run_uvu_recv_dbl<16>(P, T, x, xdot, pos, posdot, row_ptr, src, W, Wdot, grad_out, N, gbuf, edge_split, s);
+#define TPC_RUN_DBL(KP, AD) \
+  return run_uvu_recv_dbl<KP, AD>(P, T, x, xdot, pos, posdot, row_ptr, src, W, Wdot, grad_out, N, gbuf, edge_split, s)
+  if (P.K <= 8) {
+    if (Wdot) TPC_RUN_DBL(8, true);
+    TPC_RUN_DBL(8, false);
+  }
+  if (Wdot) TPC_RUN_DBL(16, true);
+  TPC_RUN_DBL(16, false);
+#undef TPC_RUN_DBL
 }
 
 cudaError_t launch_uvw_src_state(const DevPlan& P, const Tasks& T, int mode,
