@@ -66,13 +66,14 @@ def test_mul_ir_layout_every_pass(torch, cfg, n):
     ggp = workloads.normal(p.rng, p.pos.shape)
     ggw = workloads.normal(p.rng, p.W.shape)
     da = [t.cpu().numpy() for t in binding.tpconv_double_backward(a, x, pos, rp, src, *v, W, go, gg_x=cuda(ggx),
-                                                                  gg_pos=cuda(ggp), gg_W=cuda(ggw))]
+                                                                  gg_pos=cuda(ggp), gg_W=cuda(ggw), need_pos=True)]
     dm = [t.cpu().numpy() for t in binding.tpconv_double_backward(m, xm, pos, rp, src, *v, W, gom,
                                                                   gg_x=cuda(_to_mul_ir(ggx, bi)), gg_pos=cuda(ggp),
-                                                                  gg_W=cuda(ggw))]
+                                                                  gg_W=cuda(ggw), need_pos=True)]
     assert np.array_equal(_from_mul_ir(dm[0], bi), da[0])
     assert np.array_equal(dm[1], da[1])
     assert np.array_equal(_from_mul_ir(dm[2], bo), da[2])
+    assert np.array_equal(dm[3], da[3])          # dLambda/dpos: [N][3] in both layouts
 
     if p.cfg.mode == "uvw":
         Y = workloads.normal(p.rng, (p.E, p.plan.n_sh))
