@@ -432,6 +432,19 @@ def run_extras(args, dev, flush):
         ms_b = _timed(bwd, flush, steps, warm)
         rec.update({"forward_ms": round(ms_f, 4), "forward_edges_per_s": round(E / ms_f * 1e3, 1),
                     "backward_ms": round(ms_b, 4), "backward_edges_per_s": round(E / ms_b * 1e3, 1)})
+        # the same passes on the graph renumbered in Morton order of the positions (locality
+        # of the x and m_bar row gathers; results are the renumbered results)
+        perm = binding.tpconv_spatial_order(pos)
+        rp2, src2, _ = binding.tpconv_permute_graph(rp, src, perm)
+        x2, pos2, go2 = (binding.tpconv_gather_rows(a, perm) for a in (x, pos, go))
+        views2 = binding.tpconv_csr_transpose(rp2, src2, N)
+        fwd2 = lambda: binding.tpconv_forward(plan, x2, pos2, rp2, src2, W, out=o, ws=ws)  # noqa: E731
+        bwd2 = lambda: binding.tpconv_backward(plan, x2, pos2, rp2, src2, *views2, W, go2, ws=ws,  # noqa: E731
+                                               outputs=(gx, gp, gw))
+        ms_f2, ms_b2 = _timed(fwd2, flush, steps, warm), _timed(bwd2, flush, steps, warm)
+        rec["spatial_order"] = {"forward_ms": round(ms_f2, 4), "backward_ms": round(ms_b2, 4),
+                                "forward_backward_edges_per_s": round(E / (ms_f2 + ms_b2) * 1e3, 1)}
+        del x2, pos2, go2, views2, rp2, src2
         if True:  # every mode
             # the embedded-input interface: phi_e and Y_e given per edge, phi_bar and Y_bar returned
             Ye = tt(workloads.normal(rng, (E, (c.sh_lmax + 1) ** 2)))

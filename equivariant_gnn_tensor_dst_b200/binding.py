@@ -55,6 +55,11 @@ SIGNATURES = {
     "tpconv_profile_category_name": (ctypes.c_char_p, [ctypes.c_int32]),
     "tpconv_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int32)]),
     "tpconv_forward_no_alloc": (ctypes.c_int, [_c_p, _c_i64, _c_i64] + [_c_p] * 6 + [_c_p]),
+    # include/tpconv_graph.h
+    "tpconv_spatial_order_workspace_bytes": (ctypes.c_int, [_c_i64, ctypes.POINTER(ctypes.c_size_t)]),
+    "tpconv_spatial_order": (ctypes.c_int, [_c_i64, _c_p, _c_p, _c_p, ctypes.c_size_t, _c_p]),
+    "tpconv_permute_graph": (ctypes.c_int, [_c_i64, _c_i64] + [_c_p] * 6 + [_c_p]),
+    "tpconv_gather_rows": (ctypes.c_int, [_c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p]),
 }
 PROF_CATEGORIES = 13
 
@@ -327,6 +332,48 @@ def tpconv_double_backward(plan, x, pos, row_ptr, src, t_ptr, t_eid, t_dst, W, g
                                        _ptr(gp), _ptr(ws), ws.numel(), _stream(stream)),
           "tpconv_double_backward")
     return (gx, gw, gg, gp) if need_pos else (gx, gw, gg)
+
+
+def tpconv_spatial_order(pos, stream=None):
+    """perm [N] int32: nodes in Morton order of their positions (perm[k] = old id)."""
+    import torch
+    _need(pos, torch.float32, "pos")
+    N = pos.shape[0]
+    perm = torch.empty(max(N, 1), dtype=torch.int32, device=pos.device)
+    nb = ctypes.c_size_t()
+    check(lib().tpconv_spatial_order_workspace_bytes(N, ctypes.byref(nb)), "tpconv_spatial_order_workspace_bytes")
+    ws = workspace(nb.value, pos.device)
+    check(lib().tpconv_spatial_order(N, _ptr(pos), _ptr(perm), _ptr(ws), ws.numel(), _stream(stream)),
+          "tpconv_spatial_order")
+    return perm[:N]
+
+
+def tpconv_permute_graph(row_ptr, src, perm, stream=None):
+    """The receiver CSR renumbered by perm: (row_ptr_out, src_out, inv)."""
+    import torch
+    _need(row_ptr, torch.int32, "row_ptr")
+    _need(src, torch.int32, "src")
+    _need(perm, torch.int32, "perm")
+    N, E = row_ptr.numel() - 1, src.numel()
+    dev = row_ptr.device
+    rp = torch.empty(N + 1, dtype=torch.int32, device=dev)
+    so = torch.empty(max(E, 1), dtype=torch.int32, device=dev)
+    inv = torch.empty(max(N, 1), dtype=torch.int32, device=dev)
+    check(lib().tpconv_permute_graph(N, E, _ptr(row_ptr), _ptr(src), _ptr(perm), _ptr(rp), _ptr(so), _ptr(inv),
+                                     _stream(stream)), "tpconv_permute_graph")
+    return rp, so[:E], inv[:N]
+
+
+def tpconv_gather_rows(a, perm, stream=None):
+    """out[k] = a[perm[k]] for a 2-D float32 array (node features, positions)."""
+    import torch
+    _need(a, torch.float32, "a")
+    _need(perm, torch.int32, "perm")
+    rows, width = a.shape[0], (a.numel() // a.shape[0] if a.shape[0] else 0)
+    out = torch.empty_like(a)
+    check(lib().tpconv_gather_rows(perm.numel(), width, _ptr(a), _ptr(perm), _ptr(out), _stream(stream)),
+          "tpconv_gather_rows")
+    return out
 
 
 def tpconv_profile_begin(max_records=8192):

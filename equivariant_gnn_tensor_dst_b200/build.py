@@ -22,7 +22,7 @@ _PARTS = {"STATE": 1, "SRC": 2, "RECV": 3, "FWD": 4, "GRADW": 5}
 
 
 def _units():
-    units = [("k_misc.cu", {}), ("k_gemm_tc.cu", {}), ("launch.cu", {}), ("api.cu", {})]
+    units = [("k_misc.cu", {}), ("k_gemm_tc.cu", {}), ("launch.cu", {}), ("api.cu", {}), ("k_order.cu", {})]
     for kp in (8, 16):
         for src, parts in (("k_uvw.cu", ("STATE", "SRC")), ("k_uvu.cu", ("FWD", "GRADW", "SRC"))):
             for mode in (0, 1):

@@ -1,6 +1,6 @@
 """Host-side checks of the C ABI (no GPU needed).
 
-* the shared library loads and exports every function declared in include/tpconv.h;
+* the shared library loads and exports every function declared in include/*.h;
 * the plan builder enumerates the same paths, widths and weight offsets as the oracle
   and its coupling tables (computed by a different algorithm at build time) equal the
   oracle's to 1e-12;
@@ -22,9 +22,14 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def _declared():
-    txt = open(os.path.join(ROOT, "include", "tpconv.h")).read()
-    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
-    return sorted(set(re.findall(r"\b(tpconv_\w+)\s*\(", txt)))
+    """Functions declared in every header under include/."""
+    names = set()
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", h)).read()
+            txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+            names |= set(re.findall(r"\b(tpconv_\w+)\s*\(", txt))
+    return sorted(names)
 
 
 def test_library_exports_every_declared_symbol():
@@ -193,3 +198,27 @@ def test_plan_set_layout_arguments():
     assert L.tpconv_plan_set_layout(None, 0) == 1              # TPCONV_ERR_INVALID_ARG
     assert L.tpconv_plan_set_layout(p.handle, binding.LAYOUT_IR_MUL) == 0
     assert p.workspace_bytes(100, 800) == base
+
+
+def test_graph_header_symbols_and_host_checks():
+    """Every function of include/tpconv_graph.h is exported; argument checks return
+    before any launch."""
+    txt = open(os.path.join(ROOT, "include", "tpconv_graph.h")).read()
+    names = set(re.findall(r"\b(tpconv_\w+)\s*\(", txt))
+    assert names >= {"tpconv_spatial_order", "tpconv_spatial_order_workspace_bytes", "tpconv_permute_graph",
+                     "tpconv_gather_rows"}
+    L = binding.lib()
+    for n in names:
+        assert hasattr(L, n), n
+    nb = ctypes.c_size_t()
+    assert L.tpconv_spatial_order_workspace_bytes(1000, ctypes.byref(nb)) == 0
+    assert nb.value == 8 * 1024 + 256                      # keys padded to 1024, then the box
+    assert L.tpconv_spatial_order_workspace_bytes(-1, ctypes.byref(nb)) == 1
+    fake = ctypes.c_void_p(1 << 20)
+    assert L.tpconv_spatial_order(10, fake, fake, fake, 16, None) == 4     # workspace too small
+    assert L.tpconv_spatial_order(10, None, fake, fake, 1 << 20, None) == 1
+    assert L.tpconv_spatial_order(0, None, None, None, 0, None) == 0       # empty: no-op
+    assert L.tpconv_permute_graph(-1, 0, fake, fake, fake, fake, fake, fake, None) == 1
+    assert L.tpconv_permute_graph(10, 5, fake, None, fake, fake, fake, fake, None) == 1
+    assert L.tpconv_gather_rows(10, 4, None, fake, fake, None) == 1
+    assert L.tpconv_gather_rows(0, 4, None, None, None, None) == 0
