@@ -445,18 +445,17 @@ def run_extras(args, dev, flush):
         rec["spatial_order"] = {"forward_ms": round(ms_f2, 4), "backward_ms": round(ms_b2, 4),
                                 "forward_backward_edges_per_s": round(E / (ms_f2 + ms_b2) * 1e3, 1)}
         del x2, pos2, go2, views2, rp2, src2
-        if True:  # every mode
-            # the embedded-input interface: phi_e and Y_e given per edge, phi_bar and Y_bar returned
-            Ye = tt(workloads.normal(rng, (E, (c.sh_lmax + 1) ** 2)))
-            pe = tt(workloads.normal(rng, (E, c.num_basis)))
-            gphi = torch.empty(E, c.num_basis, device=dev)
-            gY = torch.empty(E, (c.sh_lmax + 1) ** 2, device=dev)
-            fe = lambda: binding.tpconv_forward_embedded(plan, x, Ye, pe, rp, src, W, out=o, ws=ws)  # noqa: E731
-            be = lambda: binding.tpconv_backward_embedded(plan, x, Ye, pe, rp, src, *views, W, go, ws=ws,  # noqa: E731
-                                                          outputs=(gx, gw, gphi, gY))
-            ms_ef, ms_eb = _timed(fe, flush, steps, warm), _timed(be, flush, steps, warm)
-            rec["embedded_interface"] = {"forward_ms": round(ms_ef, 4), "backward_ms": round(ms_eb, 4),
-                                         "forward_backward_edges_per_s": round(E / (ms_ef + ms_eb) * 1e3, 1)}
+        # the embedded-input interface: phi_e and Y_e given per edge, phi_bar and Y_bar returned
+        Ye = tt(workloads.normal(rng, (E, (c.sh_lmax + 1) ** 2)))
+        pe = tt(workloads.normal(rng, (E, c.num_basis)))
+        gphi = torch.empty(E, c.num_basis, device=dev)
+        gY = torch.empty(E, (c.sh_lmax + 1) ** 2, device=dev)
+        fe = lambda: binding.tpconv_forward_embedded(plan, x, Ye, pe, rp, src, W, out=o, ws=ws)  # noqa: E731
+        be = lambda: binding.tpconv_backward_embedded(plan, x, Ye, pe, rp, src, *views, W, go, ws=ws,  # noqa: E731
+                                                      outputs=(gx, gw, gphi, gY))
+        ms_ef, ms_eb = _timed(fe, flush, steps, warm), _timed(be, flush, steps, warm)
+        rec["embedded_interface"] = {"forward_ms": round(ms_ef, 4), "backward_ms": round(ms_eb, 4),
+                                     "forward_backward_edges_per_s": round(E / (ms_ef + ms_eb) * 1e3, 1)}
         if c.mode == "uvw":
             # the optional TF32 contraction mode (1e-2 accuracy class), reported separately
             plan.set_math(binding.MATH_TF32)
