@@ -517,7 +517,10 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
     }
   }
   // the last commit completes after every MMA of the tile (tcgen05 operations complete
-  // in issue order)
+  // in issue order).  Only the MMA and converter warps' waits here are exact: a producer
+  // warp can run more than one phase ahead of the MMA completions, so its parity wait may
+  // pass on an earlier phase.  Every thread therefore reads the accumulator only after the
+  // block barrier below, which follows the exact waits.
   if (ntiles > 0) {
     const int j = ntiles - 1;
     ok = mbar_wait<128>(smem_u32(&mdone[j % SM::NS]), (j / SM::NS) & 1) && ok;
@@ -534,6 +537,7 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
   long long* rowoff = reinterpret_cast<long long*>(ring + 65536);
   long long* coloff = rowoff + TC_M;
   __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   for (int t = tid; t < TC_M; t += TC_THREADS) {
     const int m = m0 + t;
     rowoff[t] = m < P.M ? (g.splits > 1 ? ((long long)split * P.M + m) * P.N : ixd(P.Cm, m)) : 0;
