@@ -42,10 +42,10 @@ SPLIT_MMAS = 3                                      # 3xTF32: three TF32 product
 # launches have the same 1024-node chunk shape (per step: twice its launches).  Valid for
 # the kernels as captured; only reported for that workload.
 TRAFFIC_BYTES_PER_STEP = {
-    "channel_gemm": 2 * (6 * 92.48e6 + 2 * 32.95e6 + 6 * 9.43e6),
-    "uvw_receiver_backward": 4 * 95.48e6,
-    "uvw_source_state": 4 * 35.57e6,
-    "uvw_receiver_state": 4 * 35.11e6,
+    "channel_gemm": 2 * (6 * 92.09e6 + 2 * 32.81e6 + 6 * 9.45e6),
+    "uvw_receiver_backward": 4 * 95.52e6,
+    "uvw_source_state": 4 * 35.29e6,
+    "uvw_receiver_state": 4 * 35.07e6,
 }
 
 
