@@ -63,7 +63,8 @@ def _horner(coeffs, z):
 
 
 def unit_direction(r, second=False):
-    """r_hat = r / |r| as Duals (eq. 8).  A zero-length vector maps to r_hat = 0.
+    """r_hat = r / |r| as Duals (eq. 8).  A zero-length vector maps to r_hat = 0 (and
+    sh_dual then sets every l > 0 harmonic of it to zero).
     With ``second`` the Duals also carry Hessians in r."""
     from .dual import edge_vector
     rx, ry, rz = edge_vector(r, second)
@@ -84,8 +85,12 @@ def sh_dual(lmax, r, second=False):
     gradient is d Y / d r (the raw edge vector, not r_hat); with ``second`` they also
     carry d^2 Y / dr^2.
     """
-    (x, y, z), _ = unit_direction(r, second)
+    (x, y, z), d = unit_direction(r, second)
     n = x.v.shape[0]
+    # a zero-length edge has no direction: every l > 0 harmonic is zero there (the only
+    # choice that commutes with rotations), while Y_0 = 1 keeps its constant value
+    directed = d.v >= 1e-12
+    z0 = Dual.const(0.0, n)
     # powers (x + i y)^m as (re, im) Duals
     re = [Dual.const(1.0, n)]
     im = [Dual.const(0.0, n)]
@@ -103,6 +108,8 @@ def sh_dual(lmax, r, second=False):
             else:
                 row[l + m] = q * re[m]
                 row[l - m] = q * im[m]
+        if l > 0:
+            row = [q.where(directed, z0) for q in row]
         out.extend(row)
     return out
 

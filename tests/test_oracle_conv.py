@@ -70,6 +70,24 @@ def test_forward_o3_equivariant(case, improper, rng):
     assert np.abs(m).max() > 1e-3
 
 
+@pytest.mark.parametrize("improper", [False, True])
+def test_forward_equivariant_with_coincident_nodes(improper, rng):
+    # a receiver placed on one of its sources: that zero-length edge still carries the
+    # radial limit phi(0) != 0 (Bessel), so its l > 0 harmonics must vanish for the
+    # operator to stay O(3) equivariant
+    plan, x, pos, row_ptr, src, A, _ = _problem("uvw")
+    pos = pos.copy()
+    pos[3] = pos[src[row_ptr[3]]]
+    assert radial.basis_of_vectors(plan.radial, np.zeros((1, 3)))[0].max() > 0.1
+    R0 = Rotation.random(random_state=12).as_matrix()
+    R = -R0 if improper else R0
+    det = np.linalg.det(R)
+    m = conv.forward(plan, x, pos, row_ptr, src, A)
+    m2 = conv.forward(plan, _act(plan.blocks_in, x, R0, det, rng), pos @ R.T, row_ptr, src, A)
+    expect = _act(plan.blocks_out, m, R0, det, rng)
+    assert np.abs(m2 - expect).max() <= 1e-10 * max(1.0, np.abs(m).max())
+
+
 def test_forward_permutation_equivariant():
     plan, x, pos, row_ptr, src, A, rng = _problem("uvw", n=9, k=3)
     perm = rng.permutation(9)           # new node a is old node perm[a]

@@ -104,9 +104,17 @@ def test_sh_rotation_is_orthogonal_homomorphism(rng):
 
 
 def test_zero_vector_direction():
-    Y, dY = so3.sh_with_grad(2, np.zeros((1, 3)))
-    assert np.allclose(Y[0], [1, 0, 0, 0, 0, 0, -sqrt(5) / 2, 0, 0])
-    assert np.all(np.isfinite(dY))
+    # a direction-less edge: only the invariant Y_0 survives (any nonzero l > 0 value
+    # would single out an axis and break rotation equivariance), with zero derivatives
+    Y, dY = so3.sh_with_grad(3, np.zeros((1, 3)))
+    assert np.array_equal(Y[0], np.eye(16)[0])
+    assert np.array_equal(dY, np.zeros_like(dY))
+    Y2, dY2, H2 = so3.sh_with_hessian(3, np.zeros((2, 3)))
+    assert np.array_equal(Y2, np.tile(np.eye(16)[0], (2, 1)))
+    assert not np.any(dY2) and not np.any(H2)
+    # the mask acts on exactly the zero vector: a tiny but nonzero edge keeps its direction
+    r = np.array([[0.0, 0.0, 1e-6]])
+    assert np.allclose(so3.sh(3, r), so3.sh(3, np.array([[0.0, 0.0, 1.0]])), atol=1e-12)
 
 
 # ---------------------------------------------------------------- CG
