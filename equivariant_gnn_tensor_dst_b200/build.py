@@ -24,15 +24,43 @@ _PARTS = {"STATE": 1, "SRC": 2, "RECV": 3, "FWD": 4, "GRADW": 5}
 def _units():
     units = [("k_misc.cu", {}), ("k_gemm_tc.cu", {}), ("launch.cu", {}), ("api.cu", {}), ("k_order.cu", {})]
     for kp in (8, 16):
-        for src, parts in (("k_uvw.cu", ("STATE", "SRC")), ("k_uvu.cu", ("FWD", "GRADW", "SRC"))):
-            for mode in (0, 1):
-                for part in parts:
-                    units.append((src, {"TPC_UNIT_KP": kp, "TPC_UNIT_MODE": mode,
-                                        "TPC_UNIT_PART": _PARTS[part]}))
-            # receiver backward (0) and its tangent without (1) and with (2) an A_dot term
-            for mode in (0, 1, 2):
-                units.append((src, {"TPC_UNIT_KP": kp, "TPC_UNIT_MODE": mode, "TPC_UNIT_PART": _PARTS["RECV"]}))
+        for mode in (0, 1):   # generic and fast variants of the receiver backward
+            units.append(("k_recv_edge.cu", {"TPC_UNIT_KP": kp, "TPC_UNIT_MODE": mode}))
+        for mode in (0, 1):
+            for part in ("STATE", "SRC"):
+                units.append(("k_uvw.cu", {"TPC_UNIT_KP": kp, "TPC_UNIT_MODE": mode, "TPC_UNIT_PART": _PARTS[part]}))
+            for part in ("FWD", "GRADW", "SRC"):
+                units.append(("k_uvu.cu", {"TPC_UNIT_KP": kp, "TPC_UNIT_MODE": mode, "TPC_UNIT_PART": _PARTS[part]}))
+        units.append(("k_uvu.cu", {"TPC_UNIT_KP": kp, "TPC_UNIT_MODE": 0, "TPC_UNIT_PART": _PARTS["RECV"]}))
+        # tangents of the receiver backward without (1) and with (2) an A_dot term
+        for mode in (1, 2):
+            units.append(("k_uvw_dbl.cu", {"TPC_UNIT_KP": kp, "TPC_UNIT_MODE": mode}))
+            units.append(("k_uvu_dbl.cu", {"TPC_UNIT_KP": kp, "TPC_UNIT_MODE": mode}))
     return units
+
+
+def _includes(path, dirs, seen=None):
+    """Every local header a source includes, transitively (quoted includes only)."""
+    seen = set() if seen is None else seen
+    try:
+        text = open(path).read()
+    except OSError:
+        return seen
+    for line in text.splitlines():
+        line = line.strip()
+        if not line.startswith("#include \""):
+            continue
+        name = line.split('"')[1]
+        for d in [os.path.dirname(path)] + dirs:
+            cand = os.path.normpath(os.path.join(d, name))
+            if os.path.exists(cand):
+                if cand not in seen:
+                    seen.add(cand)
+                    _includes(cand, dirs, seen)
+                break
+    return seen
+
+
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -61,9 +89,7 @@ def build(verbose=False, jobs=None, extra_flags=()):
         _run(["g++", "-O2", "-std=c++17", "-o", gen_bin, gen_src])
     if _mtime(tables) < _mtime(gen_bin):
         _run([gen_bin, tables])
-    headers = [os.path.join(CSRC, h) for h in os.listdir(CSRC) if h.endswith((".h", ".cuh"))]
-    headers += [tables, os.path.join(ROOT, "include", "tpconv.h")]
-    newest_header = max(_mtime(h) for h in headers)
+    inc_dirs = [BUILD, CSRC, os.path.join(ROOT, "include")]
     flags = ARCH + ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",
                     "-Xcompiler", "-fPIC", "-I", BUILD, "-I", CSRC, "-I", os.path.join(ROOT, "include")]
     flags += list(extra_flags)
@@ -74,11 +100,12 @@ def build(verbose=False, jobs=None, extra_flags=()):
         tag = "_".join(f"{v}" for v in defs.values())
         obj = os.path.join(BUILD, s + (("." + tag) if tag else "") + ".o")
         objs.append(obj)
-        if _mtime(obj) < max(_mtime(src), newest_header):
+        deps = _includes(src, inc_dirs)
+        if _mtime(obj) < max([_mtime(src)] + [_mtime(h) for h in deps]):
             dflags = [f"-D{k}={v}" for k, v in defs.items()]
             todo.append([_nvcc(), "-c", src, "-o", obj] + flags + dflags)
     # longest compiles (the tangent receiver units) first
-    todo.sort(key=lambda c: 0 if "-DTPC_UNIT_PART=3" in c and "-DTPC_UNIT_MODE=0" not in c else 1)
+    todo.sort(key=lambda c: 0 if "_dbl.cu" in c[2] else 1)
     if todo:
         with cf.ThreadPoolExecutor(max_workers=jobs or min(os.cpu_count() or 8, len(todo))) as ex:
             for out in ex.map(_run, todo):

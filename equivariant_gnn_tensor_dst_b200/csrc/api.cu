@@ -24,7 +24,7 @@
 #include <mutex>
 
 #include "../../include/tpconv.h"
-#include "internal.h"
+#include "launch.h"
 #include "tables.inc"
 
 using namespace tpc;
@@ -205,8 +205,25 @@ struct Layout {
   size_t gbuf = 0, part = 0;
   size_t order = 0;                 // receiver order of the pass (uvw, N ints)
   size_t total = 0;
+  long long win_edges = 0;          // edges per position-gradient staging window
   bool has_gbuf = false, has_part = false;
 };
+
+// Position-gradient staging: g_e = dL/dr_e (16 bytes per edge) is staged for a window of
+// at most win_edges edges at a time and summed into the nodes window by window.  The
+// window takes an eighth of the scratch budget (at least 32 edges, at most 16 MiB = one
+// million edges), so the workspace does not grow with the edge count.
+constexpr size_t kMaxStagingBytes = size_t(16) << 20;
+size_t staging_bytes(size_t budget) {
+  return std::max<size_t>(512, std::min(budget / 8, kMaxStagingBytes)) & ~size_t(15);
+}
+
+// Upper bound on the staging windows of one receiver range (the range's edge count is
+// known on the device only; windows past its end are empty and their launches return at
+// once).
+int windows_per_range(long long E, long long win_edges) {
+  return (int)std::max<long long>(1, (E + win_edges - 1) / win_edges);
+}
 
 // Nodes per chunk: the most that fit the budget, then evened out over the chunks that
 // number needs (so that no chunk is left with a small remainder).
@@ -220,13 +237,16 @@ int chunk_for(size_t budget_floats, long long fixed, long long per_node, long lo
 }
 
 // Workspace of one pass.  The scratch budget covers the node states of a receiver (or
-// source) range and the split-K slices of the channel contractions; backward and double
-// backward add the per-edge position-gradient staging (16 bytes per edge) on top.
+// source) range, the split-K slices of the channel contractions and, in backward and
+// double backward, the position-gradient staging window; nothing in it grows with E.
 Layout make_layout(const tpconv_plan* P, long long N, long long E, uint32_t pass) {
+  (void)E;
   Layout L;
   size_t off = 0;
   const long long st = P->dev.state_per_node, xs = P->dev.xstate_per_node;
-  const size_t bf = P->budget / 4;
+  const bool staged = pass == TPCONV_PASS_BACKWARD || pass == TPCONV_PASS_DOUBLE_BACKWARD;
+  const size_t stage = staged ? staging_bytes(P->budget) : 0;
+  const size_t bf = (P->budget - std::min(P->budget, stage)) / 4;
   if (P->mode == TPCONV_UVW) {
     const int arrays = (pass == TPCONV_PASS_DOUBLE_BACKWARD) ? 2 : 1;
     const long long fixed = (pass == TPCONV_PASS_FORWARD) ? 0 : (long long)kSplits * P->K * P->n_w;
@@ -250,10 +270,11 @@ Layout make_layout(const tpconv_plan* P, long long N, long long E, uint32_t pass
       off += align256(size_t(4) * kUvuRanges * P->K * (long long)P->n_w);
     }
   }
-  if (pass == TPCONV_PASS_BACKWARD || pass == TPCONV_PASS_DOUBLE_BACKWARD) {
+  if (staged) {
     L.has_gbuf = true;
     L.gbuf = off;
-    off += align256(size_t(16) * std::max<long long>(E, 1));
+    L.win_edges = (long long)(stage / 16);
+    off += align256(stage);
   }
   L.total = off;
   return L;
@@ -763,6 +784,14 @@ bool every_block_reached(const tpconv_plan* P, bool out_side) {
   return true;
 }
 
+// CTAs per receiver of the lane-per-edge receiver backward (each takes every split-th
+// 32-edge chunk of its receiver): twice the mean number of chunks, 1 to 8, so that
+// receivers far above the mean degree are shared while at the mean every CTA has work.
+int chunk_split(long long N, long long E) {
+  const long long mean_chunks2 = (2 * E / std::max<long long>(N, 1) + 31) / 32;
+  return (int)std::max<long long>(1, std::min<long long>(8, mean_chunks2));
+}
+
 float* fptr(void* ws, size_t off) { return reinterpret_cast<float*>(static_cast<char*>(ws) + off); }
 
 // The receiver order of a uvw pass (chunks of L.recv_chunk nodes, heaviest first), written
@@ -840,8 +869,13 @@ static tpconv_status backward_ir_mul(tpconv_plan_t P, int64_t N, int64_t E, cons
   const int edge_split = (int)std::max<long long>(1, std::min<long long>(16, (4 * E / std::max<int64_t>(N, 1) + 31) / 32));
   if (P->mode == TPCONV_UVU) {
     if (grad_pos) {
-      TPC_RUN(PC_UVU_RECV_BWD, 1, launch_uvu_recv_bwd(P->dev, P->t_in, x, pos, row_ptr, src, W, grad_out, n, gbuf, edge_split, s));
-      TPC_RUN(PC_POS, 1, launch_pos_finish(n, row_ptr, t_ptr, t_eid, gbuf, grad_pos, s));
+      TPC_TRY(cudaMemsetAsync(grad_pos, 0, sizeof(float) * 3 * (size_t)N, s));
+      for (int w = 0; w < windows_per_range(E, L.win_edges); ++w) {
+        const EdgeWindow win{0, n, w, L.win_edges};
+        TPC_RUN(PC_UVU_RECV_BWD, 1, launch_uvu_recv_bwd(P->dev, P->t_in, x, pos, row_ptr, src, W, grad_out, n, gbuf,
+                                                        win, edge_split, s));
+        TPC_RUN(PC_POS, 1, launch_pos_window(n, row_ptr, t_ptr, t_eid, gbuf, win, grad_pos, s));
+      }
     }
     if (grad_W) {
       const int nr = std::min(kUvuRanges, n);
@@ -859,12 +893,17 @@ static tpconv_status backward_ir_mul(tpconv_plan_t P, int64_t N, int64_t E, cons
   if (grad_pos) {
     DevPlan D = P->dev;
     TPC_RUN(PC_UVW_RECV_BWD, 1, attach_order(D, L, ws, n, row_ptr, s));
+    TPC_TRY(cudaMemsetAsync(grad_pos, 0, sizeof(float) * 3 * (size_t)N, s));
     for (int n0 = 0; n0 < n; n0 += L.recv_chunk) {
       const int cn = std::min(L.recv_chunk, n - n0);
       TPC_RUN(PC_GEMM, 0, gemm_sbar(P, grad_out, W, state, n0, cn, s));
-      TPC_RUN(PC_UVW_RECV_BWD, 1, launch_uvw_recv_bwd(D, P->t_in, x, pos, row_ptr, src, state, n0, cn, gbuf, edge_split, s));
+      for (int w = 0; w < windows_per_range(E, L.win_edges); ++w) {
+        const EdgeWindow win{n0, cn, w, L.win_edges};
+        TPC_RUN(PC_UVW_RECV_BWD, 1, launch_uvw_recv_edge(D, x, pos, row_ptr, src, state, n0, cn, gbuf, win,
+                                                         chunk_split(N, E), s));
+        TPC_RUN(PC_POS, 1, launch_pos_window(n, row_ptr, t_ptr, t_eid, gbuf, win, grad_pos, s));
+      }
     }
-    TPC_RUN(PC_POS, 1, launch_pos_finish(n, row_ptr, t_ptr, t_eid, gbuf, grad_pos, s));
   }
   if (grad_x && !every_block_reached(P, false))
     TPC_TRY(cudaMemsetAsync(grad_x, 0, sizeof(float) * (size_t)N * P->dim_in, s));
@@ -936,7 +975,6 @@ static tpconv_status backward_embedded_ir_mul(tpconv_plan_t P, int64_t N, int64_
   st = check_ws(L, ws, ws_bytes);
   if (st != TPCONV_OK) return st;
   const int n = (int)N;
-  float4* gbuf = reinterpret_cast<float4*>(static_cast<char*>(ws) + L.gbuf);
   float* part = fptr(ws, L.part);
   DevPlan D = P->dev;
   D.emb_Y = Y;
@@ -947,8 +985,8 @@ static tpconv_status backward_embedded_ir_mul(tpconv_plan_t P, int64_t N, int64_
   const int edge_split = (int)std::max<long long>(1, std::min<long long>(16, (4 * E / std::max<int64_t>(N, 1) + 31) / 32));
   if (P->mode == TPCONV_UVU) {
     if ((grad_phi || grad_Y) && E > 0)
-      TPC_RUN(PC_UVU_RECV_BWD, 1, launch_uvu_recv_bwd(D, P->t_in, x, nullptr, row_ptr, src, W, grad_out, n, gbuf,
-                                    edge_split, s));
+      TPC_RUN(PC_UVU_RECV_BWD, 1, launch_uvu_recv_bwd(D, P->t_in, x, nullptr, row_ptr, src, W, grad_out, n, nullptr,
+                                    whole_range(0, n), edge_split, s));
     if (grad_W) {
       const int nr = std::min(kUvuRanges, n);
       TPC_RUN(PC_UVU_GRADW, 1, launch_uvu_gradw(D, P->t_in, 0, x, nullptr, nullptr, nullptr, row_ptr, src, grad_out,
@@ -966,8 +1004,8 @@ static tpconv_status backward_embedded_ir_mul(tpconv_plan_t P, int64_t N, int64_
     for (int n0 = 0; n0 < n; n0 += L.recv_chunk) {
       const int cn = std::min(L.recv_chunk, n - n0);
       TPC_RUN(PC_GEMM, 0, gemm_sbar(P, grad_out, W, state, n0, cn, s));
-      TPC_RUN(PC_UVW_RECV_BWD, 1, launch_uvw_recv_bwd(D, P->t_in, x, nullptr, row_ptr, src, state, n0, cn, gbuf,
-                                    edge_split, s));
+      TPC_RUN(PC_UVW_RECV_BWD, 1, launch_uvw_recv_edge(D, x, nullptr, row_ptr, src, state, n0, cn, nullptr,
+                                                       whole_range(n0, cn), chunk_split(N, E), s));
     }
   }
   if (grad_x && !every_block_reached(P, false))
@@ -1031,9 +1069,13 @@ static tpconv_status double_backward_ir_mul(tpconv_plan_t P, int64_t N, int64_t 
                              grad_out, n, grad_x, s));
     if (grad_pos && any_tan) {
       // the tangent of the first-order position gradient (second derivatives of Y, phi)
-      TPC_RUN(PC_RECV_TAN, 1, launch_uvu_recv_dbl(P->dev, P->t_in, x, gg_x, pos, gg_pos, row_ptr, src, W, gg_W,
-                                                 grad_out, n, gbuf, edge_split, s));
-      TPC_RUN(PC_POS, 1, launch_pos_finish(n, row_ptr, t_ptr, t_eid, gbuf, grad_pos, s));
+      TPC_TRY(cudaMemsetAsync(grad_pos, 0, sizeof(float) * 3 * (size_t)N, s));
+      for (int w = 0; w < windows_per_range(E, L.win_edges); ++w) {
+        const EdgeWindow win{0, n, w, L.win_edges};
+        TPC_RUN(PC_RECV_TAN, 1, launch_uvu_recv_dbl(P->dev, P->t_in, x, gg_x, pos, gg_pos, row_ptr, src, W, gg_W,
+                                                   grad_out, n, gbuf, win, edge_split, s));
+        TPC_RUN(PC_POS, 1, launch_pos_window(n, row_ptr, t_ptr, t_eid, gbuf, win, grad_pos, s));
+      }
     }
     return TPCONV_OK;
   }
@@ -1078,14 +1120,18 @@ static tpconv_status double_backward_ir_mul(tpconv_plan_t P, int64_t N, int64_t 
     // of Y and phi, then the fixed-order scatter of the backward
     DevPlan D = P->dev;
     TPC_RUN(PC_RECV_TAN, 1, attach_order(D, L, ws, n, row_ptr, s));
+    TPC_TRY(cudaMemsetAsync(grad_pos, 0, sizeof(float) * 3 * (size_t)N, s));
     for (int n0 = 0; n0 < n; n0 += L.recv_chunk) {
       const int cn = std::min(L.recv_chunk, n - n0);
       TPC_RUN(PC_GEMM, 0, gemm_sbar(P, grad_out, W, sa, n0, cn, s));
       if (gg_W) TPC_RUN(PC_GEMM, 0, gemm_sbar(P, grad_out, gg_W, sb, n0, cn, s));
-      TPC_RUN(PC_RECV_TAN, 1, launch_uvw_recv_dbl(D, P->t_in, x, gg_x, pos, gg_pos, row_ptr, src, sa,
-                                                 gg_W ? sb : nullptr, n0, cn, gbuf, edge_split, s));
+      for (int w = 0; w < windows_per_range(E, L.win_edges); ++w) {
+        const EdgeWindow win{n0, cn, w, L.win_edges};
+        TPC_RUN(PC_RECV_TAN, 1, launch_uvw_recv_dbl(D, P->t_in, x, gg_x, pos, gg_pos, row_ptr, src, sa,
+                                                   gg_W ? sb : nullptr, n0, cn, gbuf, win, edge_split, s));
+        TPC_RUN(PC_POS, 1, launch_pos_window(n, row_ptr, t_ptr, t_eid, gbuf, win, grad_pos, s));
+      }
     }
-    TPC_RUN(PC_POS, 1, launch_pos_finish(n, row_ptr, t_ptr, t_eid, gbuf, grad_pos, s));
   }
   return TPCONV_OK;
 }
@@ -1274,7 +1320,9 @@ constexpr int kMaxDevices = 256;
 std::mutex g_static_mu;
 void* g_static_addr[kMaxDevices] = {};
 
-// Device address of g_static_scratch on the current device, looked up once per device.
+// Device address of g_static_scratch on the current device, looked up once per device
+// (per process: a cudaDeviceReset discards the module, so the library must not be used
+// across one).
 tpconv_status static_scratch_address(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return TPCONV_ERR_CUDA;
@@ -1290,18 +1338,26 @@ tpconv_status static_scratch_address(void** out) {
 }
 
 // Forward layout (uvw) sized for a fixed scratch: receiver ranges of node state plus
-// the split-K slices of the channel contraction.
+// the split-K slices of the channel contraction.  The two arrays are each padded to
+// 256 bytes, so the range is sized for the scratch less those paddings and then shrunk
+// while the padded total still exceeds it.
 Layout forward_layout_for(const tpconv_plan* P, long long N, size_t bytes) {
-  Layout L;
   const long long st = P->dev.state_per_node;
   const long long per_node = st + (long long)kSplits * P->dim_out;
-  const long long fit = (long long)(bytes / 4) / per_node;
-  L.recv_chunk = (int)std::max<long long>(0, std::min<long long>(fit, N));
-  L.state_a = 0;
-  const size_t one = align256(size_t(4) * L.recv_chunk * st);
-  L.has_part = true;
-  L.part = one;
-  L.total = one + align256(size_t(4) * kSplits * (long long)L.recv_chunk * P->dim_out);
+  const size_t usable = bytes > 512 ? bytes - 512 : 0;
+  long long fit = std::max<long long>(0, std::min<long long>((long long)(usable / 4) / per_node, N));
+  auto make = [&](long long chunk) {
+    Layout L;
+    L.recv_chunk = (int)chunk;
+    L.state_a = 0;
+    const size_t one = align256(size_t(4) * chunk * st);
+    L.has_part = true;
+    L.part = one;
+    L.total = one + align256(size_t(4) * kSplits * chunk * P->dim_out);
+    return L;
+  };
+  Layout L = make(fit);
+  while (fit > 0 && L.total > bytes) L = make(--fit);
   return L;
 }
 

@@ -16,12 +16,17 @@ namespace tpc {
 // spherical harmonics (polynomials in the unit direction, from the generated tables)
 // ---------------------------------------------------------------------------
 
+// Powers of the unit direction (a, b, c).  A zero-length edge arrives as (0, 0, 0) and
+// has no direction: `dir` is 0 there (1 for a unit vector), and every l > 0 harmonic
+// is scaled by it, so only the invariant Y_0 survives (the rotation-invariant value).
 struct Pow3 {
   float x[4], y[4], z[4];
+  float dir;
   __device__ __forceinline__ Pow3(float a, float b, float c) {
     x[0] = 1.f; x[1] = a; x[2] = a * a; x[3] = x[2] * a;
     y[0] = 1.f; y[1] = b; y[2] = b * b; y[3] = y[2] * b;
     z[0] = 1.f; z[1] = c; z[2] = c * c; z[3] = z[2] * c;
+    dir = (x[2] + y[2] + z[2] > 0.5f) ? 1.f : 0.f;
   }
 };
 
@@ -33,6 +38,10 @@ __device__ __forceinline__ void sh_block(const Pow3& p, float* Y) {
 #pragma unroll
   for (int t = 0; t < T::nterm; ++t)
     Y[T::k(t)] = fmaf(T::coef(t), p.x[T::ex(t)] * p.y[T::ey(t)] * p.z[T::ez(t)], Y[T::k(t)]);
+  if (L > 0) {
+#pragma unroll
+    for (int k = 0; k < 2 * L + 1; ++k) Y[k] *= p.dir;
+  }
 }
 
 // d/d(unit vector) of block L, contracted with a direction v: Yd[k] = grad P_k . v
@@ -126,7 +135,8 @@ template <int L>
 __device__ __forceinline__ void sh_block_any(int l, const Pow3& p, float* Y);
 
 // ---------------------------------------------------------------------------
-// edge geometry: r = pos[src] - pos[dst], d = |r|, r_hat = r / d (0 when d = 0)
+// edge geometry: r = pos[src] - pos[dst], d = |r|, r_hat = r / d (0 when d = 0; the
+// harmonics of that zero direction are 1 for l = 0 and 0 for l > 0, see Pow3)
 // ---------------------------------------------------------------------------
 
 struct EdgeGeo {
@@ -150,6 +160,15 @@ __device__ __forceinline__ EdgeGeo edge_geo(const float* __restrict__ pos, int i
   g.uy = g.ry * g.inv_d;
   g.uz = g.rz * g.inv_d;
   return g;
+}
+
+// Edge ids [w0, w1) of a staging window (w0 >= w1: empty).
+__device__ __forceinline__ void window_bounds(const int* __restrict__ row_ptr, const EdgeWindow& win, int& w0,
+                                              int& w1) {
+  const long long lo = __ldg(row_ptr + win.n0), hi = __ldg(row_ptr + win.n0 + win.n_nodes);
+  const long long a = lo + (long long)win.index * win.size;
+  w0 = (int)min(a, hi);
+  w1 = (int)min(a + win.size, hi);
 }
 
 // ---------------------------------------------------------------------------
@@ -375,11 +394,12 @@ __device__ __forceinline__ void recv_dbl_prep(const DevPlan& P, const float* __r
   }
 }
 
-// per edge (warp 0): the warp-ordered sums, then the tangent of g_e into gbuf
+// per edge (warp 0): the warp-ordered sums, then the tangent of g_e into gbuf (at the
+// edge id less gbase, the start of the staging window)
 template <int KP>
 __device__ __forceinline__ void recv_dbl_finish(const DevPlan& P, const float* __restrict__ pos,
                                                 const float* __restrict__ posdot, int i, int e0, int ne,
-                                                const RecvDblSmem<KP>& sm, float4* gbuf) {
+                                                const RecvDblSmem<KP>& sm, float4* gbuf, int gbase) {
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (w != 0 || lane >= ne) return;
   const int j = sm.j[lane];
@@ -409,7 +429,7 @@ __device__ __forceinline__ void recv_dbl_finish(const DevPlan& P, const float* _
     pbd[q] = b;
   }
   const float3 o = position_tangent<KP>(P, g, v.x, v.y, v.z, Yb, Ybd, pb, pbd);
-  gbuf[e0 + lane] = make_float4(o.x, o.y, o.z, 0.f);
+  gbuf[e0 + lane - gbase] = make_float4(o.x, o.y, o.z, 0.f);
 }
 
 // ---------------------------------------------------------------------------

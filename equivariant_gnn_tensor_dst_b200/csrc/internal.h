@@ -1,4 +1,6 @@
-// Internal types shared by the host plan/launch code and the kernels.
+// Internal types shared by the host plan/launch code and the kernels (the kernel
+// launchers are declared in launch.h, which kernel sources do not include, so that a new
+// launcher does not rebuild every kernel unit).
 #pragma once
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -45,6 +47,21 @@ struct DevPlan {
   const int* order;
   DevPath p[MAX_PATHS];
 };
+
+// One window of the position-gradient staging: the edges of receivers
+// [n0, n0 + n_nodes) are cut into consecutive windows of `size` edge ids, and window
+// `index` covers [row_ptr[n0] + index * size, min(that + size, row_ptr[n0 + n_nodes])).
+// The receiver kernels stage g_e of the window's edges at gbuf[e - window start]; the
+// host loops over an upper bound of the window count (empty windows do nothing), since
+// the edge count of a receiver range is known on the device only.
+struct EdgeWindow {
+  int n0, n_nodes, index;
+  long long size;
+};
+
+__host__ __device__ inline EdgeWindow whole_range(int n0, int n_nodes) {
+  return EdgeWindow{n0, n_nodes, 0, 0x7fffffffLL};
+}
 
 // A list of warp tasks: (a, b) pairs whose meaning depends on the kernel
 // (path & 32-channel chunk, or block & chunk).
@@ -108,118 +125,10 @@ struct GemmBatch {
   GemmSeg sg[MAX_GEMM_SEGS];
 };
 
-// Per-(KP, MODE) kernel runners.  Each is explicitly instantiated in its own
-// translation unit (the build compiles k_uvw.cu / k_uvu.cu once per unit) so that the
-// heavily unrolled kernels compile in parallel.
-template <int KP, int MODE>
-cudaError_t run_uvw_state(const DevPlan& P, const Tasks& T, const float* x, const float* xdot,
-                          const float* pos, const float* posdot, const int* row_ptr,
-                          const int* src, int node0, int n_nodes, float* S, float* Sdot,
-                          cudaStream_t s);
-template <int KP>
-cudaError_t run_uvw_recv_bwd(const DevPlan& P, const Tasks& T, const float* x, const float* pos,
-                             const int* row_ptr, const int* src, const float* Sbar, int node0,
-                             int n_nodes, float4* gbuf, int edge_split, cudaStream_t s);
-template <int KP, bool AD>   // AD: the A_dot tangent is present (its own build unit)
-cudaError_t run_uvw_recv_dbl(const DevPlan& P, const Tasks& T, const float* x, const float* xdot,
-                             const float* pos, const float* posdot, const int* row_ptr, const int* src,
-                             const float* Sbar, const float* Sbard, int node0, int n_nodes, float4* gbuf,
-                             int edge_split, cudaStream_t s);
-template <int KP, bool AD>
-cudaError_t run_uvu_recv_dbl(const DevPlan& P, const Tasks& T, const float* x, const float* xdot,
-                             const float* pos, const float* posdot, const int* row_ptr, const int* src,
-                             const float* W, const float* Wdot, const float* grad_out, int N, float4* gbuf,
-                             int edge_split, cudaStream_t s);
-template <int KP, int MODE>
-cudaError_t run_uvw_src_state(const DevPlan& P, const Tasks& T, const float* pos,
-                              const float* posdot, const int* t_ptr, const int* t_dst,
-                              const float* grad_out, int node0, int n_nodes, float* X,
-                              float* Xdot, cudaStream_t s);
-template <int KP, int MODE>
-cudaError_t run_uvu_fwd(const DevPlan& P, const BlockPaths& BP, const Tasks& T, const float* x,
-                        const float* xdot, const float* pos, const float* posdot,
-                        const int* row_ptr, const int* src, const float* W, const float* Wdot,
-                        int N, float* out, cudaStream_t s);
-template <int KP>
-cudaError_t run_uvu_recv_bwd(const DevPlan& P, const Tasks& T, const float* x, const float* pos,
-                             const int* row_ptr, const int* src, const float* W,
-                             const float* grad_out, int N, float4* gbuf, int edge_split, cudaStream_t s);
-template <int KP, int MODE>
-cudaError_t run_uvu_gradw(const DevPlan& P, const Tasks& T, const float* x, const float* xdot,
-                          const float* pos, const float* posdot, const int* row_ptr,
-                          const int* src, const float* grad_out, int N, int n_ranges,
-                          float* partial, cudaStream_t s);
-template <int KP, int MODE>
-cudaError_t run_uvu_src(const DevPlan& P, const BlockPaths& BP, const Tasks& T, const float* pos,
-                        const float* posdot, const int* t_ptr, const int* t_dst, const float* W,
-                        const float* Wdot, const float* grad_out, int N, float* grad_x,
-                        cudaStream_t s);
-
-// kernel launchers (dispatch on K and mode; defined in launch.cu and k_misc.cu)
-cudaError_t launch_gemm(GemmBatch& g, cudaStream_t s);     // tensor cores; fills tile0 / total_tiles
-cudaError_t launch_gemm_simt(GemmBatch& g, cudaStream_t s);  // fp32 SIMT tiles (reference kernel)
-cudaError_t launch_gemm_tc(GemmBatch& g, int* err, cudaStream_t s);
-int gemm_tiles(const GemmBatch& g);                             // output tiles of the tensor-core kernel
-int* device_error_word();                                       // set by bounded waits that give up
-cudaError_t read_and_clear_device_error(int* host_value);
-
-cudaError_t launch_uvw_state(const DevPlan& P, const Tasks& T, int mode, const float* x,
-                             const float* xdot, const float* pos, const float* posdot,
-                             const int* row_ptr, const int* src, int node0, int n_nodes,
-                             float* S, float* Sdot, cudaStream_t s);
-cudaError_t launch_uvw_recv_bwd(const DevPlan& P, const Tasks& T, const float* x,
-                                const float* pos, const int* row_ptr, const int* src,
-                                const float* Sbar, int node0, int n_nodes, float4* gbuf,
-                                int edge_split, cudaStream_t s);
-// double backward position gradient: per-edge tangent of g_e into gbuf (then pos_finish)
-cudaError_t launch_uvw_recv_dbl(const DevPlan& P, const Tasks& T, const float* x, const float* xdot,
-                                const float* pos, const float* posdot, const int* row_ptr, const int* src,
-                                const float* Sbar, const float* Sbard, int node0, int n_nodes, float4* gbuf,
-                                int edge_split, cudaStream_t s);
-cudaError_t launch_uvu_recv_dbl(const DevPlan& P, const Tasks& T, const float* x, const float* xdot,
-                                const float* pos, const float* posdot, const int* row_ptr, const int* src,
-                                const float* W, const float* Wdot, const float* grad_out, int N, float4* gbuf,
-                                int edge_split, cudaStream_t s);
-cudaError_t launch_uvw_src_state(const DevPlan& P, const Tasks& T, int mode,
-                                 const float* pos, const float* posdot, const int* t_ptr,
-                                 const int* t_eid, const int* t_dst, const float* grad_out,
-                                 int node0, int n_nodes, float* X, float* Xdot,
-                                 cudaStream_t s);
-cudaError_t launch_uvu_fwd(const DevPlan& P, const BlockPaths& BP, const Tasks& T, int mode,
-                           const float* x, const float* xdot, const float* pos,
-                           const float* posdot, const int* row_ptr, const int* src,
-                           const float* W, const float* Wdot, int N, float* out,
-                           cudaStream_t s);
-cudaError_t launch_uvu_recv_bwd(const DevPlan& P, const Tasks& T, const float* x,
-                                const float* pos, const int* row_ptr, const int* src,
-                                const float* W, const float* grad_out, int N, float4* gbuf,
-                                int edge_split, cudaStream_t s);
-cudaError_t launch_uvu_gradw(const DevPlan& P, const Tasks& T, int mode, const float* x,
-                             const float* xdot, const float* pos, const float* posdot,
-                             const int* row_ptr, const int* src, const float* grad_out,
-                             int N, int n_ranges, float* partial, cudaStream_t s);
-cudaError_t launch_uvu_src(const DevPlan& P, const BlockPaths& BP, const Tasks& T, int mode,
-                           const float* pos, const float* posdot, const int* t_ptr,
-                           const int* t_eid, const int* t_dst, const float* W,
-                           const float* Wdot, const float* grad_out, int N, float* grad_x,
-                           cudaStream_t s);
-cudaError_t launch_reduce_partials(const float* partial, int n_parts, long long n, float* out,
-                                   int accumulate, cudaStream_t s);
-cudaError_t launch_pos_finish(int N, const int* row_ptr, const int* t_ptr, const int* t_eid,
-                              const float4* gbuf, float* grad_pos, cudaStream_t s);
-cudaError_t launch_csr_transpose(int N, int E, const int* row_ptr, const int* src, int* t_ptr,
-                                 int* t_eid, int* t_dst, int* cursor, cudaStream_t s);
-cudaError_t launch_degree_order(int N, const int* row_ptr, int chunk, int* order, cudaStream_t s);
-
 // Irrep blocks of a node row, for converting between the ir_mul layout (block [2l+1][C])
 // and the mul_ir layout (block [C][2l+1]).
 struct LayoutMap {
   int n;
   int off[MAX_BLOCKS], l[MAX_BLOCKS], mul[MAX_BLOCKS];
 };
-cudaError_t launch_layout_convert(int N, int dim, const LayoutMap& M, int to_ir_mul, const float* src,
-                                  float* dst, cudaStream_t s);
-cudaError_t launch_validate_graph(int N, int E, const int* row_ptr, const int* src, int* err,
-                                  cudaStream_t s);
-
 }  // namespace tpc

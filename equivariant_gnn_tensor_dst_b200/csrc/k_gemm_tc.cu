@@ -31,7 +31,7 @@
 // bounded; a wait that gives up sets *err and the kernel still releases its TMEM.
 #include <cuda_runtime.h>
 #include <cstdint>
-#include "internal.h"
+#include "launch.h"
 #include "tpconv.h"
 
 namespace tpc {

@@ -1,140 +1,32 @@
-// Node-level contractions and graph utilities.
+// Graph utilities, the position-gradient sums and the library's device error word.
+// (The channel contractions themselves run on the tensor cores, k_gemm_tc.cu.)
 //
-//  * k_gemm / k_gemm_reduce -- the channel contractions of Sobek section 4
-//    (m = S A, eq. 35; S_bar = m_bar A^T and A_bar = S^T m_bar, eq. 36; their
-//    double-backward forms, eqs. 37-39; and the mirrored source forms x_bar = X A^T,
-//    A_bar = x^T X) on operands addressed through two-level affine index maps, so
-//    that node rows of the ir_mul tensors, the weight matrix and the workspace
-//    states are read in place.  fp32 SIMT tiles; split-K partials are reduced in a
-//    fixed order.
-//  * k_pos_finish -- position gradient: pos_bar[n] = sum_{e out of n} g_e
-//    - sum_{e into n} g_e, in source-CSR and receiver-CSR order (no atomics).
+//  * k_pos_window -- position gradient: pos_bar[n] = sum_{e out of n} g_e
+//    - sum_{e into n} g_e, one bounded staging window of g_e at a time, in source-CSR
+//    and receiver-CSR order (no atomics).
 //  * CSR transpose (stable counting sort by source) and the graph validator.
 #include <cuda_runtime.h>
-#include "internal.h"
+#include <mutex>
+#include "launch.h"
 
 namespace tpc {
 
-__device__ __forceinline__ long long ix(const Idx2& f, int i) {
-  return (long long)(i / f.d) * f.s1 + (long long)(i % f.d) * f.s2;
-}
-
-constexpr int GBM = 64, GBN = 64, GBK = 16;
-
-__global__ void __launch_bounds__(256) k_gemm(const __grid_constant__ GemmBatch g) {
-  __shared__ float As[GBK][GBM + 4];
-  __shared__ float Bs[GBK][GBN + 4];
-  const int tile = blockIdx.x;
-  int pi = 0;
-  while (pi + 1 < g.n_problems && g.pr[pi + 1].tile0 <= tile) ++pi;
-  const GemmProblem& P = g.pr[pi];
-  const int lt = tile - P.tile0;
-  const int tn = (P.N + GBN - 1) / GBN;
-  const int m0 = (lt / tn) * GBM, n0 = (lt % tn) * GBN;
-  const int split = blockIdx.y;
-  const int kper = (P.Ktot + g.splits - 1) / g.splits;
-  const int kb = split * kper, ke = min(P.Ktot, kb + kper);
-  const int tid = threadIdx.x;
-  const int tx = tid & 15, ty = tid >> 4;
-  float acc[4][4];
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
-  int kbase = 0;
-  for (int si = 0; si < P.nseg; ++si) {
-    const GemmSeg& S = g.sg[P.seg0 + si];
-    const int lo = max(kb - kbase, 0), hi = min(ke - kbase, S.K);
-    kbase += S.K;
-    for (int k0 = lo; k0 < hi; k0 += GBK) {
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int idx = tid + r * 256;
-        const int kk = idx & 15, mm = idx >> 4;
-        const int m = m0 + mm, k = k0 + kk;
-        As[kk][mm] = (m < P.M && k < hi) ? __ldg(S.A + ix(S.Am, m) + ix(S.Ak, k)) : 0.f;
-      }
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int idx = tid + r * 256;
-        const int nn = idx & 63, kk = idx >> 6;
-        const int n = n0 + nn, k = k0 + kk;
-        Bs[kk][nn] = (n < P.N && k < hi) ? __ldg(S.B + ix(S.Bk, k) + ix(S.Bn, n)) : 0.f;
-      }
-      __syncthreads();
-#pragma unroll
-      for (int kk = 0; kk < GBK; ++kk) {
-        float av[4], bv[4];
-#pragma unroll
-        for (int t = 0; t < 4; ++t) { av[t] = As[kk][ty * 4 + t]; bv[t] = Bs[kk][tx * 4 + t]; }
-#pragma unroll
-        for (int p = 0; p < 4; ++p)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) acc[p][q] = fmaf(av[p], bv[q], acc[p][q]);
-      }
-      __syncthreads();
-    }
-  }
-#pragma unroll
-  for (int p = 0; p < 4; ++p) {
-    const int m = m0 + ty * 4 + p;
-    if (m >= P.M) continue;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int n = n0 + tx * 4 + q;
-      if (n >= P.N) continue;
-      if (g.splits > 1) {
-        g.partial[P.part_off + ((long long)split * P.M + m) * P.N + n] = acc[p][q];
-      } else {
-        float* c = P.C + ix(P.Cm, m) + ix(P.Cn, n);
-        *c = g.accumulate ? *c + acc[p][q] : acc[p][q];
-      }
-    }
-  }
-}
-
-// one thread per output element of every problem; fixed-order sum over splits
-__global__ void k_gemm_reduce(const __grid_constant__ GemmBatch g, long long total) {
-  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= total) return;
-  int pi = 0;
-  long long base = 0;
-  while (pi < g.n_problems && t >= base + (long long)g.pr[pi].M * g.pr[pi].N) {
-    base += (long long)g.pr[pi].M * g.pr[pi].N;
-    ++pi;
-  }
-  const GemmProblem& P = g.pr[pi];
-  const long long loc = t - base;
-  const long long mn = (long long)P.M * P.N;
-  const int m = (int)(loc / P.N), n = (int)(loc % P.N);
-  float s = 0.f;
-  for (int sp = 0; sp < g.splits; ++sp) s += g.partial[P.part_off + sp * mn + loc];
-  float* c = P.C + ix(P.Cm, m) + ix(P.Cn, n);
-  *c = g.accumulate ? *c + s : s;
-}
-
-cudaError_t launch_gemm_simt(GemmBatch& g, cudaStream_t s) {
-  int tiles = 0;
-  long long elems = 0;
-  for (int p = 0; p < g.n_problems; ++p) {
-    g.pr[p].tile0 = tiles;
-    g.pr[p].part_off = elems * g.splits;
-    tiles += ((g.pr[p].M + GBM - 1) / GBM) * ((g.pr[p].N + GBN - 1) / GBN);
-    elems += (long long)g.pr[p].M * g.pr[p].N;
-  }
-  g.total_tiles = tiles;
-  if (tiles == 0) return cudaSuccess;
-  k_gemm<<<dim3(tiles, g.splits), 256, 0, s>>>(g);
-  if (g.splits > 1) k_gemm_reduce<<<(unsigned)((elems + 255) / 256), 256, 0, s>>>(g, elems);
-  return cudaGetLastError();
-}
-
 __device__ int g_tpc_error = 0;
 
+// Address of g_tpc_error on the current device, looked up once per device (kept for the
+// life of the process, like the static scratch of the allocation-free forward).
 int* device_error_word() {
-  static int* p = nullptr;
-  if (!p) cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_tpc_error);
-  return p;
+  static std::mutex mu;
+  static int* addr[256] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return nullptr;
+  std::lock_guard<std::mutex> g(mu);
+  if (!addr[dev]) {
+    int* p = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_tpc_error) != cudaSuccess) return nullptr;
+    addr[dev] = p;
+  }
+  return addr[dev];
 }
 
 cudaError_t launch_gemm(GemmBatch& g, cudaStream_t s) { return launch_gemm_tc(g, device_error_word(), s); }
@@ -164,29 +56,52 @@ cudaError_t launch_reduce_partials(const float* partial, int n_parts, long long 
   return cudaGetLastError();
 }
 
-__global__ void k_pos_finish(int N, const int* __restrict__ row_ptr, const int* __restrict__ t_ptr,
-                             const int* __restrict__ t_eid, const float4* __restrict__ gbuf,
+// One staging window [w0, w1) of g_e (stored at gbuf[e - w0]): every node adds the g_e of
+// its outgoing edges inside the window (source view order: t_eid is increasing within a
+// source, so they are one contiguous run, found by binary search) and subtracts those of
+// its incoming edges inside the window (a sub-range of its receiver row).  Windows are
+// applied in a fixed order, so the sums are deterministic.
+__global__ void k_pos_window(int N, const int* __restrict__ row_ptr, const int* __restrict__ t_ptr,
+                             const int* __restrict__ t_eid, const float4* __restrict__ gbuf, EdgeWindow win,
                              float* grad_pos) {
+  const long long lo = __ldg(row_ptr + win.n0), hi = __ldg(row_ptr + win.n0 + win.n_nodes);
+  const long long a = lo + (long long)win.index * win.size;
+  const int w0 = (int)min(a, hi), w1 = (int)min(a + win.size, hi);
+  if (w0 >= w1) return;
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
   if (n >= N) return;
   float x = 0.f, y = 0.f, z = 0.f;
-  for (int k = t_ptr[n]; k < t_ptr[n + 1]; ++k) {
-    const float4 g = gbuf[t_eid[k]];
+  int k0 = __ldg(t_ptr + n), k1 = __ldg(t_ptr + n + 1);
+  // first k with t_eid[k] >= w0
+  while (k0 < k1) {
+    const int mid = (k0 + k1) >> 1;
+    if (__ldg(t_eid + mid) < w0) k0 = mid + 1; else k1 = mid;
+  }
+  bool touched = false;
+  for (int k = k0, kend = __ldg(t_ptr + n + 1); k < kend; ++k) {
+    const int e = __ldg(t_eid + k);
+    if (e >= w1) break;
+    const float4 g = gbuf[e - w0];
     x += g.x; y += g.y; z += g.z;
+    touched = true;
   }
-  for (int e = row_ptr[n]; e < row_ptr[n + 1]; ++e) {
-    const float4 g = gbuf[e];
+  const int eb = max(__ldg(row_ptr + n), w0), ee = min(__ldg(row_ptr + n + 1), w1);
+  for (int e = eb; e < ee; ++e) {
+    const float4 g = gbuf[e - w0];
     x -= g.x; y -= g.y; z -= g.z;
+    touched = true;
   }
-  grad_pos[3 * n] = x;
-  grad_pos[3 * n + 1] = y;
-  grad_pos[3 * n + 2] = z;
+  if (touched) {   // nodes without an edge in the window keep their sums untouched
+    grad_pos[3 * n] += x;
+    grad_pos[3 * n + 1] += y;
+    grad_pos[3 * n + 2] += z;
+  }
 }
 
-cudaError_t launch_pos_finish(int N, const int* row_ptr, const int* t_ptr, const int* t_eid,
-                              const float4* gbuf, float* grad_pos, cudaStream_t s) {
+cudaError_t launch_pos_window(int N, const int* row_ptr, const int* t_ptr, const int* t_eid,
+                              const float4* gbuf, EdgeWindow win, float* grad_pos, cudaStream_t s) {
   if (N <= 0) return cudaSuccess;
-  k_pos_finish<<<(N + 255) / 256, 256, 0, s>>>(N, row_ptr, t_ptr, t_eid, gbuf, grad_pos);
+  k_pos_window<<<(N + 255) / 256, 256, 0, s>>>(N, row_ptr, t_ptr, t_eid, gbuf, win, grad_pos);
   return cudaGetLastError();
 }
 

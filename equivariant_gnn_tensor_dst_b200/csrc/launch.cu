@@ -1,6 +1,6 @@
 // Dispatch of the streaming kernels on the padded radial size KP (8 or 16) and on the
 // pass mode (0: primal, 1: tangent for the double backward).
-#include "internal.h"
+#include "launch.h"
 
 namespace tpc {
 
@@ -16,24 +16,32 @@ cudaError_t launch_uvw_state(const DevPlan& P, const Tasks& T, int mode, const f
   TPC_BY_KP_MODE(run_uvw_state, P, T, x, xdot, pos, posdot, row_ptr, src, node0, n_nodes, S, Sdot, s)
 }
 
-cudaError_t launch_uvw_recv_bwd(const DevPlan& P, const Tasks& T, const float* x,
-                                const float* pos, const int* row_ptr, const int* src,
-                                const float* Sbar, int node0, int n_nodes, float4* gbuf,
-                                int edge_split, cudaStream_t s) {
+cudaError_t launch_uvw_recv_edge(const DevPlan& P, const float* x, const float* pos, const int* row_ptr,
+                                 const int* src, const float* Sbar, int node0, int n_nodes, float4* gbuf,
+                                 EdgeWindow win, int split, cudaStream_t s) {
   if (n_nodes <= 0) return cudaSuccess;
-  if (edge_split < 1) edge_split = 1;
-  if (P.K <= 8) return run_uvw_recv_bwd<8>(P, T, x, pos, row_ptr, src, Sbar, node0, n_nodes, gbuf, edge_split, s);
-  return run_uvw_recv_bwd<16>(P, T, x, pos, row_ptr, src, Sbar, node0, n_nodes, gbuf, edge_split, s);
+  if (split < 1) split = 1;
+  // the fast variant needs every channel count and offset of x and of the state to be a
+  // multiple of 4 floats
+  bool fast = P.dim_in % 4 == 0 && P.state_per_node % 4 == 0;
+  for (int k = 0; k < P.n_paths; ++k)
+    fast = fast && P.p[k].c_in % 4 == 0 && P.p[k].in_off % 4 == 0 && P.p[k].st_off % 4 == 0;
+  if (P.K <= 8)
+    return fast ? run_uvw_recv_edge<8, true>(P, x, pos, row_ptr, src, Sbar, node0, n_nodes, gbuf, win, split, s)
+                : run_uvw_recv_edge<8, false>(P, x, pos, row_ptr, src, Sbar, node0, n_nodes, gbuf, win, split, s);
+  return fast ? run_uvw_recv_edge<16, true>(P, x, pos, row_ptr, src, Sbar, node0, n_nodes, gbuf, win, split, s)
+              : run_uvw_recv_edge<16, false>(P, x, pos, row_ptr, src, Sbar, node0, n_nodes, gbuf, win, split, s);
 }
 
 cudaError_t launch_uvw_recv_dbl(const DevPlan& P, const Tasks& T, const float* x, const float* xdot,
                                 const float* pos, const float* posdot, const int* row_ptr, const int* src,
                                 const float* Sbar, const float* Sbard, int node0, int n_nodes, float4* gbuf,
-                                int edge_split, cudaStream_t s) {
+                                EdgeWindow win, int edge_split, cudaStream_t s) {
   if (n_nodes <= 0) return cudaSuccess;
   if (edge_split < 1) edge_split = 1;
 #define TPC_RUN_DBL(KP, AD) \
-  return run_uvw_recv_dbl<KP, AD>(P, T, x, xdot, pos, posdot, row_ptr, src, Sbar, Sbard, node0, n_nodes, gbuf, edge_split, s)
+  return run_uvw_recv_dbl<KP, AD>(P, T, x, xdot, pos, posdot, row_ptr, src, Sbar, Sbard, node0, n_nodes, gbuf, win, \
+                                  edge_split, s)
   if (P.K <= 8) {
     if (Sbard) TPC_RUN_DBL(8, true);
     TPC_RUN_DBL(8, false);
@@ -46,11 +54,12 @@ cudaError_t launch_uvw_recv_dbl(const DevPlan& P, const Tasks& T, const float* x
 cudaError_t launch_uvu_recv_dbl(const DevPlan& P, const Tasks& T, const float* x, const float* xdot,
                                 const float* pos, const float* posdot, const int* row_ptr, const int* src,
                                 const float* W, const float* Wdot, const float* grad_out, int N, float4* gbuf,
-                                int edge_split, cudaStream_t s) {
+                                EdgeWindow win, int edge_split, cudaStream_t s) {
   if (N <= 0) return cudaSuccess;
   if (edge_split < 1) edge_split = 1;
 #define TPC_RUN_DBL(KP, AD) \
-  return run_uvu_recv_dbl<KP, AD>(P, T, x, xdot, pos, posdot, row_ptr, src, W, Wdot, grad_out, N, gbuf, edge_split, s)
+  return run_uvu_recv_dbl<KP, AD>(P, T, x, xdot, pos, posdot, row_ptr, src, W, Wdot, grad_out, N, gbuf, win, \
+                                  edge_split, s)
   if (P.K <= 8) {
     if (Wdot) TPC_RUN_DBL(8, true);
     TPC_RUN_DBL(8, false);
@@ -82,11 +91,11 @@ cudaError_t launch_uvu_fwd(const DevPlan& P, const BlockPaths& BP, const Tasks& 
 cudaError_t launch_uvu_recv_bwd(const DevPlan& P, const Tasks& T, const float* x,
                                 const float* pos, const int* row_ptr, const int* src,
                                 const float* W, const float* grad_out, int N, float4* gbuf,
-                                int edge_split, cudaStream_t s) {
+                                EdgeWindow win, int edge_split, cudaStream_t s) {
   if (N <= 0) return cudaSuccess;
   if (edge_split < 1) edge_split = 1;
-  if (P.K <= 8) return run_uvu_recv_bwd<8>(P, T, x, pos, row_ptr, src, W, grad_out, N, gbuf, edge_split, s);
-  return run_uvu_recv_bwd<16>(P, T, x, pos, row_ptr, src, W, grad_out, N, gbuf, edge_split, s);
+  if (P.K <= 8) return run_uvu_recv_bwd<8>(P, T, x, pos, row_ptr, src, W, grad_out, N, gbuf, win, edge_split, s);
+  return run_uvu_recv_bwd<16>(P, T, x, pos, row_ptr, src, W, grad_out, N, gbuf, win, edge_split, s);
 }
 
 cudaError_t launch_uvu_gradw(const DevPlan& P, const Tasks& T, int mode, const float* x,

@@ -128,9 +128,10 @@ tpconv_status tpconv_plan_path(tpconv_plan_t plan, int64_t index, int32_t out[10
 tpconv_status tpconv_plan_path_coupling(tpconv_plan_t plan, int64_t index, int32_t* idx,
                                         double* val, int64_t cap);
 
-/* Upper bound on the node-state scratch used per call (the pages cap tensor-product
- * scratch at 128 MiB, which is the default).  Larger budgets mean fewer receiver
- * ranges; results do not depend on it.                                              */
+/* Upper bound on the tensor-product scratch used per call (the pages cap it at 128 MiB,
+ * which is the default): node states, split-K slices and the position-gradient staging
+ * window.  Larger budgets mean fewer receiver ranges and staging windows; results do
+ * not depend on it beyond the order of fp32 sums.  At least 4096 bytes.               */
 tpconv_status tpconv_set_workspace_budget(tpconv_plan_t plan, size_t bytes);
 
 /* Arithmetic of the channel contractions (the per-node products with the radial
@@ -160,9 +161,11 @@ tpconv_status tpconv_plan_set_math(tpconv_plan_t plan, int32_t math);
 tpconv_status tpconv_plan_set_layout(tpconv_plan_t plan, int32_t layout);
 
 /* Workspace bytes needed by the passes in pass_mask for a graph of N nodes and E
- * edges.  The node-state part is bounded by the budget and does not grow with E;
- * backward and double backward add 16 bytes per edge of position-gradient staging
- * (used only when a position gradient is requested).                                 */
+ * edges.  The result does not depend on E: the node states of a receiver (or source)
+ * range, the split-K slices of the channel contractions and, in backward and double
+ * backward, a staging window for the per-edge position gradients (an eighth of the
+ * budget, at most 16 MiB; the edges are staged window by window) all fit the scratch
+ * budget (tpconv_set_workspace_budget), plus 4 bytes per node of receiver order.       */
 tpconv_status tpconv_workspace_bytes(tpconv_plan_t plan, int64_t N, int64_t E,
                                      uint32_t pass_mask, size_t* bytes);
 
@@ -246,12 +249,14 @@ tpconv_status tpconv_backward_embedded(tpconv_plan_t plan, int64_t N, int64_t E,
  * owns every device allocation, or code that must not call cudaMalloc because that
  * call can synchronise the device in the middle of latency-critical work.
  *
- * Same inputs, outputs and result as tpconv_forward (eq. 11 with eq. 12, evaluated as
- * eqs. 32-35), but the scratch lives in a fixed array of TPCONV_STATIC_SCRATCH_BYTES
- * compiled into the library, which every GPU that loads the library keeps until the
- * process exits.  The pages have no counterpart to this entry point.
+ * Same inputs, outputs and result as tpconv_forward, but the scratch lives in a fixed
+ * array of TPCONV_STATIC_SCRATCH_BYTES compiled into the library, which every GPU that
+ * loads the library keeps until the process exits.  The paper has no counterpart to
+ * this entry point.
  *  - The first call on a device looks up that array's device address (once per device,
- *    with the device current); make that first call before any stream capture.
+ *    with the device current); make that first call before any stream capture.  The
+ *    address is kept for the life of the process, so do not use the library across a
+ *    cudaDeviceReset.
  *  - Plans whose per-receiver state does not fit the array even one receiver at a time
  *    are rejected with TPCONV_ERR_WORKSPACE_TOO_SMALL; larger graphs are processed in
  *    receiver ranges that fit.
