@@ -1,9 +1,14 @@
 """Benchmark of the streaming tensor-product convolution on B200.
 
 One step = one pass of the whole hot path over one batch: forward plus backward
-(gradients with respect to x, positions and W) of the uvw workload
-"64x0e+64x1o+64x2e, SH lmax 3, N=4096, kNN k=32, E=131072, K=8 Bessel, cutoff 5"
-(synthetic, seeded).  Metric: edges per second of the step (higher is better).
+(gradients with respect to x, positions and W) of the edge-scaling uvw workload
+"128x0e+64x1o+32x2e+16x3o, SH lmax 3, N=50000, power-law in-degrees 16..512 (E about
+2.8M), K=8 Bessel, cutoff 6" (synthetic, seeded), the largest of the method's workloads.
+Metric: edges per second of the step (higher is better).  The line also reports
+edges/s of each pass on its own (forward and backward of the step's workload, the
+force-training double backward, and the N=4096 uvw workload), the roofline of the
+whole step (the slower of its FP32 work, tensor-core work and compulsory HBM bytes
+at the peaks) and of its dominant kernel, and the peak workspace.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
 
@@ -32,21 +37,15 @@ from equivariant_gnn_tensor_dst_b200 import workloads  # noqa: E402
 
 METRIC = "TP-conv edges/sec fwd/bwd/double-bwd; % of roofline; peak workspace bytes"
 UNIT = "edges/s"
-CFG = 2
+CFG = 4                                             # the step's workload (edge scaling, uvw)
 FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # SM count x FP32 lanes x FMA x max clock
 L2_FLUSH_BYTES = 256 << 20                          # > 126 MB L2
 TF32_PER_BF16 = 1.1 / 2.25                          # nominal dense TF32 / BF16 tensor rates
 SPLIT_MMAS = 3                                      # 3xTF32: three TF32 products per fp32 product
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per step of the N=4096 uvw
-# workload for each kernel category, from one ncu capture of the 2048-node case whose
-# launches have the same 1024-node chunk shape (per step: twice its launches).  Valid for
-# the kernels as captured; only reported for that workload.
-TRAFFIC_BYTES_PER_STEP = {
-    "channel_gemm": 2 * (6 * 92.09e6 + 2 * 32.81e6 + 6 * 9.45e6),
-    "uvw_receiver_backward": 4 * 95.52e6,
-    "uvw_source_state": 4 * 35.29e6,
-    "uvw_receiver_state": 4 * 35.07e6,
-}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per step for a kernel category
+# of the step's workload, from an ncu capture of the kernels as they are now (scaled from
+# the captured case by the edges processed).  None: no capture of the current kernels.
+TRAFFIC_BYTES_PER_STEP = {}
 
 
 def measured_peaks():
@@ -61,22 +60,10 @@ def measured_peaks():
         return {"hbm_gbs": 6650.0, "bf16": 1590.0, "source": "of fallback (6.65 TB/s, 1.59 PFLOP/s bf16 burst)"}
 
 
-def _workload_config(c, E):
-    return {"workload": "uvw forward+backward, N=4096 kNN k=32 (E=131072), 64x0e+64x1o+64x2e, "
-                        "SH lmax 3, K=8 Bessel r_c=5",
-            "nodes": c.n_nodes, "edges": int(E), "irreps": c.irreps_in, "sh_lmax": c.sh_lmax,
-            "mode": c.mode, "radial": f"{c.radial} K={c.num_basis} r_c={c.r_cut}",
-            "pass": "forward + backward (x, pos, W)", "l2": "flushed between timed steps"}
-
-
-def _config_line(c, g):
-    d = _workload_config(c, g.n_edges)
-    if c.cfg != CFG:
-        d["workload"] = c.name
-        d.update({"irreps": c.irreps_in, "sh_lmax": c.sh_lmax, "mode": c.mode,
-                  "radial": f"{c.radial} K={c.num_basis} r_c={c.r_cut}"})
-    d["nodes"] = g.n_nodes
-    return d
+def _workload_config(c, g, passes="forward + backward (x, pos, W)"):
+    return {"workload": c.name, "nodes": int(g.n_nodes), "edges": int(g.n_edges), "irreps": c.irreps_in,
+            "sh_lmax": c.sh_lmax, "mode": c.mode, "radial": f"{c.radial} K={c.num_basis} r_c={c.r_cut}",
+            "pass": passes, "l2": "flushed between timed steps"}
 
 
 def _dist():
@@ -106,8 +93,12 @@ def reduce_over_ranks(total_ms, edges, device=None):
 # ---------------------------------------------------------------------------
 
 def flop_model(plan):
+    """Per-edge and per-node operation counts of each kernel category, from the plan's
+    paths (FMA = 2 flop).  Only the work the streaming evaluation has to do is counted,
+    not the materialised per-edge weights it avoids."""
     K = plan.num_basis
-    f = dict(state=0, recv=0, src=0, gemm_node=0, gemm_node_bytes=0, uvu_fwd=0, uvu_recv=0, uvu_gradw=0, uvu_src=0)
+    f = dict(state=0, recv=0, src=0, state_tan=0, src_tan=0, gemm_node=0, gemm_fwd_node=0, gemm_dbl_node=0,
+             gemm_node_bytes=0, uvu_fwd=0, uvu_recv=0, uvu_gradw=0, uvu_src=0)
     for p in plan.paths():
         ri, ro = 2 * p["l_in"] + 1, 2 * p["l_out"] + 1
         nnz, ci, co = p["nnz"], p["c_in"], p["c_out"]
@@ -121,14 +112,68 @@ def flop_model(plan):
         f["state"] += 2 * ci * (nnz + K * ro)              # eq. 32 coupling + eq. 33 outer product
         f["recv"] += 2 * ci * (2 * nnz + 2 * K * ro)       # coupling, phi_bar, T_bar, Y_bar
         f["src"] += 2 * co * (nnz + K * ri)                # adjoint coupling + source state
+        # tangents along pos_dot (double backward, gg_pos alone): coupling with Y and Y_dot,
+        # outer products with phi and phi_dot, on each side
+        f["state_tan"] += 2 * ci * (2 * nnz + 2 * K * ro)
+        f["src_tan"] += 2 * co * (2 * nnz + 2 * K * ri)
         # S A, m_bar A^T (receiver side); X A^T, x^T X (source side, which also gives A_bar)
         f["gemm_node"] += 2 * K * ci * co * (2 * ro + 2 * ri)
+        f["gemm_fwd_node"] += 2 * K * ci * co * ro
+        # double backward: grad_W = S_dot^T m_bar, grad_x = X' A^T
+        f["gemm_dbl_node"] += 2 * K * ci * co * (ro + ri)
         # fp32 operand bytes of the four channel contractions of a forward+backward step:
         # m = S A (read S, write m), S_bar = m_bar A^T (read m_bar, write S_bar),
         # x_bar = X A^T (read X, write x_bar), A_bar = x^T X (read x, X); the weights stay
         # in L2.
         f["gemm_node_bytes"] += 4 * (2 * ro * K * ci + 2 * ro * co + 2 * ri * K * co + 2 * ri * ci)
     return f
+
+
+def pass_counts(plan, N, E, which):
+    """Algorithmic FP32 (SIMT) flops, tensor-core flops and compulsory HBM bytes of one
+    pass ("fwd", "bwd" with x, pos and W gradients, "fwd+bwd", or "dbl": the force-
+    training double backward with gg_pos alone, returning grad_x and grad_W).
+    Compulsory bytes: every input read once and every output written once (x, pos, the
+    graph, A, upstream gradients and tangents; results)."""
+    f = flop_model(plan)
+    din, dout, nw = plan.dim_in, plan.dim_out, plan.num_basis * plan.weight_cols
+    uvu = plan.mode == "uvu"
+    graph = 4 * (N + 1) + 4 * E
+    tgraph = 4 * (N + 1) + 8 * E
+    fwd = dict(simt=E * (f["uvu_fwd"] if uvu else f["state"]), tc=0 if uvu else N * f["gemm_fwd_node"],
+               bytes=4 * (N * din + 3 * N + nw + N * dout) + graph)
+    bwd = dict(simt=E * ((f["uvu_recv"] + f["uvu_gradw"] + f["uvu_src"]) if uvu else (f["recv"] + f["src"])),
+               # backward contractions: S_bar = m_bar A^T (receiver), x_bar = X A^T, A_bar = x^T X
+               tc=0 if uvu else N * (f["gemm_node"] - f["gemm_fwd_node"]),
+               bytes=4 * (N * din + 3 * N + nw + N * dout) + graph + tgraph + 4 * (N * din + 3 * N + nw))
+    dbl = dict(simt=E * (f["state_tan"] + f["src_tan"]), tc=N * f["gemm_dbl_node"],
+               bytes=4 * (N * din + 3 * N + nw + N * dout + 3 * N + N * din + nw) + graph + tgraph)
+    if which == "fwd":
+        return fwd
+    if which == "bwd":
+        return bwd
+    if which == "dbl":
+        return dbl
+    both = dict(simt=fwd["simt"] + bwd["simt"], tc=fwd["tc"] + bwd["tc"],
+                bytes=bwd["bytes"] + 4 * N * dout)   # the forward adds only its output
+    return both
+
+
+def step_roofline(counts, ms, peaks):
+    """T_roof = max(F_simt / P_fp32, F_tc / P_tc, B_comp / BW_hbm) against the measured
+    time; P_tc for fp32 products is three TF32 products at the nominal TF32/BF16 ratio of
+    the measured BF16 peak."""
+    tc_peak = peaks["bf16"] * TF32_PER_BF16 / SPLIT_MMAS
+    t = {"fp32_alu": counts["simt"] / (FP32_PEAK_TFLOPS * 1e12),
+         "tensor_3xtf32": counts["tc"] / (tc_peak * 1e12),
+         "hbm": counts["bytes"] / (peaks["hbm_gbs"] * 1e9)}
+    bound = max(t, key=t.get)
+    t_roof = t[bound]
+    return {"bound": bound, "t_roof_ms": round(t_roof * 1e3, 4), "t_measured_ms": round(ms, 4),
+            "frac": round(t_roof / (ms / 1e3), 4), "simt_gflop": round(counts["simt"] / 1e9, 3),
+            "tc_gflop": round(counts["tc"] / 1e9, 3), "compulsory_mb": round(counts["bytes"] / 1e6, 2),
+            "peaks": {"fp32_tflops": round(FP32_PEAK_TFLOPS, 1), "tc_tflops": round(tc_peak, 1),
+                      "hbm_gbs": peaks["hbm_gbs"]}}
 
 
 # ---------------------------------------------------------------------------
@@ -252,7 +297,9 @@ def run_native(args):
     torch.cuda.synchronize()
     sampler.start()
     time.sleep(0.25)
-    binding.tpconv_profile_begin(max(8192, 64 * args.steps))
+    # enough records for every launch scope of the timed steps (a scope that finds the pool
+    # full is counted but not timed)
+    binding.tpconv_profile_begin(8192 + 4096 * args.steps)
     for k in range(args.steps):
         flush.zero_()
         starts[k].record(stream)
@@ -266,6 +313,12 @@ def run_native(args):
     total_ms, edges_all = reduce_over_ranks(total_ms, E, dev)
     ms_step = total_ms / args.steps
     value = edges_all * args.steps / (total_ms / 1e3)
+
+    # a bounded wait inside a tensor-core kernel that gave up skips that launch's work: a
+    # timed region that set the device error word is not a measurement
+    dev_err = binding.tpconv_device_error()
+    if dev_err != 0:
+        raise SystemExit(f"device error word {dev_err} set during the timed region: no measurement")
 
     # live roofline of every kernel category (CUDA events over the timed region)
     fm = flop_model(plan)
@@ -284,23 +337,15 @@ def run_native(args):
             continue
         ach = algo[k] / (ms / args.steps / 1e3) / 1e12
         if k == "channel_gemm":
-            # the channel contraction is bound by whichever of its tensor-core time and its
-            # HBM time is longer at the peaks
-            t_tc = algo[k] / (tc_peak * 1e12)
-            t_hbm = fm["gemm_node_bytes"] * N / (peaks["hbm_gbs"] * 1e9)
-            if t_tc >= t_hbm:
-                rl = {"bound": "tensor", "achieved": round(ach, 3), "peak": round(tc_peak, 1), "unit": "TFLOP/s",
-                      "peak_note": f"fp32 products via 3xTF32: bf16 x {TF32_PER_BF16:.3f} (nominal TF32/BF16) "
-                                   f"/ {SPLIT_MMAS}, bf16 {peaks['source']}"}
-            else:
-                gbs = fm["gemm_node_bytes"] * N / (ms / args.steps / 1e3) / 1e9
-                rl = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                      "peak_note": f"HBM copy bandwidth {peaks['source']}"}
-            rl["algorithmic_per_step"] = {"flop": algo[k], "bytes": fm["gemm_node_bytes"] * N}
+            # the channel contractions are bound by the tensor cores (fp32 products from three
+            # TF32 products); their compulsory bytes are a small part of the step's
+            rl = {"bound": "tensor", "achieved": round(ach, 3), "peak": round(tc_peak, 1), "unit": "TFLOP/s",
+                  "peak_note": f"fp32 products via 3xTF32: bf16 x {TF32_PER_BF16:.3f} (nominal TF32/BF16) "
+                               f"/ {SPLIT_MMAS}, bf16 {peaks['source']}"}
         else:
             rl = {"bound": "alu", "achieved": round(ach, 3), "peak": round(FP32_PEAK_TFLOPS, 1), "unit": "TFLOP/s",
                   "peak_note": "derived: 148 SMs x 128 FP32 lanes x 2 flop x 1965 MHz"}
-            rl["algorithmic_per_step"] = {"flop": algo[k]}
+        rl["algorithmic_per_step"] = {"flop": algo[k]}
         rl["frac"] = round(rl["achieved"] / rl["peak"], 4)
         headline = args.cfg == CFG and args.nodes is None
         tb = TRAFFIC_BYTES_PER_STEP.get(k) if headline else None
@@ -313,6 +358,21 @@ def run_native(args):
     breakdown = {k: {"ms_per_step": round(v[0] / args.steps, 4), "launches_per_step": v[1] / args.steps,
                      "share": round(v[0] / timed_ms, 4) if timed_ms else None} for k, v in kern.items()}
     total_algo = sum(v for k, v in algo.items() if k in kern)
+    step_roof = step_roofline(pass_counts(plan, N, E, "fwd+bwd"), ms_step, peaks)
+
+    # each pass on its own: forward and backward of this workload, the force-training double
+    # backward, and the N=4096 uvw workload's forward and backward
+    passes = None
+    if not args.no_passes and rank == 0:
+        passes = {"this_workload": time_passes(plan, c, N, E, dict(x=x, pos=pos, row_ptr=row_ptr, src=src, W=W,
+                                                                   gout=gout, views=(t_ptr, t_eid, t_dst)),
+                                               ws, flush, args, peaks, ("fwd", "bwd"))}
+        for cfg in (5, 2):
+            if cfg != args.cfg:
+                passes[f"workload_{cfg}"] = time_workload(cfg, dev, flush, args, peaks)
+        err2 = binding.tpconv_device_error()
+        if err2 != 0:
+            raise SystemExit(f"device error word {err2} set while timing the passes: no measurement")
 
     # end-to-end through the public API: pinned host inputs in, results out, every step
     e2e = None
@@ -362,13 +422,15 @@ def run_native(args):
         line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-                "config": _config_line(c, g), "impl": "native",
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": gpu_launches,
+                "config": _workload_config(c, g), "impl": "native",
+                "roofline": roofline, "step_roofline": step_roof, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": gpu_launches,
                 "gpu_launches_per_step": gpu_launches / args.steps, "clocks": clocks,
                 "workspace_bytes": {"declared": int(ws_bytes), "peak_alloc_delta": int(peak_delta)},
+                "device_error_word": 0,
                 "step_algorithmic_tflop": round(total_algo / 1e12, 4),
                 "step_tflops_achieved": round(total_algo / (ms_step / 1e3) / 1e12, 3),
-                "breakdown": breakdown, "rooflines": rooflines}
+                "breakdown": breakdown, "rooflines": rooflines, "passes": passes}
         if extras is not None:
             line["extras"] = extras
         print(json.dumps(line), flush=True)
@@ -395,6 +457,81 @@ def _timed(fn, flush, steps, warmup):
         b.record()
     torch.cuda.synchronize()
     return sum(a.elapsed_time(b) for a, b in ev) / steps
+
+
+def _scalar_mask(c, dim_out):
+    mask = np.zeros(dim_out, np.float32)
+    off = 0
+    for tok in c.irreps_out.split("+"):
+        mul, ir = tok.split("x")
+        l = int(ir[:-1])
+        if l == 0 and ir[-1] == "e":
+            mask[off:off + int(mul)] = 1.0
+        off += int(mul) * (2 * l + 1)
+    return mask
+
+
+def time_passes(plan, c, N, E, t, ws, flush, args, peaks, which):
+    """CUDA-event time, edges/s and step roofline of each pass in `which` on resident
+    inputs t (dict of device tensors).  "dbl" is the force-training double backward:
+    m_bar = 1 on every scalar output channel, gg_pos = 2 (pos_bar + F_ref) from a first
+    backward, outputs grad_x and grad_W."""
+    import torch
+
+    from equivariant_gnn_tensor_dst_b200 import binding
+    dev = t["x"].device
+    steps, warm = max(5, min(args.steps, 20)), 3
+    o = torch.empty(N, plan.dim_out, device=dev)
+    gx = torch.empty(N, plan.dim_in, device=dev)
+    gp = torch.empty(N, 3, device=dev)
+    gw = torch.empty(plan.num_basis, plan.weight_cols, device=dev)
+    rec = {}
+    for name in which:
+        if name == "fwd":
+            fn = lambda: binding.tpconv_forward(plan, t["x"], t["pos"], t["row_ptr"], t["src"], t["W"],  # noqa: E731
+                                                out=o, ws=ws)
+        elif name == "bwd":
+            fn = lambda: binding.tpconv_backward(plan, t["x"], t["pos"], t["row_ptr"], t["src"],  # noqa: E731
+                                                 *t["views"], t["W"], t["gout"], ws=ws, outputs=(gx, gp, gw))
+        else:
+            mbar = torch.from_numpy(np.tile(_scalar_mask(c, plan.dim_out), (N, 1))).to(dev)
+            F_ref = torch.from_numpy(workloads.normal(np.random.default_rng(1000 + c.cfg + 1), (N, 3))).to(dev)
+            binding.tpconv_backward(plan, t["x"], t["pos"], t["row_ptr"], t["src"], *t["views"], t["W"], mbar,
+                                    ws=ws, outputs=(None, gp, None))
+            gg = torch.mul(torch.add(gp, F_ref), 2.0)      # d loss / d pos_bar
+            fn = lambda: binding.tpconv_double_backward(plan, t["x"], t["pos"], t["row_ptr"], t["src"],  # noqa: E731
+                                                        *t["views"], t["W"], mbar, gg_pos=gg, ws=ws,
+                                                        outputs=(gx, gw, None))
+        ms = _timed(fn, flush, steps, warm)
+        key = {"fwd": "forward", "bwd": "backward", "dbl": "double_backward"}[name]
+        rec[key] = {"ms": round(ms, 4), "edges_per_s": round(E / ms * 1e3, 1),
+                    "roofline": step_roofline(pass_counts(plan, N, E, name), ms, peaks)}
+    return rec
+
+
+def time_workload(cfg, dev, flush, args, peaks):
+    """Every pass of workload `cfg` (its own graph and inputs) with time_passes."""
+    import torch
+
+    from equivariant_gnn_tensor_dst_b200 import binding
+    c = workloads.CONFIGS[cfg]
+    plan = binding.Plan(c.irreps_in, c.sh_lmax, c.irreps_out, c.mode, c.radial, c.num_basis, c.r_cut,
+                        c.r_min, c.r_max)
+    g, rng = workloads.make_graph(c)
+    N, E = g.n_nodes, g.n_edges
+    tt = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)  # noqa: E731
+    t = dict(x=tt(workloads.normal(rng, (N, plan.dim_in))),
+             W=tt(workloads.weights(rng, c.num_basis, plan.fan_in_per_column())),
+             gout=tt(workloads.normal(rng, (N, plan.dim_out))), pos=tt(g.pos), row_ptr=tt(g.row_ptr),
+             src=tt(g.src))
+    t["views"] = binding.tpconv_csr_transpose(t["row_ptr"], t["src"], N)
+    wsb = plan.workspace_bytes(N, E)
+    ws = binding.workspace(wsb, dev)
+    rec = {"workload": c.name, "nodes": N, "edges": E, "workspace_bytes": int(wsb)}
+    rec.update(time_passes(plan, c, N, E, t, ws, flush, args, peaks, c.passes))
+    del ws, t
+    torch.cuda.empty_cache()
+    return rec
 
 
 def run_extras(args, dev, flush):
@@ -466,15 +603,7 @@ def run_extras(args, dev, flush):
         if "dbl" in c.passes:
             # force training: energy = sum of scalar outputs, F = -dE/dpos, loss |F - F_ref|^2,
             # then d loss / d(W, x) by the double backward
-            mask = np.zeros(plan.dim_out, np.float32)
-            off = 0
-            for tok in c.irreps_out.split("+"):
-                mul, ir = tok.split("x")
-                l = int(ir[:-1])
-                if l == 0 and ir[-1] == "e":
-                    mask[off:off + int(mul)] = 1.0
-                off += int(mul) * (2 * l + 1)
-            mbar = tt(np.tile(mask, (N, 1)))
+            mbar = tt(np.tile(_scalar_mask(c, plan.dim_out), (N, 1)))
             F_ref = tt(workloads.normal(rng, (N, 3)))
             dx = torch.empty(N, plan.dim_in, device=dev)
             dw = torch.empty(plan.num_basis, plan.weight_cols, device=dev)
@@ -593,10 +722,12 @@ def _oracle_sample(seconds_target):
 
     def run(n_recv):
         edges = np.arange(rp[0], rp[n_recv])
-        t0 = time.perf_counter()
+        t0, c0 = time.perf_counter(), time.process_time()
         conv.forward(op, x, g.pos, g.row_ptr, g.src, W, edges=edges)
         conv.backward(op, x, g.pos, g.row_ptr, g.src, W, go, edges=edges)
-        return time.perf_counter() - t0, edges.size
+        dt = time.perf_counter() - t0
+        run.cores = (time.process_time() - c0) / max(dt, 1e-9)   # CPU seconds per wall second
+        return dt, edges.size
 
     # warm up, calibrate on a small sample, then size the sample for the target duration
     run(2)
@@ -605,7 +736,7 @@ def _oracle_sample(seconds_target):
     return run, n_recv, g
 
 
-def _threads_used():
+def _threads_available():
     try:
         from threadpoolctl import threadpool_info
         return max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
@@ -616,7 +747,10 @@ def _threads_used():
 def cpu_baseline(seconds):
     run, n_recv, g = _oracle_sample(seconds)
     dt, ne = run(n_recv)
-    return {"value": round(ne / dt, 2), "unit": UNIT, "cores": _threads_used(), "kind": "oracle",
+    # cores = the CPU time the oracle's process used per second of wall time (its numpy
+    # kernels use a thread pool only in some steps), not the size of that pool
+    return {"value": round(ne / dt, 2), "unit": UNIT, "cores": round(run.cores, 2), "kind": "oracle",
+            "threads_available": _threads_available(),
             "sample": f"forward+backward over the first {n_recv} receivers ({ne} edges) of the workload",
             "seconds": round(dt, 2)}
 
@@ -628,19 +762,21 @@ def run_reference(args):
     run, n_recv, g = _oracle_sample(args.cpu_seconds / max(1, args.steps))
     for _ in range(args.warmup):
         run(min(n_recv, 8))
-    times, ne = [], 0
+    times, cores, ne = [], [], 0
     for _ in range(args.steps):
         dt, ne = run(n_recv)
         times.append(dt)
+        cores.append(run.cores)
     total = sum(times)
     value = ne * args.steps / total
     c = workloads.CONFIGS[CFG]
-    cpu = {"value": round(value, 2), "unit": UNIT, "cores": _threads_used(), "kind": "oracle",
+    cpu = {"value": round(value, 2), "unit": UNIT, "cores": round(statistics.median(cores), 2), "kind": "oracle",
+           "threads_available": _threads_available(),
            "sample": f"each step: forward+backward over the first {n_recv} receivers ({ne} edges)"}
     line = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": _workload_config(c, g.n_edges), "impl": "reference", "cpu_baseline": cpu,
+            "config": _workload_config(c, g), "impl": "reference", "cpu_baseline": cpu,
             "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -648,17 +784,19 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("native", "reference"), default="native")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-passes", action="store_true",
+                    help="skip timing each pass on its own (this workload, force training, N=4096 uvw)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--extras", action="store_true",
                     help="also time every pass on the other workloads (adds ~1-2 minutes)")
     ap.add_argument("--extras-cfgs", type=int, nargs="*", default=[2, 3, 5, 4])
     ap.add_argument("--cfg", type=int, default=CFG, choices=sorted(workloads.CONFIGS),
-                    help="workload of the timed step (default: the uvw forward+backward workload)")
+                    help="workload of the timed step (default: the edge-scaling uvw workload)")
     ap.add_argument("--nodes", type=int, default=None,
                     help="resize the workload (same density and degree); for profiling small cases")
     ap.add_argument("--profiles", action="store_true",
