@@ -15,7 +15,7 @@ LIB_PATH = os.path.join(_HERE, "libtpconv.so")
 UVW, UVU = 0, 1
 BESSEL, GAUSSIAN = 0, 1
 PASS_FORWARD, PASS_BACKWARD, PASS_DOUBLE_BACKWARD = 1, 2, 4
-MATH_FP32, MATH_TF32 = 0, 1
+MATH_FP32, MATH_TF32, MATH_BF16 = 0, 1, 2
 LAYOUT_IR_MUL, LAYOUT_MUL_IR = 0, 1
 
 _c_i64 = ctypes.c_int64
@@ -155,7 +155,8 @@ class Plan:
         check(lib().tpconv_plan_set_layout(self._h, int(layout)), "tpconv_plan_set_layout")
 
     def set_math(self, math):
-        """MATH_FP32 (default, 3xTF32 contractions) or MATH_TF32 (one TF32 product)."""
+        """MATH_FP32 (default, 3xTF32 contractions), MATH_TF32 (one TF32 product) or
+        MATH_BF16 (operands rounded to bf16, one bf16 product)."""
         check(lib().tpconv_plan_set_math(self._h, int(math)), "tpconv_plan_set_math")
 
     def workspace_bytes(self, n_nodes, n_edges, passes=PASS_FORWARD | PASS_BACKWARD | PASS_DOUBLE_BACKWARD):

@@ -206,6 +206,7 @@ struct Layout {
   size_t order = 0;                 // receiver order of the pass (uvw, N ints)
   size_t total = 0;
   long long win_edges = 0;          // edges per position-gradient staging window
+  size_t cursor = 0;                // per-node cursor of the window sums (N ints)
   bool has_gbuf = false, has_part = false;
 };
 
@@ -275,6 +276,8 @@ Layout make_layout(const tpconv_plan* P, long long N, long long E, uint32_t pass
     L.gbuf = off;
     L.win_edges = (long long)(stage / 16);
     off += align256(stage);
+    L.cursor = off;                 // per-node position in the source view (N ints)
+    off += align256(size_t(4) * std::max<long long>(N, 1));
   }
   L.total = off;
   return L;
@@ -520,7 +523,7 @@ tpconv_status tpconv_plan_set_layout(tpconv_plan_t P, int32_t layout) {
 
 tpconv_status tpconv_plan_set_math(tpconv_plan_t P, int32_t math) {
   if (!P) return TPCONV_ERR_INVALID_ARG;
-  if (math != TPCONV_MATH_FP32 && math != TPCONV_MATH_TF32) return TPCONV_ERR_UNSUPPORTED;
+  if (math != TPCONV_MATH_FP32 && math != TPCONV_MATH_TF32 && math != TPCONV_MATH_BF16) return TPCONV_ERR_UNSUPPORTED;
   P->math = math;
   return TPCONV_OK;
 }
@@ -870,11 +873,13 @@ static tpconv_status backward_ir_mul(tpconv_plan_t P, int64_t N, int64_t E, cons
   if (P->mode == TPCONV_UVU) {
     if (grad_pos) {
       TPC_TRY(cudaMemsetAsync(grad_pos, 0, sizeof(float) * 3 * (size_t)N, s));
+      int* cursor = reinterpret_cast<int*>(static_cast<char*>(ws) + L.cursor);
+      TPC_TRY(cudaMemcpyAsync(cursor, t_ptr, sizeof(int) * (size_t)N, cudaMemcpyDeviceToDevice, s));
       for (int w = 0; w < windows_per_range(E, L.win_edges); ++w) {
         const EdgeWindow win{0, n, w, L.win_edges};
         TPC_RUN(PC_UVU_RECV_BWD, 1, launch_uvu_recv_bwd(P->dev, P->t_in, x, pos, row_ptr, src, W, grad_out, n, gbuf,
                                                         win, edge_split, s));
-        TPC_RUN(PC_POS, 1, launch_pos_window(n, row_ptr, t_ptr, t_eid, gbuf, win, grad_pos, s));
+        TPC_RUN(PC_POS, 1, launch_pos_window(n, row_ptr, t_ptr, t_eid, gbuf, win, cursor, grad_pos, s));
       }
     }
     if (grad_W) {
@@ -894,6 +899,8 @@ static tpconv_status backward_ir_mul(tpconv_plan_t P, int64_t N, int64_t E, cons
     DevPlan D = P->dev;
     TPC_RUN(PC_UVW_RECV_BWD, 1, attach_order(D, L, ws, n, row_ptr, s));
     TPC_TRY(cudaMemsetAsync(grad_pos, 0, sizeof(float) * 3 * (size_t)N, s));
+    int* cursor = reinterpret_cast<int*>(static_cast<char*>(ws) + L.cursor);
+    TPC_TRY(cudaMemcpyAsync(cursor, t_ptr, sizeof(int) * (size_t)N, cudaMemcpyDeviceToDevice, s));
     for (int n0 = 0; n0 < n; n0 += L.recv_chunk) {
       const int cn = std::min(L.recv_chunk, n - n0);
       TPC_RUN(PC_GEMM, 0, gemm_sbar(P, grad_out, W, state, n0, cn, s));
@@ -901,7 +908,7 @@ static tpconv_status backward_ir_mul(tpconv_plan_t P, int64_t N, int64_t E, cons
         const EdgeWindow win{n0, cn, w, L.win_edges};
         TPC_RUN(PC_UVW_RECV_BWD, 1, launch_uvw_recv_edge(D, x, pos, row_ptr, src, state, n0, cn, gbuf, win,
                                                          chunk_split(N, E), s));
-        TPC_RUN(PC_POS, 1, launch_pos_window(n, row_ptr, t_ptr, t_eid, gbuf, win, grad_pos, s));
+        TPC_RUN(PC_POS, 1, launch_pos_window(n, row_ptr, t_ptr, t_eid, gbuf, win, cursor, grad_pos, s));
       }
     }
   }
@@ -1070,11 +1077,13 @@ static tpconv_status double_backward_ir_mul(tpconv_plan_t P, int64_t N, int64_t 
     if (grad_pos && any_tan) {
       // the tangent of the first-order position gradient (second derivatives of Y, phi)
       TPC_TRY(cudaMemsetAsync(grad_pos, 0, sizeof(float) * 3 * (size_t)N, s));
+      int* cursor = reinterpret_cast<int*>(static_cast<char*>(ws) + L.cursor);
+      TPC_TRY(cudaMemcpyAsync(cursor, t_ptr, sizeof(int) * (size_t)N, cudaMemcpyDeviceToDevice, s));
       for (int w = 0; w < windows_per_range(E, L.win_edges); ++w) {
         const EdgeWindow win{0, n, w, L.win_edges};
         TPC_RUN(PC_RECV_TAN, 1, launch_uvu_recv_dbl(P->dev, P->t_in, x, gg_x, pos, gg_pos, row_ptr, src, W, gg_W,
                                                    grad_out, n, gbuf, win, edge_split, s));
-        TPC_RUN(PC_POS, 1, launch_pos_window(n, row_ptr, t_ptr, t_eid, gbuf, win, grad_pos, s));
+        TPC_RUN(PC_POS, 1, launch_pos_window(n, row_ptr, t_ptr, t_eid, gbuf, win, cursor, grad_pos, s));
       }
     }
     return TPCONV_OK;
@@ -1121,6 +1130,8 @@ static tpconv_status double_backward_ir_mul(tpconv_plan_t P, int64_t N, int64_t 
     DevPlan D = P->dev;
     TPC_RUN(PC_RECV_TAN, 1, attach_order(D, L, ws, n, row_ptr, s));
     TPC_TRY(cudaMemsetAsync(grad_pos, 0, sizeof(float) * 3 * (size_t)N, s));
+    int* cursor = reinterpret_cast<int*>(static_cast<char*>(ws) + L.cursor);
+    TPC_TRY(cudaMemcpyAsync(cursor, t_ptr, sizeof(int) * (size_t)N, cudaMemcpyDeviceToDevice, s));
     for (int n0 = 0; n0 < n; n0 += L.recv_chunk) {
       const int cn = std::min(L.recv_chunk, n - n0);
       TPC_RUN(PC_GEMM, 0, gemm_sbar(P, grad_out, W, sa, n0, cn, s));
@@ -1129,7 +1140,7 @@ static tpconv_status double_backward_ir_mul(tpconv_plan_t P, int64_t N, int64_t 
         const EdgeWindow win{n0, cn, w, L.win_edges};
         TPC_RUN(PC_RECV_TAN, 1, launch_uvw_recv_dbl(D, P->t_in, x, gg_x, pos, gg_pos, row_ptr, src, sa,
                                                    gg_W ? sb : nullptr, n0, cn, gbuf, win, edge_split, s));
-        TPC_RUN(PC_POS, 1, launch_pos_window(n, row_ptr, t_ptr, t_eid, gbuf, win, grad_pos, s));
+        TPC_RUN(PC_POS, 1, launch_pos_window(n, row_ptr, t_ptr, t_eid, gbuf, win, cursor, grad_pos, s));
       }
     }
   }

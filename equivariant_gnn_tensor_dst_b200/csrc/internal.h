@@ -119,7 +119,7 @@ struct GemmProblem {
 
 struct GemmBatch {
   int n_problems, n_segs, splits, total_tiles, accumulate;
-  int math;                      // TPCONV_MATH_FP32 (3xTF32) or TPCONV_MATH_TF32 (one TF32 product)
+  int math;                      // TPCONV_MATH_FP32 (3xTF32), _TF32 (one TF32 product) or _BF16
   float* partial;
   GemmProblem pr[MAX_GEMM_PROBLEMS];
   GemmSeg sg[MAX_GEMM_SEGS];

@@ -10,7 +10,9 @@
 // a = hi + lo with hi = a truncated to TF32 and lo = a - hi; each k-step
 // issues hi*hi + hi*lo + lo*hi into the same fp32 accumulator ("3xTF32", the
 // decomposition of Ootomo and Yokota, 2022), which keeps the relative error near
-// 2^-21 instead of TF32's 2^-11.  The optional TF32 mode issues hi*hi only.
+// 2^-21 instead of TF32's 2^-11.  The optional TF32 mode issues hi*hi only; the optional
+// BF16 mode rounds both operands to bf16 and issues one kind::f16 product per K=16 step
+// (relative error near 2^-9).
 //
 // Structure: one CTA of 288 threads per 128 x NT output tile (NT = 64 or 128) and
 // split-K slice, two CTAs per SM, warp-specialised around two rings: raw stages of 32 k
@@ -78,6 +80,21 @@ __host__ __device__ constexpr uint32_t instr_desc() {
   // D fp32 (bits 4-5 = 1), A and B tf32 (bits 7-9, 10-12 = 2), both K-major,
   // N >> 3 at bits 17-22, M >> 4 at bits 24-28
   return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(NT >> 3) << 17) | ((uint32_t)(TC_M >> 4) << 24);
+}
+
+template <int NT>
+__host__ __device__ constexpr uint32_t instr_desc_bf16() {
+  // kind::f16 with D fp32 (bits 4-5 = 1), A and B both bf16 (bits 7-9, 10-12 = 1), both
+  // K-major, N >> 3 at bits 17-22, M >> 4 at bits 24-28
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(NT >> 3) << 17) | ((uint32_t)(TC_M >> 4) << 24);
+}
+
+// Two floats rounded to bf16 (nearest even) and packed: the first in the low half, the
+// lower k index of an A operand pair in a TMEM cell, of a B pair in shared memory.
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 // Bounded wait for the completion of an mbarrier phase.  SLEEP_NS > 0 backs off between
@@ -266,7 +283,9 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
   const uint32_t tmem = *tmem_slot;
 
   constexpr uint32_t IDESC = instr_desc<NT>();
+  constexpr uint32_t IDESC_BF16 = instr_desc_bf16<NT>();
   const bool tf32 = g.math == TPCONV_MATH_TF32;  // one TF32 product per term, no residuals
+  const bool bf16 = g.math == TPCONV_MATH_BF16;  // operands rounded to bf16, one product
   constexpr int KWB = TC_K / (TC_PRODUCERS / NT);    // k values per producer for the B operand
   bool ok = true;
 
@@ -410,9 +429,33 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
       // have completed
       if (it >= SM::NS) ok = mbar_wait(smem_u32(&mdone[os]), ((it / SM::NS) - 1) & 1) && ok;
       const uint32_t acol = (uint32_t)(NT + 64 * os);
+      if (bf16) {
+        // the 32 A values of this row as bf16 pairs, k and k + 1 in one TMEM cell
+        uint32_t pk[16];
+#pragma unroll
+        for (int k2 = 0; k2 < 16; ++k2) {
+          float v0, v1;
+          if (mm) {
+            const float* a = reinterpret_cast<const float*>(st);
+            v0 = a[(2 * k2) * 128 + m];
+            v1 = a[(2 * k2 + 1) * 128 + m];
+          } else {
+            const float2 v = *reinterpret_cast<const float2*>(st + km_off(m, k2 >> 1) + (k2 & 1) * 8);
+            v0 = v.x;
+            v1 = v.y;
+          }
+          pk[k2] = pack_bf16(v0, v1);
+        }
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+                tlane + acol),
+            "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3]), "r"(pk[4]), "r"(pk[5]), "r"(pk[6]), "r"(pk[7]),
+            "r"(pk[8]), "r"(pk[9]), "r"(pk[10]), "r"(pk[11]), "r"(pk[12]), "r"(pk[13]), "r"(pk[14]), "r"(pk[15])
+            : "memory");
+      }
       // two halves of 16 k values: split, then store hi and lo to this thread's TMEM lane
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      for (int h = 0; h < (bf16 ? 0 : 2); ++h) {
         uint32_t hi[16], lo[16];
         if (mm) {
           const float* a = reinterpret_cast<const float*>(st);
@@ -453,7 +496,18 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
       const char* braw = st + SM::A_BYTES;
       char* bhi = ops + os * 2 * SM::B_BYTES;
       char* blo = bhi + SM::B_BYTES;
-      if (tf32) {
+      if (bf16) {
+        // 16-byte raw chunk = 4 consecutive k of one row (core column k / 4 of the fp32
+        // layout) -> 8 bytes of the 16-bit K-major layout (core column k / 8, LBO and SBO
+        // as for fp32)
+#pragma unroll
+        for (int q = c; q < SM::B_BYTES / 16; q += TC_CONVERTERS) {
+          const float4 v = *reinterpret_cast<const float4*>(braw + q * 16);
+          const int kc4 = (q * 16) / (NT * 16), rem = (q * 16) - kc4 * (NT * 16);
+          const int dst = (kc4 >> 1) * (NT * 16) + rem + (kc4 & 1) * 8;
+          *reinterpret_cast<uint2*>(bhi + dst) = make_uint2(pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
+        }
+      } else if (tf32) {
 #pragma unroll
         for (int q = c; q < SM::B_BYTES / 16; q += TC_CONVERTERS)
           *reinterpret_cast<float4*>(bhi + q * 16) = *reinterpret_cast<const float4*>(braw + q * 16);
@@ -484,7 +538,25 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
       const int os = it % SM::NS;
       ok = mbar_wait(smem_u32(&conv[os]), (it / SM::NS) & 1) && ok;
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      if (lane == 0) {
+      if (lane == 0 && bf16) {
+        // two K=16 steps of bf16: 8 TMEM columns of A (two k per cell), two 8-wide k
+        // columns of B
+        const uint32_t b_hi = smem_u32(ops + os * 2 * SM::B_BYTES);
+        const uint32_t acol = (uint32_t)(NT + 64 * os);
+#pragma unroll
+        for (int ks = 0; ks < TC_K / 16; ++ks) {
+          const uint32_t aaddr = tmem + acol + 8 * ks;
+          const uint64_t db = smem_desc<NT>(b_hi + ks * 2 * (NT * 16));
+          const uint32_t acc0 = (it > 0 || ks > 0) ? 1u : 0u;
+          asm volatile(
+              "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+              "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem),
+              "r"(aaddr), "l"(db), "r"(IDESC_BF16), "r"(acc0));
+        }
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                         smem_u32(&mdone[os]))
+                     : "memory");
+      } else if (lane == 0) {
         const uint32_t b_hi = smem_u32(ops + os * 2 * SM::B_BYTES), b_lo = b_hi + SM::B_BYTES;
         const uint32_t acol = (uint32_t)(NT + 64 * os);
 #pragma unroll

@@ -3,7 +3,7 @@
 //
 //  * k_pos_window -- position gradient: pos_bar[n] = sum_{e out of n} g_e
 //    - sum_{e into n} g_e, one bounded staging window of g_e at a time, in source-CSR
-//    and receiver-CSR order (no atomics).
+//    and receiver-CSR order (no atomics; a per-node cursor walks the source rows).
 //  * CSR transpose (stable counting sort by source) and the graph validator.
 #include <cuda_runtime.h>
 #include <mutex>
@@ -57,13 +57,15 @@ cudaError_t launch_reduce_partials(const float* partial, int n_parts, long long 
 }
 
 // One staging window [w0, w1) of g_e (stored at gbuf[e - w0]): every node adds the g_e of
-// its outgoing edges inside the window (source view order: t_eid is increasing within a
-// source, so they are one contiguous run, found by binary search) and subtracts those of
-// its incoming edges inside the window (a sub-range of its receiver row).  Windows are
-// applied in a fixed order, so the sums are deterministic.
+// its outgoing edges inside the window and subtracts those of its incoming edges inside
+// the window (a sub-range of its receiver row).  The windows of a pass cover the edge ids
+// in increasing order, and t_eid is increasing within a source, so a node's outgoing
+// edges in the window are the next run of its t_eid row: cursor[n] (initialised to
+// t_ptr[n]) marks where the run starts and is advanced past it.  Windows are applied in
+// a fixed order, so the sums are deterministic.
 __global__ void k_pos_window(int N, const int* __restrict__ row_ptr, const int* __restrict__ t_ptr,
                              const int* __restrict__ t_eid, const float4* __restrict__ gbuf, EdgeWindow win,
-                             float* grad_pos) {
+                             int* cursor, float* grad_pos) {
   const long long lo = __ldg(row_ptr + win.n0), hi = __ldg(row_ptr + win.n0 + win.n_nodes);
   const long long a = lo + (long long)win.index * win.size;
   const int w0 = (int)min(a, hi), w1 = (int)min(a + win.size, hi);
@@ -71,20 +73,17 @@ __global__ void k_pos_window(int N, const int* __restrict__ row_ptr, const int* 
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
   if (n >= N) return;
   float x = 0.f, y = 0.f, z = 0.f;
-  int k0 = __ldg(t_ptr + n), k1 = __ldg(t_ptr + n + 1);
-  // first k with t_eid[k] >= w0
-  while (k0 < k1) {
-    const int mid = (k0 + k1) >> 1;
-    if (__ldg(t_eid + mid) < w0) k0 = mid + 1; else k1 = mid;
-  }
   bool touched = false;
-  for (int k = k0, kend = __ldg(t_ptr + n + 1); k < kend; ++k) {
+  const int kend = __ldg(t_ptr + n + 1);
+  int k = cursor[n];
+  for (; k < kend; ++k) {
     const int e = __ldg(t_eid + k);
     if (e >= w1) break;
     const float4 g = gbuf[e - w0];
     x += g.x; y += g.y; z += g.z;
     touched = true;
   }
+  if (touched) cursor[n] = k;
   const int eb = max(__ldg(row_ptr + n), w0), ee = min(__ldg(row_ptr + n + 1), w1);
   for (int e = eb; e < ee; ++e) {
     const float4 g = gbuf[e - w0];
@@ -99,9 +98,9 @@ __global__ void k_pos_window(int N, const int* __restrict__ row_ptr, const int* 
 }
 
 cudaError_t launch_pos_window(int N, const int* row_ptr, const int* t_ptr, const int* t_eid,
-                              const float4* gbuf, EdgeWindow win, float* grad_pos, cudaStream_t s) {
+                              const float4* gbuf, EdgeWindow win, int* cursor, float* grad_pos, cudaStream_t s) {
   if (N <= 0) return cudaSuccess;
-  k_pos_window<<<(N + 255) / 256, 256, 0, s>>>(N, row_ptr, t_ptr, t_eid, gbuf, win, grad_pos);
+  k_pos_window<<<(N + 255) / 256, 256, 0, s>>>(N, row_ptr, t_ptr, t_eid, gbuf, win, cursor, grad_pos);
   return cudaGetLastError();
 }
 

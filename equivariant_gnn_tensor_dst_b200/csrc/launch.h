@@ -103,9 +103,10 @@ cudaError_t launch_uvu_src(const DevPlan& P, const BlockPaths& BP, const Tasks& 
                            cudaStream_t s);
 cudaError_t launch_reduce_partials(const float* partial, int n_parts, long long n, float* out,
                                    int accumulate, cudaStream_t s);
-// grad_pos[n] += sum_{e out of n, e in win} g_e - sum_{e into n, e in win} g_e
+// grad_pos[n] += sum_{e out of n, e in win} g_e - sum_{e into n, e in win} g_e; cursor [N]
+// starts as a copy of t_ptr and is advanced window by window
 cudaError_t launch_pos_window(int N, const int* row_ptr, const int* t_ptr, const int* t_eid,
-                              const float4* gbuf, EdgeWindow win, float* grad_pos, cudaStream_t s);
+                              const float4* gbuf, EdgeWindow win, int* cursor, float* grad_pos, cudaStream_t s);
 cudaError_t launch_csr_transpose(int N, int E, const int* row_ptr, const int* src, int* t_ptr,
                                  int* t_eid, int* t_dst, int* cursor, cudaStream_t s);
 cudaError_t launch_degree_order(int N, const int* row_ptr, int chunk, int* order, cudaStream_t s);

@@ -140,10 +140,13 @@ tpconv_status tpconv_set_workspace_budget(tpconv_plan_t plan, size_t bytes);
  *     per term (hi*hi + hi*lo + lo*hi); results match fp32 to about 1e-6 relative.
  *   TPCONV_MATH_TF32: one TF32 product per term (operands truncated to 10 mantissa
  *     bits); about 1e-3 relative error, faster contractions.
- * The streaming (edge) arithmetic is fp32 in both modes.  Any other value returns
+ *   TPCONV_MATH_BF16: both operands rounded to bf16 (8 mantissa bits), one bf16
+ *     tensor-core product per term with fp32 accumulation; about 3e-3 relative error.
+ * The streaming (edge) arithmetic is fp32 in every mode.  Any other value returns
  * TPCONV_ERR_UNSUPPORTED and leaves the plan unchanged.                             */
 #define TPCONV_MATH_FP32 0
 #define TPCONV_MATH_TF32 1
+#define TPCONV_MATH_BF16 2
 tpconv_status tpconv_plan_set_math(tpconv_plan_t plan, int32_t math);
 
 /* Boundary layout of the node arrays x, out, grad_out, gg_x, grad_x and grad_grad_out
@@ -165,7 +168,8 @@ tpconv_status tpconv_plan_set_layout(tpconv_plan_t plan, int32_t layout);
  * range, the split-K slices of the channel contractions and, in backward and double
  * backward, a staging window for the per-edge position gradients (an eighth of the
  * budget, at most 16 MiB; the edges are staged window by window) all fit the scratch
- * budget (tpconv_set_workspace_budget), plus 4 bytes per node of receiver order.       */
+ * budget (tpconv_set_workspace_budget), plus 8 bytes per node (receiver order; cursors
+ * into the source view for the position sums).                                         */
 tpconv_status tpconv_workspace_bytes(tpconv_plan_t plan, int64_t N, int64_t E,
                                      uint32_t pass_mask, size_t* bytes);
 

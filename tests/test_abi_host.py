@@ -125,7 +125,7 @@ def test_workspace_is_bounded_and_independent_of_edges():
         ws = [lp.workspace_bytes(4096, 4096 * k, mask) for k in (8, 16, 32, 64, 128)]
         ws.append(lp.workspace_bytes(4096, 50_000_000, mask))
         assert len(set(ws)) == 1
-        assert ws[0] <= (128 << 20) + 4 * 4096 + 4096
+        assert ws[0] <= (128 << 20) + 8 * 4096 + 4096   # + receiver order and source cursor
 
 
 def test_forward_rejects_bad_arguments_before_launch():
@@ -192,6 +192,7 @@ def test_plan_set_math_arguments():
     L = binding.lib()
     p = binding.Plan("8x0e+8x1o", 2, "8x0e+8x1o", "uvw", "bessel", 8, 3.0)
     assert L.tpconv_plan_set_math(p.handle, binding.MATH_TF32) == 0
+    assert L.tpconv_plan_set_math(p.handle, binding.MATH_BF16) == 0
     assert L.tpconv_plan_set_math(p.handle, binding.MATH_FP32) == 0
     assert L.tpconv_plan_set_math(p.handle, 7) == 3          # TPCONV_ERR_UNSUPPORTED
     assert L.tpconv_plan_set_math(None, binding.MATH_FP32) == 1   # TPCONV_ERR_INVALID_ARG
