@@ -1,8 +1,9 @@
 """Real spherical harmonics and real Clebsch-Gordan coupling tensors (oracle side).
 
-The pages only say that Y_ij "contains spherical harmonics of r_hat_ij" (Sobek,
-section 2, after eq. 8) and that c^pi "contains the path normalization and sparse
-Clebsch-Gordan coefficient" (section 4, eq. 32).  The readings taken here:
+The pages build Y_ij from spherical harmonics of the edge direction (Sobek, section 2,
+after eq. 8) and let c^pi carry both a path normalisation and the sparse Clebsch-Gordan
+coefficients (section 4, eq. 32), but fix neither the basis nor the normalisation.  The
+readings taken here:
 
 * Real SH, z polar axis, no Condon-Shortley phase, component normalisation
   (sum_m Y_lm^2 = 2l+1).  For m >= 0
