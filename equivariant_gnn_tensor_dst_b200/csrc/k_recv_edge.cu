@@ -97,7 +97,7 @@ __device__ __forceinline__ void recv_edge_piece(const DevPlan& P, const DevPath&
   float ybl[RS];
 #pragma unroll
   for (int k = 0; k < RS; ++k) ybl[k] = 0.f;
-#pragma unroll 2
+#pragma unroll 1
   for (int cc = 0; cc < cw; cc += U) {
     float xv[U][RI];
 #pragma unroll
@@ -180,10 +180,10 @@ __device__ __forceinline__ bool next_piece(const DevPlan& P, int w, int& pi, int
 }
 
 // Grid: CTAs enumerate (receiver slot, share); share s of a receiver takes its 32-edge
-// chunks s, s + split, ...  Three CTAs per SM for K <= 8, two for K <= 16 (its
+// chunks s, s + split, ...  Four CTAs per SM for K <= 8, three for K <= 16 (its
 // accumulators need more registers).
 template <int KP, bool FAST>
-__global__ void __launch_bounds__(128, KP == 8 ? 3 : 2)
+__global__ void __launch_bounds__(128, KP == 8 ? 4 : 3)
     k_uvw_recv_edge(DevPlan P, const float* __restrict__ x, const float* __restrict__ pos,
                     const int* __restrict__ row_ptr, const int* __restrict__ src, const float* __restrict__ Sbar,
                     int node0, int n_nodes, float4* gbuf, EdgeWindow win, int split) {
