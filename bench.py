@@ -43,9 +43,15 @@ L2_FLUSH_BYTES = 256 << 20                          # > 126 MB L2
 TF32_PER_BF16 = 1.1 / 2.25                          # nominal dense TF32 / BF16 tensor rates
 SPLIT_MMAS = 3                                      # 3xTF32: three TF32 products per fp32 product
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per step for a kernel category
-# of the step's workload, from an ncu capture of the kernels as they are now (scaled from
-# the captured case by the edges processed).  None: no capture of the current kernels.
-TRAFFIC_BYTES_PER_STEP = {}
+# of the step's workload, from an ncu capture of the current kernels on the N=8000 resize of
+# the workload, scaled by its edge ratio (2 800 256 / 433 220); profiles/
+# edge_scaling_N8000_dram_traffic.md.
+TRAFFIC_BYTES_PER_STEP = {
+    "uvw_receiver_backward": 10.98e9,
+    "uvw_receiver_state": 6.41e9,
+    "uvw_source_state": 4.49e9,
+    "channel_gemm": 29.91e9,
+}
 
 
 def measured_peaks():
@@ -351,7 +357,8 @@ def run_native(args):
         tb = TRAFFIC_BYTES_PER_STEP.get(k) if headline else None
         rl["traffic"] = round(tb) if tb else None
         if tb:
-            rl["traffic_note"] = "DRAM bytes per step (all launches of the category), ncu capture"
+            rl["traffic_note"] = ("DRAM bytes per step (all launches of the category), ncu capture of the N=8000 "
+                                  "resize scaled by the edge ratio")
         rooflines[k] = rl
     dom = max(rooflines, key=lambda k: kern[k][0]) if rooflines else None
     roofline = dict(rooflines[dom], kernel=dom) if dom else None
