@@ -601,12 +601,16 @@ def run_extras(args, dev, flush):
         rec["embedded_interface"] = {"forward_ms": round(ms_ef, 4), "backward_ms": round(ms_eb, 4),
                                      "forward_backward_edges_per_s": round(E / (ms_ef + ms_eb) * 1e3, 1)}
         if c.mode == "uvw":
-            # the optional TF32 contraction mode (1e-2 accuracy class), reported separately
+            # the optional TF32 and BF16 contraction modes (1e-2 accuracy class), reported separately
             plan.set_math(binding.MATH_TF32)
             ms_tf, ms_tb = _timed(fwd, flush, steps, warm), _timed(bwd, flush, steps, warm)
+            plan.set_math(binding.MATH_BF16)
+            ms_bf, ms_bb = _timed(fwd, flush, steps, warm), _timed(bwd, flush, steps, warm)
             plan.set_math(binding.MATH_FP32)
             rec["tf32_contractions"] = {"forward_ms": round(ms_tf, 4), "backward_ms": round(ms_tb, 4),
                                         "forward_backward_edges_per_s": round(E / (ms_tf + ms_tb) * 1e3, 1)}
+            rec["bf16_contractions"] = {"forward_ms": round(ms_bf, 4), "backward_ms": round(ms_bb, 4),
+                                        "forward_backward_edges_per_s": round(E / (ms_bf + ms_bb) * 1e3, 1)}
         if "dbl" in c.passes:
             # force training: energy = sum of scalar outputs, F = -dE/dpos, loss |F - F_ref|^2,
             # then d loss / d(W, x) by the double backward

@@ -185,6 +185,25 @@ __device__ __forceinline__ void envelope(const DevPlan& P, float t, float& u, fl
   du = -P.env_a * p * tpm1 + P.env_b * (p + 1.f) * tp - P.env_c * (p + 2.f) * tp1;
 }
 
+// sin(b pi t) and cos(b pi t) for b = 1..KP from one sincospif: the three-term recurrence
+// sin((b+1)a) = 2 cos(a) sin(b a) - sin((b-1)a) (and the same for cos), exact in exact
+// arithmetic; in fp32 its absolute error grows like b^2 times the rounding of cos(a): below
+// 3e-6 for b <= 8 and 1.1e-5 for b <= 16 on t in (0, 1) (values bounded by 1).
+template <int KP>
+__device__ __forceinline__ void sincos_multiples(float t, float* sn, float* cs) {
+  float s1, c1;
+  sincospif(t, &s1, &c1);
+  const float two_c = 2.f * c1;
+  float sp = 0.f, cp = 1.f, sc = s1, cc = c1;   // b - 1 and b
+#pragma unroll
+  for (int q = 0; q < KP; ++q) {
+    sn[q] = sc;
+    cs[q] = cc;
+    const float sn1 = fmaf(two_c, sc, -sp), cn1 = fmaf(two_c, cc, -cp);
+    sp = sc; cp = cc; sc = sn1; cc = cn1;
+  }
+}
+
 template <int KP, bool DERIV>
 __device__ __forceinline__ void radial(const DevPlan& P, float d, float* phi, float* dphi) {
   const float t = d * P.inv_r_cut;
@@ -193,14 +212,15 @@ __device__ __forceinline__ void radial(const DevPlan& P, float d, float* phi, fl
   du *= P.inv_r_cut;  // d u / d d
   if (P.radial_kind == 0) {
     const float inv_d = d > 0.f ? 1.f / d : 0.f;
+    float sn[KP], cs[KP];
+    sincos_multiples<KP>(t, sn, cs);
 #pragma unroll
     for (int q = 0; q < KP; ++q) {
       float f = 0.f, df = 0.f;
       if (q < P.K && u != 0.f) {
         const float b = (float)(q + 1);
         if (d > 0.f) {
-          float s, c;
-          sincospif(b * t, &s, &c);
+          const float s = sn[q], c = cs[q];
           const float base = P.bessel_pref * s * inv_d;  // sqrt(2/rc) sin(b pi t)/d
           f = base * u;
           if (DERIV) {
@@ -254,6 +274,8 @@ __device__ __forceinline__ void radial2(const DevPlan& P, float d, float* phi, f
   ddu *= P.inv_r_cut * P.inv_r_cut;
   if (P.radial_kind == 0) {
     const float inv_d = d > 0.f ? 1.f / d : 0.f;
+    float sn[KP], cs[KP];
+    sincos_multiples<KP>(t, sn, cs);
 #pragma unroll
     for (int q = 0; q < KP; ++q) {
       float f = 0.f, df = 0.f, d2f = 0.f;
@@ -261,8 +283,7 @@ __device__ __forceinline__ void radial2(const DevPlan& P, float d, float* phi, f
         const float b = (float)(q + 1);
         const float k = b * 3.14159265358979f * P.inv_r_cut;
         if (d > 0.f) {
-          float s, c;
-          sincospif(b * t, &s, &c);
+          const float s = sn[q], c = cs[q];
           const float base = P.bessel_pref * s * inv_d;
           const float g1 = (k * c - s * inv_d) * inv_d;   // d/dd of sin(kd)/d
           const float dbase = P.bessel_pref * g1;
