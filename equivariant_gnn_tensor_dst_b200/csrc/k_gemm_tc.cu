@@ -260,6 +260,12 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
   const int split = blockIdx.y;
   const int kper = ((P.Ktot + g.splits - 1) / g.splits + TC_K - 1) / TC_K * TC_K;
   const int kb = split * kper, ke = min(P.Ktot, kb + kper);
+  // Width of the products of this tile: its valid columns rounded up to a multiple of 32
+  // (the narrowest width in use), so that the narrow output blocks of a plan (16 or 32
+  // channels) do not pay for full-width products, B copies and B splits.  B rows at or
+  // beyond `neff` are neither copied nor split (the products do not read them), and the
+  // accumulator columns beyond it are neither written nor read.
+  const int neff = min(NT, (min(NT, P.N - n0) + 31) & ~31);
 
   if (tid == 0) {
     for (int i = 0; i < SM::RR; ++i) {
@@ -282,8 +288,9 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = *tmem_slot;
 
-  constexpr uint32_t IDESC = instr_desc<NT>();
-  constexpr uint32_t IDESC_BF16 = instr_desc_bf16<NT>();
+  // instruction descriptors with the tile's product width in the N field (bits 17-22)
+  const uint32_t IDESC = (instr_desc<NT>() & ~(0x3Fu << 17)) | ((uint32_t)(neff >> 3) << 17);
+  const uint32_t IDESC_BF16 = (instr_desc_bf16<NT>() & ~(0x3Fu << 17)) | ((uint32_t)(neff >> 3) << 17);
   const bool tf32 = g.math == TPCONV_MATH_TF32;  // one TF32 product per term, no residuals
   const bool bf16 = g.math == TPCONV_MATH_BF16;  // operands rounded to bf16, one product
   constexpr int KWB = TC_K / (TC_PRODUCERS / NT);    // k values per producer for the B operand
@@ -396,7 +403,7 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
           kstep(q2, r2, a_d, 1);
         }
       }
-      issue_operand<KWB, NT>(cb, S.B, kt, khi, kbegB, rowB, S.b_vec4 != 0, dB);
+      if (rowB < neff) issue_operand<KWB, NT>(cb, S.B, kt, khi, kbegB, rowB, S.b_vec4 != 0, dB);
       // the stage's full barrier completes when this thread's copies (and its earlier
       // ones) have landed; nothing the copies write is read by the tensor core directly
       asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&full[slot])) : "memory");
@@ -496,30 +503,36 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
       const char* braw = st + SM::A_BYTES;
       char* bhi = ops + os * 2 * SM::B_BYTES;
       char* blo = bhi + SM::B_BYTES;
+      // 16-byte chunk q of the rows below neff: 4 consecutive k (core column kc4) of one row
+      // (neff is 32, 64 or 128 for every plan whose blocks have at most 128 channels: a
+      // shift; otherwise a division)
+      const int nsh = (neff & (neff - 1)) == 0 ? __ffs(neff) - 1 : -1;
       if (bf16) {
-        // 16-byte raw chunk = 4 consecutive k of one row (core column k / 4 of the fp32
-        // layout) -> 8 bytes of the 16-bit K-major layout (core column k / 8, LBO and SBO
-        // as for fp32)
-#pragma unroll
-        for (int q = c; q < SM::B_BYTES / 16; q += TC_CONVERTERS) {
-          const float4 v = *reinterpret_cast<const float4*>(braw + q * 16);
-          const int kc4 = (q * 16) / (NT * 16), rem = (q * 16) - kc4 * (NT * 16);
-          const int dst = (kc4 >> 1) * (NT * 16) + rem + (kc4 & 1) * 8;
+        // fp32 core column kc4 -> 8 bytes of the 16-bit K-major layout (core column kc4 / 2,
+        // LBO and SBO as for fp32)
+        for (int q = c; q < 8 * neff; q += TC_CONVERTERS) {
+          const int kc4 = nsh >= 0 ? q >> nsh : q / neff, row = q - kc4 * neff;
+          const int off = kc4 * (NT * 16) + row * 16;
+          const float4 v = *reinterpret_cast<const float4*>(braw + off);
+          const int dst = (kc4 >> 1) * (NT * 16) + row * 16 + (kc4 & 1) * 8;
           *reinterpret_cast<uint2*>(bhi + dst) = make_uint2(pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
         }
       } else if (tf32) {
-#pragma unroll
-        for (int q = c; q < SM::B_BYTES / 16; q += TC_CONVERTERS)
-          *reinterpret_cast<float4*>(bhi + q * 16) = *reinterpret_cast<const float4*>(braw + q * 16);
+        for (int q = c; q < 8 * neff; q += TC_CONVERTERS) {
+          const int kc4 = nsh >= 0 ? q >> nsh : q / neff, row = q - kc4 * neff;
+          const int off = kc4 * (NT * 16) + row * 16;
+          *reinterpret_cast<float4*>(bhi + off) = *reinterpret_cast<const float4*>(braw + off);
+        }
       } else {
-#pragma unroll
-        for (int q = c; q < SM::B_BYTES / 16; q += TC_CONVERTERS) {
-          const float4 v = *reinterpret_cast<const float4*>(braw + q * 16);
+        for (int q = c; q < 8 * neff; q += TC_CONVERTERS) {
+          const int kc4 = nsh >= 0 ? q >> nsh : q / neff, row = q - kc4 * neff;
+          const int off = kc4 * (NT * 16) + row * 16;
+          const float4 v = *reinterpret_cast<const float4*>(braw + off);
           float4 h, l;
           h.x = tf32_hi(v.x); h.y = tf32_hi(v.y); h.z = tf32_hi(v.z); h.w = tf32_hi(v.w);
           l.x = v.x - h.x; l.y = v.y - h.y; l.z = v.z - h.z; l.w = v.w - h.w;
-          *reinterpret_cast<float4*>(bhi + q * 16) = h;
-          *reinterpret_cast<float4*>(blo + q * 16) = l;
+          *reinterpret_cast<float4*>(bhi + off) = h;
+          *reinterpret_cast<float4*>(blo + off) = l;
         }
       }
       // every value read from the raw stage has been used: the producers may refill it
@@ -622,7 +635,7 @@ __global__ void __launch_bounds__(TC_THREADS, 2) k_gemm_tc(const __grid_constant
   const int quad = warp & 3, half = warp >> 2;
   const bool epi = warp < 8;                             // the MMA warp takes no part
 #pragma unroll 1
-  for (int c0 = 0; c0 < NT; c0 += 64) {
+  for (int c0 = 0; c0 < neff; c0 += 64) {
     uint32_t r[32];
     const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(c0 + half * 32);
     if (epi) asm volatile(
