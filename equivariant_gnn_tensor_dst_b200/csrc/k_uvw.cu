@@ -100,7 +100,10 @@ __device__ __forceinline__ void prep_edge(const DevPlan& P, const float* __restr
 // the KP x R accumulators (and their tangents in MODE 1), or that measured faster.
 #define TPC_MINB_STATE (KP == 8 ? (MODE == 0 ? 5 : 3) : (MODE == 0 ? 3 : 2))
 
-template <int LI, int LS, int LO, int KP, int MODE>
+// SQ (primal pass, paths of at most 16 input channels): the two half-warps take the two
+// halves of the radial index q for the same 16 channels, instead of leaving half of the
+// lanes idle; each lane then keeps KP / 2 accumulators per output component.
+template <int LI, int LS, int LO, int KP, int MODE, bool SQ>
 __device__ __forceinline__ void uvw_state_body(const DevPlan& P, const DevPath& p, int chunk, int i,
                                                int node_local, const float* __restrict__ x,
                                                const float* __restrict__ xdot,
@@ -111,14 +114,17 @@ __device__ __forceinline__ void uvw_state_body(const DevPlan& P, const DevPath& 
                                                GeoSmem<KP, MODE == 1>& sm) {
   constexpr int RI = 2 * LI + 1, RS = 2 * LS + 1, RO = 2 * LO + 1;
   constexpr bool TAN = MODE == 1;
+  static_assert(!(SQ && TAN), "the radial split is for the primal pass");
+  constexpr int KQ = SQ ? KP / 2 : KP;   // radial values per lane
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int u = chunk * 32 + lane;
+  const int q0 = SQ ? (lane >> 4) * KQ : 0;
+  const int u = SQ ? (lane & 15) : chunk * 32 + lane;
   const bool act = u < p.c_in;
   const float* xb = x + p.in_off + (act ? u : 0);
   const float* xdb = xdot ? xdot + p.in_off + (act ? u : 0) : nullptr;
-  float acc[KP][RO], acc0[KP][RO];
+  float acc[KQ][RO], acc0[KQ][RO];
 #pragma unroll
-  for (int q = 0; q < KP; ++q)
+  for (int q = 0; q < KQ; ++q)
 #pragma unroll
     for (int o = 0; o < RO; ++o) { acc[q][o] = 0.f; acc0[q][o] = 0.f; }
 
@@ -152,17 +158,17 @@ __device__ __forceinline__ void uvw_state_body(const DevPlan& P, const DevPath& 
           if (TAN && xdb) xdn[m] = act ? __ldg(xdb + row + m * p.c_in) : 0.f;
         }
       }
-      float phi[KP];
+      float phi[KQ];
 #pragma unroll
-      for (int q = 0; q < KP; q += 4) {
-        const float4 v = reinterpret_cast<const float4*>(sm.phi[w][t])[q / 4];
+      for (int q = 0; q < KQ; q += 4) {
+        const float4 v = reinterpret_cast<const float4*>(sm.phi[w][t] + q0)[q / 4];
         phi[q] = v.x; phi[q + 1] = v.y; phi[q + 2] = v.z; phi[q + 3] = v.w;
       }
       float C[RO];
       cg_couple_cy<LI, LS, LO>(xv, sm.cy[w][t], C);
-      if (!TAN) {
+      if constexpr (!TAN) {
 #pragma unroll
-        for (int q = 0; q < KP; ++q)
+        for (int q = 0; q < KQ; ++q)
 #pragma unroll
           for (int o = 0; o < RO; ++o) acc[q][o] = fmaf(phi[q], C[o], acc[q][o]);
       } else {
@@ -196,14 +202,16 @@ __device__ __forceinline__ void uvw_state_body(const DevPlan& P, const DevPath& 
 #pragma unroll
   for (int o = 0; o < RO; ++o)
 #pragma unroll
-    for (int q = 0; q < KP; ++q)
-      if (q < P.K) out[base + (long long)o * rs + q * p.c_in] = acc[q][o];
-  if (TAN && S) {
+    for (int q = 0; q < KQ; ++q)
+      if (q0 + q < P.K) out[base + (long long)o * rs + (q0 + q) * p.c_in] = acc[q][o];
+  if constexpr (TAN) {
+    if (S) {
 #pragma unroll
-    for (int o = 0; o < RO; ++o)
+      for (int o = 0; o < RO; ++o)
 #pragma unroll
-      for (int q = 0; q < KP; ++q)
-        if (q < P.K) S[base + (long long)o * rs + q * p.c_in] = acc0[q][o];
+        for (int q = 0; q < KP; ++q)
+          if (q < P.K) S[base + (long long)o * rs + q * p.c_in] = acc0[q][o];
+    }
   }
 }
 
@@ -225,10 +233,20 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32, TPC_MINB_STATE)
   const DevPath& p = P.p[T.a[task]];
   const int chunk = T.b[task];
   const int i = node0 + node_local;
+  if constexpr (MODE == 0) {
+    if (p.c_in <= 16) {
+      dispatch_type(p.type, [&](auto tr) {
+        using TR = decltype(tr);
+        uvw_state_body<TR::li, TR::ls, TR::lo, KP, MODE, true>(P, p, chunk, i, node_local, x, xdot, pos,
+                                                               posdot, row_ptr, src, S, Sd, sm);
+      });
+      return;
+    }
+  }
   dispatch_type(p.type, [&](auto tr) {
     using TR = decltype(tr);
-    uvw_state_body<TR::li, TR::ls, TR::lo, KP, MODE>(P, p, chunk, i, node_local, x, xdot, pos,
-                                                     posdot, row_ptr, src, S, Sd, sm);
+    uvw_state_body<TR::li, TR::ls, TR::lo, KP, MODE, false>(P, p, chunk, i, node_local, x, xdot, pos,
+                                                            posdot, row_ptr, src, S, Sd, sm);
   });
 }
 
@@ -236,7 +254,8 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32, TPC_MINB_STATE)
 // source state X (and its tangent for the double backward)
 // ---------------------------------------------------------------------------
 
-template <int LI, int LS, int LO, int KP, int MODE>
+// SQ: as for the receiver state, for paths of at most 16 output channels.
+template <int LI, int LS, int LO, int KP, int MODE, bool SQ>
 __device__ __forceinline__ void uvw_src_body(const DevPlan& P, const DevPath& p, int chunk, int j,
                                              int node_local, const float* __restrict__ pos,
                                              const float* __restrict__ posdot,
@@ -246,13 +265,16 @@ __device__ __forceinline__ void uvw_src_body(const DevPlan& P, const DevPath& p,
                                              GeoSmem<KP, MODE == 1>& sm) {
   constexpr int RI = 2 * LI + 1, RS = 2 * LS + 1, RO = 2 * LO + 1;
   constexpr bool TAN = MODE == 1;
+  static_assert(!(SQ && TAN), "the radial split is for the primal pass");
+  constexpr int KQ = SQ ? KP / 2 : KP;   // radial values per lane
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int c = chunk * 32 + lane;
+  const int q0 = SQ ? (lane >> 4) * KQ : 0;
+  const int c = SQ ? (lane & 15) : chunk * 32 + lane;
   const bool act = c < p.c_out;
   const float* gb = gout + p.out_off + (act ? c : 0);
-  float acc[KP][RI], acc0[KP][RI];
+  float acc[KQ][RI], acc0[KQ][RI];
 #pragma unroll
-  for (int q = 0; q < KP; ++q)
+  for (int q = 0; q < KQ; ++q)
 #pragma unroll
     for (int m = 0; m < RI; ++m) { acc[q][m] = 0.f; acc0[q][m] = 0.f; }
   const int kb = __ldg(t_ptr + j), ke = __ldg(t_ptr + j + 1);
@@ -280,17 +302,17 @@ __device__ __forceinline__ void uvw_src_body(const DevPlan& P, const DevPath& p,
 #pragma unroll
         for (int o = 0; o < RO; ++o) mn[o] = act ? __ldg(gb + row + o * p.c_out) : 0.f;
       }
-      float phi[KP];
+      float phi[KQ];
 #pragma unroll
-      for (int q = 0; q < KP; q += 4) {
-        const float4 v = reinterpret_cast<const float4*>(sm.phi[w][t])[q / 4];
+      for (int q = 0; q < KQ; q += 4) {
+        const float4 v = reinterpret_cast<const float4*>(sm.phi[w][t] + q0)[q / 4];
         phi[q] = v.x; phi[q + 1] = v.y; phi[q + 2] = v.z; phi[q + 3] = v.w;
       }
       float U[RI];
       cg_adj_x_cy<LI, LS, LO>(sm.cy[w][t], mb, U);
-      if (!TAN) {
+      if constexpr (!TAN) {
 #pragma unroll
-        for (int q = 0; q < KP; ++q)
+        for (int q = 0; q < KQ; ++q)
 #pragma unroll
           for (int m = 0; m < RI; ++m) acc[q][m] = fmaf(phi[q], U[m], acc[q][m]);
       } else {
@@ -319,14 +341,16 @@ __device__ __forceinline__ void uvw_src_body(const DevPlan& P, const DevPath& p,
 #pragma unroll
   for (int m = 0; m < RI; ++m)
 #pragma unroll
-    for (int q = 0; q < KP; ++q)
-      if (q < P.K) out[base + (long long)m * rs + q * p.c_out] = acc[q][m];
-  if (TAN && X) {
+    for (int q = 0; q < KQ; ++q)
+      if (q0 + q < P.K) out[base + (long long)m * rs + (q0 + q) * p.c_out] = acc[q][m];
+  if constexpr (TAN) {
+    if (X) {
 #pragma unroll
-    for (int m = 0; m < RI; ++m)
+      for (int m = 0; m < RI; ++m)
 #pragma unroll
-      for (int q = 0; q < KP; ++q)
-        if (q < P.K) X[base + (long long)m * rs + q * p.c_out] = acc0[q][m];
+        for (int q = 0; q < KP; ++q)
+          if (q < P.K) X[base + (long long)m * rs + q * p.c_out] = acc0[q][m];
+    }
   }
 }
 
@@ -347,10 +371,20 @@ __global__ void __launch_bounds__(WARPS_PER_CTA * 32, TPC_MINB_STATE)
   const DevPath& p = P.p[T.a[task]];
   const int chunk = T.b[task];
   const int j = node0 + node_local;
+  if constexpr (MODE == 0) {
+    if (p.c_out <= 16) {
+      dispatch_type(p.type, [&](auto tr) {
+        using TR = decltype(tr);
+        uvw_src_body<TR::li, TR::ls, TR::lo, KP, MODE, true>(P, p, chunk, j, node_local, pos, posdot, t_ptr,
+                                                             t_dst, gout, X, Xd, sm);
+      });
+      return;
+    }
+  }
   dispatch_type(p.type, [&](auto tr) {
     using TR = decltype(tr);
-    uvw_src_body<TR::li, TR::ls, TR::lo, KP, MODE>(P, p, chunk, j, node_local, pos, posdot, t_ptr,
-                                                   t_dst, gout, X, Xd, sm);
+    uvw_src_body<TR::li, TR::ls, TR::lo, KP, MODE, false>(P, p, chunk, j, node_local, pos, posdot, t_ptr,
+                                                          t_dst, gout, X, Xd, sm);
   });
 }
 
