@@ -48,9 +48,11 @@ SPLIT_MMAS = 3                                      # 3xTF32: three TF32 product
 # edge_scaling_N8000_dram_traffic.md.
 TRAFFIC_BYTES_PER_STEP = {
     "uvw_receiver_backward": 10.98e9,
-    "uvw_receiver_state": 6.41e9,
-    "uvw_source_state": 4.49e9,
-    "channel_gemm": 29.91e9,
+    # the receiver state, source state and contraction kernels have changed since that
+    # capture (radial split of the 16-channel paths, per-tile product width): no figure
+    "uvw_receiver_state": None,
+    "uvw_source_state": None,
+    "channel_gemm": None,
 }
 
 
